@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Benchmark of one DDTree tree-verify step on B200s.
+
+A step = ddt_build_tree -> ddt_verify_attn -> ddt_accept_compact (all three
+calls of the C ABI, one stream) over one batch of synthetic Kimi-K2.6-shaped
+inputs. Metric: verified tree nodes per second (whole job), with the verify
+attention's TFLOP/s against the measured bf16 dense peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+N > 1 runs under torch.distributed.run, one process per GPU. Requests are
+independent, so every rank runs its own replica of the workload (weak scaling)
+with no collective on the data path; NCCL only carries the timing barrier and
+the max-over-ranks of the elapsed time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from ddtree_speculative_decode_b200 import synth  # noqa: E402
+
+METRIC = "verified tree-nodes/s per B200; verify-attn TFLOP/s as % of BF16 peak"
+UNIT = "nodes/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def attn_flops(shape: synth.Shape, cache_len, depth, n_nodes) -> float:
+    """Algorithmic FLOPs of one verify-attention launch: for every real row
+    (b, i, h), 2 * (visible keys) * (d_qk + d_l); visible keys = L_b + depth_i + 1."""
+    f = 0.0
+    for b in range(len(n_nodes)):
+        n = int(n_nodes[b])
+        vis = int(cache_len[b]) * n + int(np.sum(depth[b, :n] + 1))
+        f += 2.0 * shape.H * vis * (shape.d_qk + shape.d_l)
+    return f
+
+
+class ClockSampler:
+    """nvidia-smi sampler (200 ms) for SM clock and throttle reasons."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.proc = None
+        self.path = None
+        if uuid is None:
+            return
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="ddt_clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", uuid, f"--query-gpu={self.Q}", "--format=csv,noheader",
+                                          "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append({"sm": float(f[1].split()[0]), "max": float(f[2].split()[0]),
+                             "hw_slowdown": f[5] == "Active", "hw_thermal_slowdown": f[6] == "Active",
+                             "sw_thermal_slowdown": f[7] == "Active", "sw_power_cap": f[8] == "Active"})
+            except Exception:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = sorted({k for r in rows for k in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                                    "sw_power_cap") if r[k]})
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline; never the product path)
+# ---------------------------------------------------------------------------
+
+
+def oracle_step_time(shape: synth.Shape, x, logits, tree, attn_nodes: int, seed: int = 0):
+    """Seconds the oracle needs for one full step of this workload, from a
+    bounded sample: the whole tree build, attention for `attn_nodes` sampled
+    nodes (all heads) scaled by the node count, the whole accept + compaction."""
+    import oracle
+
+    t0 = time.perf_counter()
+    oracle.build_tree(x.logp, x.tok, x.root_tok, x.cache_len, shape.N)
+    t_build = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    all_rows = [(b, i) for b in range(shape.B) for i in range(int(tree["n_nodes"][b]))]
+    pick = [all_rows[j] for j in sorted(rng.choice(len(all_rows), size=min(attn_nodes, len(all_rows)),
+                                                   replace=False))]
+    t0 = time.perf_counter()
+    oracle.verify_attn(x.q, x.kv, x.cache_off, x.cache_len, tree["mask"], tree["n_nodes"], shape.H, shape.d_l,
+                       shape.d_r, shape.scale, shape.dtype, rows=pick)
+    t_attn = (time.perf_counter() - t0) * len(all_rows) / max(1, len(pick))
+    kv = x.kv.copy()
+    t0 = time.perf_counter()
+    oracle.accept_compact(logits, shape.dtype, tree["node_tok"], tree["parent"], tree["n_nodes"], kv, x.cache_off,
+                          x.cache_len, x.cache_cap)
+    t_acc = time.perf_counter() - t0
+    return t_build + t_attn + t_acc, len(pick), len(all_rows)
+
+
+def run_reference(args, shape: synth.Shape, rank: int):
+    """--impl reference: the oracle as it stands, timed on the host cores."""
+    if rank != 0:
+        return
+    import oracle
+
+    x = synth.make_step(shape)
+    tree = oracle.build_tree(x.logp, x.tok, x.root_tok, x.cache_len, shape.N)
+    logits = synth.target_logits(shape, tree["parent"], tree["node_tok"], tree["n_nodes"])
+    nodes = int(tree["n_nodes"].sum())
+    sample = max(1, min(nodes, args.ref_nodes))
+    for _ in range(args.warmup if args.warmup < 2 else 1):
+        oracle_step_time(shape, x, logits, tree, sample)
+    times = []
+    for k in range(args.steps):
+        t, _, _ = oracle_step_time(shape, x, logits, tree, sample, seed=k)
+        times.append(t)
+    sec = float(np.mean(times))
+    value = nodes / sec
+    desc = (f"per step: full tree build, attention on {sample} sampled nodes x {shape.H} heads scaled to "
+            f"{nodes} nodes, full accept + compaction")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(shape),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(shape: synth.Shape, extra=None):
+    d = {"workload": shape.name, "B": shape.B, "N": shape.N, "D": shape.D, "K": shape.K, "H": shape.H,
+         "d_latent": shape.d_l, "d_rope": shape.d_r, "V": shape.V, "cache_len": list(shape.L)[:4] +
+         (["..."] if len(shape.L) > 4 else []), "in_dtype": shape.dtype}
+    if extra:
+        d.update(extra)
+    return d
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+
+def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    from ddtree_speculative_decode_b200 import lib
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    lib.load()
+    bf = shape.dtype == "bf16"
+    tdt = torch.bfloat16 if bf else torch.float32
+
+    def dev_t(a, as_bf16=False):
+        a = np.ascontiguousarray(a)
+        if as_bf16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    # ---- inputs (host draw, then resident in HBM) ---------------------------
+    x = synth.make_step(shape)
+    logp, tok = dev_t(x.logp), dev_t(x.tok)
+    root, cl0 = dev_t(x.root_tok), dev_t(x.cache_len)
+    off, cap = dev_t(x.cache_off), dev_t(x.cache_cap)
+    tree = lib.build_tree(logp, tok, root, cl0, shape.N)
+    torch.cuda.synchronize()
+    t_host = {k: v.cpu().numpy() for k, v in tree.items()}
+    logits_h = synth.target_logits(shape, t_host["parent"], t_host["node_tok"], t_host["n_nodes"])
+    set_bytes = x.kv.nbytes + x.q.nbytes + logits_h.nbytes
+    n_sets = max(1, min(16, math.ceil(2 * L2_BYTES / set_bytes)))
+    sets = []
+    for _ in range(n_sets):
+        sets.append({"kv": dev_t(x.kv, bf), "q": dev_t(x.q, bf), "logits": dev_t(logits_h, bf)})
+    maxL = int(max(shape.L))
+    B, N, H = shape.B, shape.N, shape.H
+    ws_attn = torch.empty(max(256, lib.verify_attn_workspace_size(B, N, H, shape.d_l, shape.d_r, maxL, tdt)),
+                          dtype=torch.uint8, device=dev)
+    ws_acc = torch.empty(max(256, lib.accept_compact_workspace_size(B, N, shape.V)), dtype=torch.uint8, device=dev)
+    out = torch.empty(B, N, H, shape.d_l, dtype=tdt, device=dev)
+    lse = torch.empty(B, N, H, dtype=torch.float32, device=dev)
+    acc = lib.alloc_accept(B, N, dev)
+    cl = cl0.clone()
+    stream = torch.cuda.current_stream(dev)
+    n_nodes_total = int(t_host["n_nodes"].sum())
+    flops = attn_flops(shape, x.cache_len, t_host["depth"], t_host["n_nodes"])
+    acc_bytes = float(t_host["n_nodes"].sum()) * shape.V * (2 if bf else 4)
+
+    def step(s, ev=None):
+        cl.copy_(cl0, non_blocking=True)
+        if ev is not None:
+            ev[0].record(stream)
+        lib.build_tree(logp, tok, root, cl, N, out=tree, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        lib.verify_attn(s["q"], s["kv"], off, cl, tree["mask"], tree["n_nodes"], shape.d_l, shape.d_r, shape.scale,
+                        maxL, out=out, lse=lse, workspace=ws_attn, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        lib.accept_compact(s["logits"], tree["node_tok"], tree["parent"], tree["n_nodes"], s["kv"], off, cl, cap,
+                           out=acc, workspace=ws_acc, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    # ---- warm-up ---------------------------------------------------------------
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid) if rank == 0 else ClockSampler(None)
+    for w in range(args.warmup):
+        step(sets[w % n_sets])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    # ---- timed region: exactly K steps ------------------------------------------
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(sets[k % n_sets], evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    clocks = sampler.stop()
+    build_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    accept_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    el = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(el, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(el.item())
+    value = n_nodes_total * world * args.steps / (elapsed_ms / 1e3)
+
+    # ---- end to end through the public API with host buffers -------------------------
+    e2e = run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_acc, out, lse, off, cap, maxL,
+                  world)
+
+    if rank != 0:
+        return
+    pk = peaks()
+    achieved = flops / (attn_ms / 1e3) / 1e12
+    peak = pk["bf16_tflops_sustained"]
+    launches_per_step = (1 + attn_launches(shape) + 2)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic",
+        "config": config_dict(shape, {"parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                                      "l2": f"{n_sets} rotating input sets of {set_bytes / 2**20:.1f} MiB "
+                                            f"(> 2x 126 MiB L2)"}),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "ddt_verify_attn", "peak_kind": f"bf16 dense, sustained, {pk['source']}"},
+        "stages_ms": {"build_tree": build_ms, "verify_attn": attn_ms, "accept_compact": accept_ms},
+        "accept_hbm": {"achieved_gbs": acc_bytes / (accept_ms / 1e3) / 1e9, "peak_gbs": pk["hbm_gbs"],
+                       "frac": acc_bytes / (accept_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
+        "nodes_per_step": n_nodes_total,
+        "attn_gflop_per_step": flops / 1e9,
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": e2e,
+        "clocks": clocks,
+    }
+    if args.cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(args, shape, x, logits_h, t_host)
+    print(json.dumps(line), flush=True)
+
+
+def attn_launches(shape: synth.Shape) -> int:
+    from ddtree_speculative_decode_b200 import lib
+    return 2 if lib.verify_attn_workspace_size(shape.B, shape.N, shape.H, shape.d_l, shape.d_r, max(shape.L),
+                                               _tdtype(shape)) > 0 else 1
+
+
+def _tdtype(shape):
+    import torch
+    return torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+
+
+def run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_acc, out, lse, off, cap, maxL, world):
+    """Same step through the public API, inputs from pinned host memory each
+    step (drafter output, queries, the tree rows' latent KV, target logits,
+    cache lengths) and the committed tokens read back."""
+    import torch
+    import torch.distributed as dist
+
+    bf = shape.dtype == "bf16"
+
+    def pin(a, as_bf16=False):
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if as_bf16 else np.ascontiguousarray(a))
+        t = t.pin_memory()
+        return t.view(torch.bfloat16) if as_bf16 else t
+
+    B, N = shape.B, shape.N
+    h = {"logp": pin(x.logp), "tok": pin(x.tok), "root": pin(x.root_tok), "cl": pin(x.cache_len),
+         "q": pin(x.q, bf), "logits": pin(logits_h, bf)}
+    tree_rows = [pin(x.kv[int(x.cache_off[b]) + int(x.cache_len[b]):int(x.cache_off[b]) + int(x.cache_len[b]) + N],
+                     bf) for b in range(B)]
+    d = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in h.items()}
+    kv = torch.from_numpy(x.kv.view(np.int16) if bf else x.kv).to(dev)
+    kv = kv.view(torch.bfloat16) if bf else kv
+    res_h = {"out_tok": torch.empty(B, N, dtype=torch.int32).pin_memory(),
+             "acc_len": torch.empty(B, dtype=torch.int32).pin_memory(),
+             "bonus": torch.empty(B, dtype=torch.int32).pin_memory()}
+    h2d = sum(v.numel() * v.element_size() for v in h.values()) + sum(t.numel() * t.element_size() for t in tree_rows)
+    d2h = sum(v.numel() * v.element_size() for v in res_h.values())
+
+    def step():
+        for k in h:
+            d[k].copy_(h[k], non_blocking=True)
+        for b in range(B):
+            o = int(x.cache_off[b]) + int(x.cache_len[b])
+            kv[o:o + N].copy_(tree_rows[b], non_blocking=True)
+        lib.build_tree(d["logp"], d["tok"], d["root"], d["cl"], N, out=tree, stream=stream)
+        lib.verify_attn(d["q"], kv, off, d["cl"], tree["mask"], tree["n_nodes"], shape.d_l, shape.d_r, shape.scale,
+                        maxL, out=out, lse=lse, workspace=ws_attn, stream=stream)
+        lib.accept_compact(d["logits"], tree["node_tok"], tree["parent"], tree["n_nodes"], kv, off, d["cl"], cap,
+                           out=acc, workspace=ws_acc, stream=stream)
+        res_h["out_tok"].copy_(acc["out_tok"], non_blocking=True)
+        res_h["acc_len"].copy_(acc["acc_len"], non_blocking=True)
+        res_h["bonus"].copy_(acc["bonus"], non_blocking=True)
+
+    steps = max(3, min(args.steps, args.e2e_steps))
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    nodes = int(tree["n_nodes"].sum().item())
+    return {"value": nodes * world * steps / (float(t.item()) / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps}
+
+
+def cpu_baseline(args, shape, x, logits_h, t_host):
+    import oracle
+    tree = oracle.build_tree(x.logp, x.tok, x.root_tok, x.cache_len, shape.N)
+    sec, picked, total = oracle_step_time(shape, x, logits_h, tree, args.ref_nodes)
+    return {"value": total / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"one step: full build, attention on {picked} of {total} nodes (all heads) scaled by "
+                      f"{total}/{picked}, full accept + compaction"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="kimi-1req", choices=sorted(synth.NAMED))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--ref-nodes", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    shape = synth.NAMED[args.config]()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, shape, rank)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    try:
+        run_ours(args, shape, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,217 @@
+/*
+ * ddt.h -- C ABI of libddt.so: one DDTree speculative-decoding tree-verify
+ * step on an NVIDIA B200 (sm_100a).
+ *
+ * The step has three calls, issued in this order on one CUDA stream:
+ *
+ *   ddt_build_tree      best-first draft tree from the drafter's per-depth
+ *                       top-k log-probs ("autoregressive_test_driver_kdtree_
+ *                       engine", section "The Broader Context": GPU best-first
+ *                       tree builder replacing a per-request CPU heapq;
+ *                       "ddtree_speculative_decode_test_capstone", section
+ *                       "What the Test Validated": the drafter contract);
+ *   ddt_verify_attn     MLA-absorb attention of every tree node's heads over the
+ *                       request's latent KV cache plus its visible tree
+ *                       ancestors (first page, "The Broader Context":
+ *                       tree-verify MLA-absorb attention with visibility
+ *                       masking);
+ *   ddt_accept_compact  greedy accept walk over the target's argmax and
+ *                       compaction of the accepted nodes' latent KV rows into
+ *                       the contiguous cache (first page, "The Broader
+ *                       Context": greedy tree-accept kernel, KV cache with
+ *                       post-verify compaction).
+ *
+ * Common conventions
+ *   - Every pointer argument is DEVICE memory owned by the caller, except where
+ *     a comment says "host". The library allocates no device memory: scratch
+ *     comes from a caller-provided workspace whose size a *_workspace_size()
+ *     query returns.
+ *   - Calls are asynchronous and stream-ordered on `stream` (0 = legacy default
+ *     stream); none synchronises the host. Calls on different streams with
+ *     disjoint buffers may run concurrently.
+ *   - The return value is a ddt_status. Host-side argument checks (null
+ *     pointers, sizes, unsupported shapes or dtypes) are synchronous and
+ *     launch nothing. A failed launch returns DDT_ERR_CUDA.
+ *   - Device-side preconditions (bad drafter log-probs, cache capacity) never
+ *     trap: the kernel writes a ddt_status value to dev_status[b] (when
+ *     dev_status is non-null, else the problem is only visible through the
+ *     padded outputs) and skips that request as documented per call.
+ *   - Shapes: B requests, D drafter depth, K top-k, N verify rows per request
+ *     INCLUDING the root (N - 1 drafted nodes; block_size = budget + 1 on the
+ *     capstone page), H heads, d_l latent dim, d_r RoPE dim, d_qk = d_l + d_r,
+ *     V vocab, W = ceil(N / 32) mask words. Arrays are row-major, innermost
+ *     index last.
+ *   - Limits: 1 <= N <= 1024, 1 <= K <= 32, 1 <= D <= 64, B >= 1, and the
+ *     tree's tie-break key (ceil(log2 K) bits per level, min(D, N - 1) levels)
+ *     must fit 64 bits, else DDT_ERR_UNSUPPORTED.
+ */
+#ifndef DDT_H_
+#define DDT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define DDT_API __attribute__((visibility("default")))
+#else
+#define DDT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DDT_OK = 0,
+  DDT_ERR_INVALID_ARG = 1, /* null pointer, size out of range, bad workspace */
+  DDT_ERR_UNSUPPORTED = 2, /* valid but not implemented (shape / dtype combo) */
+  DDT_ERR_CAPACITY = 3,    /* device: cache_len + n_nodes > cache_cap         */
+  DDT_ERR_INPUT = 4,       /* device: drafter log-probs violate preconditions */
+  DDT_ERR_CUDA = 5,        /* a CUDA launch or driver call failed             */
+  DDT_ERR_TIMEOUT = 6      /* device: a bounded intra-kernel wait gave up     */
+} ddt_status;
+
+typedef enum { DDT_F32 = 0, DDT_BF16 = 1 } ddt_dtype;
+
+/* Human-readable name of a status code (static string, never null). */
+DDT_API const char* ddt_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+DDT_API int ddt_version(void);
+
+/*
+ * ddt_build_tree -- best-first draft tree for every request.
+ *
+ * Passage: capstone page, "What the Test Validated" (a drafter returns, per
+ * depth up to a limit, log-probs and token ids of its top-k candidates, sorted
+ * so the tree builder's best-first search takes the best first) and first
+ * page, "The Broader Context" (GPU best-first builder replacing a heapq).
+ *
+ * Definition (readings the pages leave open are fixed here):
+ *   A rank path r = (r_1..r_d), 1 <= d <= D, scores the float32 sum
+ *   s = (((0 + logp[b][0][r_1]) + logp[b][1][r_2]) + ...) added left to right
+ *   in round-to-nearest (no fused or reassociated adds). Paths are ordered by
+ *   (s descending, d ascending, (r_1..r_d) lexicographically ascending); the
+ *   tree holds the first min(N - 1, sum_d K^d) of them. Node 0 is the root
+ *   (previous step's bonus token); node i >= 1 is the i-th path in order, so
+ *   parent[i] < i. tok = tok[b][d-1][r_d], depth = d, pos = cache_len[b] + d,
+ *   score = s. mask row i has bit j (word j >> 5, bit j & 31) set iff node j is
+ *   node i or one of its ancestors.
+ *
+ * Inputs (device):
+ *   logp      [B][D][K] float32, per depth non-increasing in k, finite, <= 0.
+ *   tok       [B][D][K] int32 candidate token ids.
+ *   root_tok  [B] int32, cache_len [B] int32 (committed rows before the step).
+ * Outputs (device, fully written for all N rows):
+ *   node_tok, parent, depth, pos [B][N] int32; score [B][N] float32;
+ *   mask [B][N][W] uint32; n_nodes [B] int32.
+ *   Pad rows i >= n_nodes[b]: node_tok/parent/depth/pos = -1, score = -inf,
+ *   mask = 0.
+ *   dev_status [B] int32 (nullable): DDT_OK, or DDT_ERR_INPUT when logp[b]
+ *   breaks its precondition -- that request then gets n_nodes = 0 and every
+ *   row padded.
+ * One warp per request; no workspace.
+ */
+DDT_API int ddt_build_tree(const float* logp, const int32_t* tok, const int32_t* root_tok,
+                   const int32_t* cache_len, int B, int D, int K, int N,
+                   int32_t* node_tok, int32_t* parent, int32_t* depth, int32_t* pos,
+                   float* score, uint32_t* mask, int32_t* n_nodes, int32_t* dev_status,
+                   cudaStream_t stream);
+
+/*
+ * ddt_verify_attn -- MLA-absorb tree-verify attention.
+ *
+ * Passage: first page, "The Broader Context" (tree-verify MLA-absorb
+ * attention kernel with visibility masking) and capstone page, "Context and
+ * Motivation" (the target verifies the drafted tree in one batched forward).
+ *
+ * Definition: each pool row is [c (d_l latent) ; k_pe (d_r RoPE key)]; the key
+ * is the whole row, the value its first d_l entries (absorbed MLA: one latent
+ * row serves every head). For request b, node i < n_nodes[b], head h:
+ *   visible keys j: every committed row j in [0, cache_len[b]) and tree row
+ *                   cache_len[b] + t for each node t < n_nodes[b] whose bit is
+ *                   set in mask[b][i];
+ *   s_j = scale * dot(q[b][i][h][:], kv[cache_off[b] + j][:])   (d_qk terms)
+ *   out[b][i][h][:] = sum_j softmax(s)_j * kv[cache_off[b] + j][0:d_l]
+ *   lse[b][i][h]    = ln sum_j exp(s_j)
+ * Pad rows (i >= n_nodes[b]): out = 0, lse = -inf.
+ *
+ * Inputs (device):
+ *   q         [B][N][H][d_qk] in_dtype; q_pe and k_pe already RoPE-rotated.
+ *   kv        pool [kv_rows][d_qk] in_dtype. Request b's rows start at
+ *             cache_off[b]: cache_len[b] committed rows, then the N tree rows
+ *             in node order (tree row t = node t's latent row).
+ *   cache_off [B] int64, cache_len [B] int32, mask [B][N][W] uint32,
+ *             n_nodes [B] int32 (as written by ddt_build_tree).
+ *   max_cache_len (host): an upper bound on every cache_len[b]; it sizes the
+ *             launch and the workspace. kv_rows (host): rows in the pool.
+ * Outputs (device): out [B][N][H][d_l] out_dtype; lse [B][N][H] float32
+ *   (nullable).
+ * Supported: in_dtype F32 (CUDA-core kernel, any d_l, d_r with d_qk <= 1024)
+ *   and BF16 with (d_l, d_r) = (512, 64) (tensor-core kernel); out_dtype F32
+ *   or BF16. Accumulation is float32 throughout. The bf16 kernel rounds the
+ *   softmax probabilities to bf16 before the P.V product.
+ * workspace: at least ddt_verify_attn_workspace_size(...) bytes of device
+ *   memory, 256-byte aligned (may be null when that size is 0). Its contents
+ *   on entry do not matter.
+ * Errors: DDT_ERR_INVALID_ARG (nulls, sizes, workspace too small or
+ *   misaligned, kv / q not 16-byte aligned for bf16), DDT_ERR_UNSUPPORTED.
+ */
+DDT_API size_t ddt_verify_attn_workspace_size(int B, int N, int H, int d_latent, int d_rope,
+                                      int max_cache_len, int in_dtype);
+
+DDT_API int ddt_verify_attn(const void* q, const void* kv, int64_t kv_rows, const int64_t* cache_off,
+                    const int32_t* cache_len, const uint32_t* mask, const int32_t* n_nodes,
+                    int B, int N, int H, int d_latent, int d_rope, float scale,
+                    int max_cache_len, int in_dtype, int out_dtype, void* out, float* lse,
+                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * ddt_accept_compact -- greedy accept walk, then latent-KV compaction.
+ *
+ * Passage: first page, "The Broader Context" (greedy tree-accept kernel; KV
+ * cache with post-verify compaction); capstone page, "What the Test
+ * Validated" (the target's prediction at the last accepted node is the bonus
+ * token; budget = block size - 1 leaves room for it).
+ *
+ * Definition: am[b][i] = the lowest index of the largest logit of row i
+ * (logits compared exactly; bf16 widened to float32). Walk: cur = 0; while some
+ * child c of cur has node_tok[b][c] == am[b][cur], move to the lowest such c.
+ * The path (root first) has a + 1 nodes; acc_len[b] = a. Committed tokens:
+ * out_tok[b][0..a] = the a accepted nodes' tokens, then bonus[b] =
+ * am[b][path[a]]. Compaction, on every layer l:
+ *   kv[l*layer_stride_rows + cache_off[b] + cache_len[b] + j]
+ *       <- kv[l*layer_stride_rows + cache_off[b] + cache_len[b] + path[j]],
+ *   j = 0..a, every source row read before any is written; then
+ *   cache_len[b] += a + 1.
+ *
+ * Inputs (device): logits [B][N][V] logits_dtype, finite; node_tok, parent
+ *   [B][N] int32 and n_nodes [B] (from ddt_build_tree); kv pool with rows of
+ *   row_elems elements of kv_dtype (row_elems * element size a multiple of
+ *   4 bytes); cache_off [B] int64; cache_cap [B] int32 (rows owned by b).
+ * In/out: cache_len [B] int32 (advanced by a + 1).
+ * Outputs (device): am [B][N] int32 (nullable; -1 on pad rows), acc_len [B],
+ *   acc_nodes [B][N] (path, -1 padded), out_tok [B][N] (-1 padded), bonus [B].
+ *   dev_status [B] (nullable): DDT_OK; DDT_ERR_CAPACITY when cache_len[b] +
+ *   n_nodes[b] > cache_cap[b] (request skipped: acc_len 0, bonus -1, nothing
+ *   copied, cache_len unchanged). Requests with n_nodes[b] == 0 are skipped
+ *   the same way with DDT_OK.
+ * workspace: ddt_accept_compact_workspace_size(B, N, V) bytes, 256-byte
+ *   aligned; contents on entry do not matter.
+ */
+DDT_API size_t ddt_accept_compact_workspace_size(int B, int N, int V);
+
+DDT_API int ddt_accept_compact(const void* logits, int logits_dtype, int V, const int32_t* node_tok,
+                       const int32_t* parent, const int32_t* n_nodes, int B, int N, void* kv,
+                       int kv_dtype, int row_elems, int n_layers, int64_t layer_stride_rows,
+                       const int64_t* cache_off, int32_t* cache_len, const int32_t* cache_cap,
+                       int32_t* am, int32_t* acc_len, int32_t* acc_nodes, int32_t* out_tok,
+                       int32_t* bonus, int32_t* dev_status, void* workspace,
+                       size_t workspace_bytes, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DDT_H_ */

@@ -1,0 +1,68 @@
+"""The C-ABI library builds, loads without a GPU and exports every entry point
+include/ddt.h declares; host-side argument checks answer without launching."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from ddtree_speculative_decode_b200 import build, lib
+
+HDR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "ddt.h")
+
+
+@pytest.fixture(scope="module")
+def so():
+    build.build()
+    return lib.load()
+
+
+def declared():
+    txt = open(HDR).read()
+    return re.findall(r"DDT_API\s+[\w\s\*]+?\b(ddt_\w+)\s*\(", txt)
+
+
+def test_header_declares_the_three_calls():
+    names = declared()
+    for n in ("ddt_build_tree", "ddt_verify_attn", "ddt_accept_compact"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(so):
+    names = declared()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(so, n), n
+    assert set(names) == set(lib.EXPORTS) | (set(names) - set(lib.EXPORTS))
+    for n in lib.EXPORTS:
+        assert n in names
+
+
+def test_status_strings_and_version(so):
+    assert lib.status_string(0) == "DDT_OK"
+    assert lib.status_string(4) == "DDT_ERR_INPUT"
+    assert lib.status_string(99) == "DDT_UNKNOWN_STATUS"
+    assert lib.version() >= 100
+
+
+def test_workspace_queries(so):
+    # accept: one 8-byte key per (row, 16384-entry vocab chunk)
+    assert lib.accept_compact_workspace_size(1, 64, 163840) == 64 * 10 * 8
+    assert lib.accept_compact_workspace_size(0, 64, 10) == 0
+    assert so.ddt_verify_attn_workspace_size(1, 8, 4, 64, 16, 32, 0) == 0  # f32 path needs none
+
+
+def test_host_validation_without_gpu(so):
+    # null pointers / out-of-range sizes are rejected before any CUDA call
+    st = so.ddt_build_tree(None, None, None, None, 1, 1, 1, 1, None, None, None, None, None, None, None, None, None)
+    assert st == lib.DDT_ERR_INVALID_ARG
+    p = ctypes.c_void_p(16)
+    args = [p] * 4 + [1, 2, 2, 2000] + [p] * 8 + [None]
+    assert so.ddt_build_tree(*args) == lib.DDT_ERR_INVALID_ARG
+    args = [p] * 4 + [1, 40, 32, 1024] + [p] * 8 + [None]  # 5 bits x 40 levels > 64
+    assert so.ddt_build_tree(*args) == lib.DDT_ERR_UNSUPPORTED
+    st = so.ddt_verify_attn(p, p, 10, p, p, p, p, 1, 8, 4, 64, 16, ctypes.c_float(-1.0), 32, 0, 0, p, None, None,
+                            0, None)
+    assert st == lib.DDT_ERR_INVALID_ARG
+    st = so.ddt_accept_compact(p, 0, 10, p, p, p, 1, 4, p, 0, 8, 1, 0, p, p, p, p, p, p, p, p, p, p, 0, None)
+    assert st == lib.DDT_ERR_INVALID_ARG  # workspace too small
