@@ -229,7 +229,7 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
         sets.append({"kv": dev_t(x.kv, bf), "q": dev_t(x.q, bf), "logits": dev_t(logits_h, bf)})
     maxL = int(max(shape.L))
     B, N, H = shape.B, shape.N, shape.H
-    ws_attn = torch.empty(max(256, lib.verify_attn_workspace_size(B, N, H, shape.d_l, shape.d_r, maxL, tdt)),
+    ws_attn = torch.zeros(max(256, lib.verify_attn_workspace_size(B, N, H, shape.d_l, shape.d_r, maxL, tdt)),
                           dtype=torch.uint8, device=dev)
     ws_acc = torch.empty(max(256, lib.accept_compact_workspace_size(B, N, shape.V)), dtype=torch.uint8, device=dev)
     out = torch.empty(B, N, H, shape.d_l, dtype=tdt, device=dev)

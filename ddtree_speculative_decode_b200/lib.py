@@ -159,6 +159,12 @@ def alloc_tree(B: int, N: int, device) -> dict:
     }
 
 
+def verify_attn_status(workspace: torch.Tensor) -> int:
+    """Device status word of a verify-attention workspace (DDT_OK or
+    DDT_ERR_TIMEOUT); reading it synchronises with the device."""
+    return int(workspace[:4].view(torch.int32).item())
+
+
 def verify_attn_workspace_size(B: int, N: int, H: int, d_l: int, d_r: int, max_cache_len: int,
                                in_dtype: torch.dtype) -> int:
     return int(load().ddt_verify_attn_workspace_size(B, N, H, d_l, d_r, max_cache_len,
@@ -193,7 +199,7 @@ def verify_attn(q: torch.Tensor, kv: torch.Tensor, cache_off: torch.Tensor, cach
         _check(lse, "lse", torch.float32, (B, N, H))
     need = verify_attn_workspace_size(B, N, H, d_l, d_r, max_cache_len, q.dtype)
     if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)  # status word must start at 0
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = load().ddt_verify_attn(_ptr(q), _ptr(kv), kv.shape[0], _ptr(cache_off), _ptr(cache_len), _ptr(mask),
                                 _ptr(n_nodes), B, N, H, d_l, d_r, float(scale), int(max_cache_len), _dt(q),

@@ -153,8 +153,13 @@ DDT_API int ddt_build_tree(const float* logp, const int32_t* tok, const int32_t*
  *   or BF16. Accumulation is float32 throughout. The bf16 kernel rounds the
  *   softmax probabilities to bf16 before the P.V product.
  * workspace: at least ddt_verify_attn_workspace_size(...) bytes of device
- *   memory, 256-byte aligned (may be null when that size is 0). Its contents
- *   on entry do not matter.
+ *   memory, 256-byte aligned (may be null when that size is 0). Its first 256
+ *   bytes are a device status word that must be zero before the first call
+ *   (zero the buffer once after allocating it). Every wait inside the bf16
+ *   kernel is bounded (about 2 s); if one expires the kernel stores
+ *   DDT_ERR_TIMEOUT there and returns, and later calls with that workspace
+ *   return at once until the caller zeroes it again. The rest of the
+ *   workspace holds per-split partial results; its contents do not matter.
  * Errors: DDT_ERR_INVALID_ARG (nulls, sizes, workspace too small or
  *   misaligned, kv / q not 16-byte aligned for bf16), DDT_ERR_UNSUPPORTED.
  */

@@ -111,3 +111,41 @@ def test_attn_bf16_small(L, N):
     t = _tree(x, s)
     g, gl, r, rl = _attn(s, x, t, out_dtype=torch.bfloat16)
     _check(g, gl, r, rl, True)
+
+
+@pytest.mark.parametrize("L,maxL", [(300, 20000), (0, 5000), (700, 3000)])
+def test_attn_bf16_many_splits(L, maxL):
+    """A generous max_cache_len makes the launch split every request's keys
+    into many slices, most of them empty: the split partials and the combine
+    step must still give the oracle's answer."""
+    s = synth.custom(B=2, D=4, K=4, N=24, H=64, d_l=512, d_r=64, V=64, L=(L, L + 33), dtype="bf16",
+                     kv_scale=0.1, scale=1.0 / np.sqrt(192.0), seed=L + 1)
+    x = synth.make_step(s)
+    t = _tree(x, s)
+    d = step_to_device(x, DEV)
+    mask = t_from(t["mask"].view(np.int32), DEV)
+    nn = t_from(t["n_nodes"], DEV)
+    ws = torch.zeros(lib.verify_attn_workspace_size(s.B, s.N, s.H, 512, 64, maxL, torch.bfloat16), dtype=torch.uint8,
+                     device=DEV)
+    assert ws.numel() > 256  # split partials are in use
+    out, lse = lib.verify_attn(d["q"], d["kv"], d["cache_off"], d["cache_len"], mask, nn, 512, 64, s.scale, maxL,
+                               workspace=ws)
+    torch.cuda.synchronize()
+    assert lib.verify_attn_status(ws) == 0
+    ref, rl = oracle.verify_attn(x.q, x.kv, x.cache_off, x.cache_len, t["mask"], t["n_nodes"], s.H, 512, 64, s.scale,
+                                 "bf16")
+    _check(widen_out(out), lse.cpu().numpy().astype(np.float64), ref, rl, True)
+
+
+def test_attn_bf16_status_word_stays_zero():
+    s = synth.kimi_1req()
+    x = synth.make_step(s)
+    t = _tree(x, s)
+    d = step_to_device(x, DEV)
+    ws = torch.zeros(lib.verify_attn_workspace_size(1, 64, 64, 512, 64, 4096, torch.bfloat16), dtype=torch.uint8,
+                     device=DEV)
+    for _ in range(3):
+        lib.verify_attn(d["q"], d["kv"], d["cache_off"], d["cache_len"], t_from(t["mask"].view(np.int32), DEV),
+                        t_from(t["n_nodes"], DEV), 512, 64, s.scale, 4096, workspace=ws)
+    torch.cuda.synchronize()
+    assert lib.verify_attn_status(ws) == lib.DDT_OK
