@@ -231,7 +231,7 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
     B, N, H = shape.B, shape.N, shape.H
     ws_attn = torch.zeros(max(256, lib.verify_attn_workspace_size(B, N, H, shape.d_l, shape.d_r, maxL, tdt)),
                           dtype=torch.uint8, device=dev)
-    ws_acc = torch.empty(max(256, lib.accept_compact_workspace_size(B, N, shape.V)), dtype=torch.uint8, device=dev)
+    ws_acc = torch.zeros(max(256, lib.accept_compact_workspace_size(B, N, shape.V)), dtype=torch.uint8, device=dev)
     out = torch.empty(B, N, H, shape.d_l, dtype=tdt, device=dev)
     lse = torch.empty(B, N, H, dtype=torch.float32, device=dev)
     acc = lib.alloc_accept(B, N, dev)
@@ -418,8 +418,8 @@ def cpu_baseline(args, shape, x, logits_h, t_host):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--config", default="kimi-1req", choices=sorted(synth.NAMED))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=200)

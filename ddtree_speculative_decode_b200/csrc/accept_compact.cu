@@ -8,16 +8,18 @@
 // post-verify compaction; "ddtree_speculative_decode_test_capstone", section
 // "What the Test Validated": the bonus token).
 //
-// Two launches:
-//  1. row_argmax_kernel: the HBM-bound part. Every (row, vocab-chunk) pair is
-//     one CTA that streams its 16-byte vectors once and reduces to one packed
-//     64-bit key (order-preserving value bits << 32 | ~index): the max key is
-//     the largest logit at its lowest index. Partial keys go to the workspace.
-//  2. walk_compact_kernel: one CTA per request folds the partial keys into
-//     am[], walks the tree with warp ballots, then copies the accepted rows.
-//     path[j] >= j and the path is increasing, so copying rows in increasing j
-//     is already read-before-write per byte; the kernel still stages each group
-//     of rows in registers behind a barrier so many rows are in flight at once.
+// One launch:
+//  * Every (row, vocab-chunk) pair is one CTA that streams its 16-byte
+//    vectors once and reduces them to one packed 64-bit key (order-preserving
+//    value bits << 32 | ~index): the max key is the largest logit at its
+//    lowest index. Partial keys go to the workspace.
+//  * The CTA that finishes a request's last chunk (a per-request arrival
+//    counter in the workspace; it resets the counter to zero for the next call)
+//    folds the partial keys into am[], walks the tree with warp ballots, then
+//    copies the accepted rows. path[j] >= j and the path is increasing, so
+//    copying rows in increasing j is already read-before-write per byte; the
+//    CTA still stages groups of rows in registers behind a barrier so many rows
+//    are in flight at once.
 #include "ddt_kernels.cuh"
 
 namespace ddt {
@@ -34,13 +36,22 @@ __device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsig
   return a > b ? a : b;
 }
 
+__device__ __noinline__ void walk_compact_body(const AcceptParams& p, int b);
+
 template <bool kBF16>
-__global__ void __launch_bounds__(kArgmaxThreads) row_argmax_kernel(AcceptParams p) {
+__global__ void __launch_bounds__(kArgmaxThreads) accept_kernel(AcceptParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int row = blockIdx.x / p.chunks;  // b * N + i
   const int chunk = blockIdx.x - row * p.chunks;
   const int b = row / p.N;
   const int i = row - b * p.N;
-  if (i >= p.n_nodes[b]) return;
+  const int n = p.n_nodes[b];
+  if (i >= n) {
+    // an empty tree has no argmax CTAs: one CTA writes its (skipped) outputs
+    if (n <= 0 && i == 0 && chunk == 0) walk_compact_body(p, b);
+    return;
+  }
   const int v0 = chunk * kArgmaxChunk;
   const int v1 = min(p.V, v0 + kArgmaxChunk);
   unsigned long long best = 0ull;
@@ -106,12 +117,21 @@ __global__ void __launch_bounds__(kArgmaxThreads) row_argmax_kernel(AcceptParams
   __shared__ unsigned long long wbest[kArgmaxThreads / 32];
   if ((threadIdx.x & 31) == 0) wbest[threadIdx.x >> 5] = best;
   __syncthreads();
+  __shared__ int s_last;
   if (threadIdx.x == 0) {
     unsigned long long m = wbest[0];
 #pragma unroll
     for (int w = 1; w < kArgmaxThreads / 32; ++w) m = umax64(m, wbest[w]);
     p.partial[(size_t)row * p.chunks + chunk] = m;
+    __threadfence();
+    const unsigned prev = atomicAdd(p.counter + b, 1u);
+    s_last = (prev == (unsigned)(n * p.chunks - 1));
   }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  walk_compact_body(p, b);
+  if (threadIdx.x == 0) p.counter[b] = 0u;
 }
 
 constexpr int kWalkThreads = 256;
@@ -119,8 +139,7 @@ constexpr int kMaxN = 1024;
 constexpr int kStageRows = 16;  // rows staged per copy round
 constexpr int kStageVec = 8;    // 16-byte vectors per thread per round (256 * 8 * 16 B = 32 KB)
 
-__global__ void __launch_bounds__(kWalkThreads) walk_compact_kernel(AcceptParams p) {
-  const int b = blockIdx.x;
+__device__ __noinline__ void walk_compact_body(const AcceptParams& p, int b) {
   const int N = p.N;
   const int n = p.n_nodes[b];
   __shared__ int32_t s_am[kMaxN];
@@ -141,7 +160,7 @@ __global__ void __launch_bounds__(kWalkThreads) walk_compact_kernel(AcceptParams
     if (i < n) {
       const unsigned long long* pk = p.partial + ((size_t)b * N + i) * p.chunks;
       unsigned long long m = 0ull;
-      for (int c = 0; c < p.chunks; ++c) m = umax64(m, pk[c]);
+      for (int c = 0; c < p.chunks; ++c) m = umax64(m, __ldcg(pk + c));
       a = static_cast<int>(~static_cast<uint32_t>(m & 0xffffffffull));
     }
     s_am[i] = a;
@@ -259,22 +278,20 @@ __global__ void __launch_bounds__(kWalkThreads) walk_compact_kernel(AcceptParams
   if (threadIdx.x == 0) p.cache_len[b] = L + rows;
 }
 
+static size_t counter_bytes(int B) { return ((size_t)B * 4 + 255) / 256 * 256; }
+
 size_t accept_workspace_bytes(int B, int N, int V) {
   const size_t chunks = (size_t)ceil_div(V, kArgmaxChunk);
-  return (size_t)B * N * chunks * sizeof(unsigned long long);
+  return counter_bytes(B) + (size_t)B * N * chunks * sizeof(unsigned long long);
 }
 
-int launch_accept_compact(AcceptParams p, cudaStream_t stream) {
+int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream) {
   p.chunks = ceil_div(p.V, kArgmaxChunk);
-  const unsigned g1 = (unsigned)p.chunks * (unsigned)(p.B * p.N);
-  if (p.logits_dtype == DDT_BF16)
-    row_argmax_kernel<true><<<g1, kArgmaxThreads, 0, stream>>>(p);
-  else
-    row_argmax_kernel<false><<<g1, kArgmaxThreads, 0, stream>>>(p);
-  int st = launch_status();
-  if (st != DDT_OK) return st;
-  walk_compact_kernel<<<p.B, kWalkThreads, 0, stream>>>(p);
-  return launch_status();
+  p.counter = static_cast<unsigned*>(workspace);
+  p.partial = reinterpret_cast<unsigned long long*>(static_cast<unsigned char*>(workspace) + counter_bytes(p.B));
+  const unsigned grid = (unsigned)p.chunks * (unsigned)(p.B * p.N);
+  if (p.logits_dtype == DDT_BF16) return launch_pdl(accept_kernel<true>, grid, kArgmaxThreads, 0, stream, p);
+  return launch_pdl(accept_kernel<false>, grid, kArgmaxThreads, 0, stream, p);
 }
 
 }  // namespace ddt

@@ -50,8 +50,91 @@ __device__ __forceinline__ bool better(float sa, int da, uint64_t ka, float sb, 
   return ka < kb;
 }
 
+
+// Ancestor masks of nodes [0, n): one lane per node walks its parent chain
+// (parent < child) and writes the row's W words, highest word first.
+__device__ __forceinline__ void write_masks(uint32_t* o_mask, int W, int n, const int32_t* n_parent, int lane) {
+  for (int i = lane; i < n; i += 32) {
+    uint32_t* row = o_mask + (size_t)i * W;
+    for (int w = (i >> 5) + 1; w < W; ++w) row[w] = 0u;
+    int cw = i >> 5;
+    uint32_t bits = 0u;
+    int j = i;
+    while (j >= 0) {
+      const int w = j >> 5;
+      while (w < cw) {
+        row[cw] = bits;
+        bits = 0u;
+        --cw;
+      }
+      bits |= 1u << (j & 31);
+      j = n_parent[j];
+    }
+    row[cw] = bits;
+    for (int w = cw - 1; w >= 0; --w) row[w] = 0u;
+  }
+}
+
+// Pad rows [n, N): token / parent / depth / pos -1, score -inf, mask 0.
+__device__ __forceinline__ void write_pads(int32_t* o_tok, int32_t* o_par, int32_t* o_dep, int32_t* o_pos,
+                                           float* o_sc, uint32_t* o_mask, int W, int n, int N, int lane) {
+  for (int i = n + lane; i < N; i += 32) {
+    o_tok[i] = -1;
+    o_par[i] = -1;
+    o_dep[i] = -1;
+    o_pos[i] = -1;
+    o_sc[i] = -INFINITY;
+    uint32_t* row = o_mask + (size_t)i * W;
+    for (int w = 0; w < W; ++w) row[w] = 0u;
+  }
+}
+
+// Loads one request's drafter output into shared memory and checks its
+// precondition (finite, <= 0, non-increasing along k). Returns true if bad.
+__device__ __forceinline__ bool load_drafter(const BuildParams& p, int b, float* lp, int32_t* tk, int lane) {
+  const int DK = p.D * p.K;
+  const float* lp_g = p.logp + (size_t)b * DK;
+  const int32_t* tk_g = p.tok + (size_t)b * DK;
+  bool bad = false;
+  for (int e = lane; e < DK; e += 32) {
+    const float v = lp_g[e];
+    lp[e] = v;
+    tk[e] = tk_g[e];
+    if (!(v <= 0.0f) || isinf(v)) bad = true;  // NaN, +inf, > 0, -inf
+    if ((e % p.K) != 0 && !(v <= lp_g[e - 1])) bad = true;
+  }
+  bad = __any_sync(DDT_FULL_MASK, bad);
+  __syncwarp();
+  return bad;
+}
+
+// Warp-wide winner among the lanes' local bests: score first (redux.sync on an
+// order-preserving key), then depth, then the packed rank key. Returns the
+// winning lane; `valid` marks lanes that hold a candidate.
+__device__ __forceinline__ int warp_winner(bool valid, float bs, int bd, uint64_t bk, int lane) {
+  const uint32_t so = valid ? float_order_key(bs) : 0u;
+  const uint32_t top = __reduce_max_sync(DDT_FULL_MASK, so);
+  uint32_t cand = __ballot_sync(DDT_FULL_MASK, valid && so == top);
+  if (__popc(cand) > 1) {
+    bool in = (cand >> lane) & 1u;
+    const uint32_t dmin = __reduce_min_sync(DDT_FULL_MASK, in ? (uint32_t)bd : 0xffffffffu);
+    cand = __ballot_sync(DDT_FULL_MASK, in && (uint32_t)bd == dmin);
+    if (__popc(cand) > 1) {
+      in = (cand >> lane) & 1u;
+      const uint32_t khi = __reduce_min_sync(DDT_FULL_MASK, in ? (uint32_t)(bk >> 32) : 0xffffffffu);
+      cand = __ballot_sync(DDT_FULL_MASK, in && (uint32_t)(bk >> 32) == khi);
+      in = (cand >> lane) & 1u;
+      const uint32_t klo = __reduce_min_sync(DDT_FULL_MASK, in ? (uint32_t)bk : 0xffffffffu);
+      cand = __ballot_sync(DDT_FULL_MASK, in && (uint32_t)bk == klo);
+    }
+  }
+  return __ffs(cand) - 1;
+}
+
 __global__ void __launch_bounds__(32) build_tree_kernel(BuildParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_wait();
+  pdl_launch_dependents();
   const int b = blockIdx.x;
   const int lane = threadIdx.x;
   const int N = p.N, D = p.D, K = p.K, W = p.W;
@@ -69,18 +152,7 @@ __global__ void __launch_bounds__(32) build_tree_kernel(BuildParams p) {
   s.tk = reinterpret_cast<int32_t*>(cur);
 
   // ---- load drafter output, check its precondition -------------------------
-  const float* lp_g = p.logp + (size_t)b * D * K;
-  const int32_t* tk_g = p.tok + (size_t)b * D * K;
-  bool bad = false;
-  for (int e = lane; e < D * K; e += 32) {
-    float v = lp_g[e];
-    s.lp[e] = v;
-    s.tk[e] = tk_g[e];
-    if (!(v <= 0.0f) || isinf(v)) bad = true;  // NaN, +inf, > 0, -inf
-    if ((e % K) != 0 && !(v <= lp_g[e - 1])) bad = true;
-  }
-  bad = __any_sync(DDT_FULL_MASK, bad);
-  __syncwarp();
+  const bool bad = load_drafter(p, b, s.lp, s.tk, lane);
 
   const int L = p.cache_len[b];
   int32_t* o_tok = p.node_tok + (size_t)b * N;
@@ -125,24 +197,7 @@ __global__ void __launch_bounds__(32) build_tree_kernel(BuildParams p) {
           bs = sc; bd = dd; bk = kk; bslot = f;
         }
       }
-      // warp-wide winner: score, then depth, then packed ranks
-      uint32_t so = bslot >= 0 ? float_order_key(bs) : 0u;
-      uint32_t top = __reduce_max_sync(DDT_FULL_MASK, so);
-      uint32_t cand = __ballot_sync(DDT_FULL_MASK, bslot >= 0 && so == top);
-      if (__popc(cand) > 1) {
-        bool in = (cand >> lane) & 1u;
-        uint32_t dmin = __reduce_min_sync(DDT_FULL_MASK, in ? (uint32_t)bd : 0xffffffffu);
-        cand = __ballot_sync(DDT_FULL_MASK, in && (uint32_t)bd == dmin);
-        if (__popc(cand) > 1) {
-          in = (cand >> lane) & 1u;
-          uint32_t khi = __reduce_min_sync(DDT_FULL_MASK, in ? (uint32_t)(bk >> 32) : 0xffffffffu);
-          cand = __ballot_sync(DDT_FULL_MASK, in && (uint32_t)(bk >> 32) == khi);
-          in = (cand >> lane) & 1u;
-          uint32_t klo = __reduce_min_sync(DDT_FULL_MASK, in ? (uint32_t)bk : 0xffffffffu);
-          cand = __ballot_sync(DDT_FULL_MASK, in && (uint32_t)bk == klo);
-        }
-      }
-      const int wl = __ffs(cand) - 1;
+      const int wl = warp_winner(bslot >= 0, bs, bd, bk, lane);
       const int slot = __shfl_sync(DDT_FULL_MASK, bslot, wl);
       if (lane == 0) {
         const float sc = s.f_score[slot];
@@ -196,52 +251,177 @@ __global__ void __launch_bounds__(32) build_tree_kernel(BuildParams p) {
       ++n;
       __syncwarp();
     }
-    // ---- ancestor masks: one lane per node, walk parents -----------------
-    for (int i = lane; i < n; i += 32) {
-      uint32_t* row = o_mask + (size_t)i * W;
-      for (int w = (i >> 5) + 1; w < W; ++w) row[w] = 0u;
-      int cw = i >> 5;
-      uint32_t bits = 0u;
-      int j = i;
-      while (j >= 0) {
-        const int w = j >> 5;
-        while (w < cw) {
-          row[cw] = bits;
-          bits = 0u;
-          --cw;
-        }
-        bits |= 1u << (j & 31);
-        j = s.n_parent[j];
-      }
-      row[cw] = bits;
-      for (int w = cw - 1; w >= 0; --w) row[w] = 0u;
-    }
+    write_masks(o_mask, W, n, s.n_parent, lane);
   }
-  // ---- pad rows -------------------------------------------------------------
-  for (int i = n + lane; i < N; i += 32) {
-    o_tok[i] = -1;
-    o_par[i] = -1;
-    o_dep[i] = -1;
-    o_pos[i] = -1;
-    o_sc[i] = -INFINITY;
-    uint32_t* row = o_mask + (size_t)i * W;
-    for (int w = 0; w < W; ++w) row[w] = 0u;
-  }
+  write_pads(o_tok, o_par, o_dep, o_pos, o_sc, o_mask, W, n, N, lane);
   if (lane == 0) {
     p.n_nodes[b] = n;
     if (p.dev_status) p.dev_status[b] = bad ? DDT_ERR_INPUT : DDT_OK;
   }
 }
 
+
+// Same search with the frontier in registers: slot f lives in lane f % 32,
+// register f / 32 (SPL = slots per lane, N <= 32 * SPL). A pop then needs no
+// shared-memory traffic: each lane scans its own registers, the winner's entry
+// is broadcast with shuffles, and only the owner lanes of the (at most two)
+// updated slots write.
+template <int SPL>
+__global__ void __launch_bounds__(32) build_tree_reg_kernel(BuildParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int b = blockIdx.x;
+  const int lane = threadIdx.x;
+  const int N = p.N, D = p.D, K = p.K, W = p.W;
+  int32_t* n_parent = reinterpret_cast<int32_t*>(smem_raw);
+  float* lp = reinterpret_cast<float*>(smem_raw + (size_t)N * 4);
+  int32_t* tk = reinterpret_cast<int32_t*>(smem_raw + (size_t)N * 4 + (size_t)D * K * 4);
+  const bool bad = load_drafter(p, b, lp, tk, lane);
+
+  const int L = p.cache_len[b];
+  int32_t* o_tok = p.node_tok + (size_t)b * N;
+  int32_t* o_par = p.parent + (size_t)b * N;
+  int32_t* o_dep = p.depth + (size_t)b * N;
+  int32_t* o_pos = p.pos + (size_t)b * N;
+  float* o_sc = p.score + (size_t)b * N;
+  uint32_t* o_mask = p.mask + (size_t)b * N * W;
+
+  int n = 0;
+  if (!bad) {
+    float f_sc[SPL], f_ps[SPL];
+    int f_d[SPL], f_r[SPL], f_p[SPL];
+    uint64_t f_k[SPL];
+#pragma unroll
+    for (int q = 0; q < SPL; ++q) {
+      f_sc[q] = 0.0f; f_ps[q] = 0.0f; f_d[q] = 0; f_r[q] = 0; f_p[q] = 0; f_k[q] = 0ull;
+    }
+    if (lane == 0) {
+      o_tok[0] = p.root_tok[b];
+      o_par[0] = -1;
+      o_dep[0] = 0;
+      o_pos[0] = L;
+      o_sc[0] = 0.0f;
+      n_parent[0] = -1;
+      f_sc[0] = __fadd_rn(0.0f, lp[0]);  // rank 0 at depth 1
+      f_d[0] = 1;
+    }
+    int fsize = (N > 1) ? 1 : 0;
+    n = 1;
+    while (n < N && fsize > 0) {
+      // lane-local best over this lane's slots
+      int bj = -1;
+      float bs = 0.0f;
+      int bd = 0;
+      uint64_t bk = 0ull;
+#pragma unroll
+      for (int q = 0; q < SPL; ++q) {
+        if (32 * q + lane < fsize && (bj < 0 || better(f_sc[q], f_d[q], f_k[q], bs, bd, bk))) {
+          bj = q; bs = f_sc[q]; bd = f_d[q]; bk = f_k[q];
+        }
+      }
+      const int wl = warp_winner(bj >= 0, bs, bd, bk, lane);
+      // the winner's remaining fields
+      float ps_l = 0.0f;
+      int r_l = 0, p_l = 0;
+#pragma unroll
+      for (int q = 0; q < SPL; ++q)
+        if (q == bj) { ps_l = f_ps[q]; r_l = f_r[q]; p_l = f_p[q]; }
+      const int wj = __shfl_sync(DDT_FULL_MASK, bj, wl);
+      const float sc = __shfl_sync(DDT_FULL_MASK, bs, wl);
+      const int dd = __shfl_sync(DDT_FULL_MASK, bd, wl);
+      const uint64_t kk = __shfl_sync(DDT_FULL_MASK, bk, wl);
+      const float psc = __shfl_sync(DDT_FULL_MASK, ps_l, wl);
+      const int rr = __shfl_sync(DDT_FULL_MASK, r_l, wl);
+      const int pp = __shfl_sync(DDT_FULL_MASK, p_l, wl);
+      const int slot = 32 * wj + wl;
+      const int i = n;
+      if (lane == wl) {
+        o_tok[i] = tk[(dd - 1) * K + rr];
+        o_par[i] = pp;
+        o_dep[i] = dd;
+        o_pos[i] = L + dd;
+        o_sc[i] = sc;
+        n_parent[i] = pp;
+      }
+      const bool has_child = dd < D;
+      const bool has_sib = rr + 1 < K;
+      if (has_child && lane == wl) {  // first child takes the popped slot
+        const float cs = __fadd_rn(sc, lp[dd * K]);
+#pragma unroll
+        for (int q = 0; q < SPL; ++q)
+          if (q == wj) { f_sc[q] = cs; f_ps[q] = sc; f_d[q] = dd + 1; f_r[q] = 0; f_p[q] = i; f_k[q] = kk << p.bpl; }
+      }
+      if (has_sib) {  // next sibling: the popped slot, or a new one at the end
+        const int t = has_child ? fsize : slot;
+        if (lane == (t & 31)) {
+          const float ss = __fadd_rn(psc, lp[(dd - 1) * K + rr + 1]);
+          const int tj = t >> 5;
+#pragma unroll
+          for (int q = 0; q < SPL; ++q)
+            if (q == tj) { f_sc[q] = ss; f_ps[q] = psc; f_d[q] = dd; f_r[q] = rr + 1; f_p[q] = pp; f_k[q] = kk + 1ull; }
+        }
+        if (has_child) ++fsize;
+      }
+      if (!has_child && !has_sib) {  // remove the popped slot: move the last entry into it
+        const int last = fsize - 1;
+        if (last != slot) {
+          const int ll = last & 31, lj = last >> 5;
+          float m_sc = 0.0f, m_ps = 0.0f;
+          int m_d = 0, m_r = 0, m_p = 0;
+          uint64_t m_k = 0ull;
+#pragma unroll
+          for (int q = 0; q < SPL; ++q)
+            if (q == lj) { m_sc = f_sc[q]; m_ps = f_ps[q]; m_d = f_d[q]; m_r = f_r[q]; m_p = f_p[q]; m_k = f_k[q]; }
+          m_sc = __shfl_sync(DDT_FULL_MASK, m_sc, ll);
+          m_ps = __shfl_sync(DDT_FULL_MASK, m_ps, ll);
+          m_d = __shfl_sync(DDT_FULL_MASK, m_d, ll);
+          m_r = __shfl_sync(DDT_FULL_MASK, m_r, ll);
+          m_p = __shfl_sync(DDT_FULL_MASK, m_p, ll);
+          m_k = __shfl_sync(DDT_FULL_MASK, m_k, ll);
+          if (lane == wl) {
+#pragma unroll
+            for (int q = 0; q < SPL; ++q)
+              if (q == wj) { f_sc[q] = m_sc; f_ps[q] = m_ps; f_d[q] = m_d; f_r[q] = m_r; f_p[q] = m_p; f_k[q] = m_k; }
+          }
+        }
+        --fsize;
+      }
+      ++n;
+    }
+    __syncwarp();
+    write_masks(o_mask, W, n, n_parent, lane);
+  }
+  write_pads(o_tok, o_par, o_dep, o_pos, o_sc, o_mask, W, n, N, lane);
+  if (lane == 0) {
+    p.n_nodes[b] = n;
+    if (p.dev_status) p.dev_status[b] = bad ? DDT_ERR_INPUT : DDT_OK;
+  }
+}
+
+template <int SPL>
+static int launch_reg(const BuildParams& p, cudaStream_t stream) {
+  const size_t smem = (size_t)p.N * 4 + (size_t)p.D * p.K * 8;
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(build_tree_reg_kernel<SPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return DDT_ERR_CUDA;
+  }
+  return launch_pdl(build_tree_reg_kernel<SPL>, (unsigned)p.B, 32, smem, stream, p);
+}
+
 int launch_build_tree(const BuildParams& p, cudaStream_t stream) {
+  if (p.N <= 32) return launch_reg<1>(p, stream);
+  if (p.N <= 64) return launch_reg<2>(p, stream);
+  if (p.N <= 128) return launch_reg<4>(p, stream);
+  if (p.N <= 256) return launch_reg<8>(p, stream);
   const size_t smem = build_smem_bytes(p.N, p.D, p.K);
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(build_tree_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return DDT_ERR_CUDA;
   }
-  build_tree_kernel<<<p.B, 32, smem, stream>>>(p);
-  return launch_status();
+  return launch_pdl(build_tree_kernel, (unsigned)p.B, 32, smem, stream, p);
 }
 
 }  // namespace ddt

@@ -131,8 +131,7 @@ int ddt_accept_compact(const void* logits, int logits_dtype, int V, const int32_
   p.out_tok = out_tok;
   p.bonus = bonus;
   p.dev_status = dev_status;
-  p.partial = static_cast<unsigned long long*>(workspace);
-  return ddt::launch_accept_compact(p, stream);
+  return ddt::launch_accept_compact(p, workspace, stream);
 }
 
 }  // extern "C"

@@ -46,10 +46,11 @@ struct AcceptParams {
   int32_t* bonus;
   int32_t* dev_status;
   unsigned long long* partial;  // [B*N][chunks] packed (value, ~index) keys
+  unsigned* counter;            // [B] chunk arrivals per request (zero between calls)
   int chunks;
 };
 size_t accept_workspace_bytes(int B, int N, int V);
-int launch_accept_compact(AcceptParams p, cudaStream_t stream);
+int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream);
 
 // ---- verify attention -------------------------------------------------------
 struct AttnParams {

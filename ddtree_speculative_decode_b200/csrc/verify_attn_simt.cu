@@ -28,6 +28,8 @@ __device__ __forceinline__ float ld_elem<uint16_t>(const uint16_t* p, int i) { r
 
 template <typename Tin, int PL>
 __global__ void __launch_bounds__(32 * kSimtWarps) attn_simt_kernel(AttnParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * kSimtWarps + warp;  // ((b * N) + i) * H + h
   const long long total = (long long)p.B * p.N * p.H;
@@ -117,14 +119,13 @@ static int launch_simt_t(const AttnParams& p, cudaStream_t stream) {
   const int d_qk = p.d_l + p.d_r;
   const int pl = ceil_div(d_qk, 32);
   if (pl <= 4)
-    attn_simt_kernel<Tin, 4><<<grid, 32 * kSimtWarps, 0, stream>>>(p);
+    return launch_pdl(attn_simt_kernel<Tin, 4>, grid, 32 * kSimtWarps, 0, stream, p);
   else if (pl <= 8)
-    attn_simt_kernel<Tin, 8><<<grid, 32 * kSimtWarps, 0, stream>>>(p);
+    return launch_pdl(attn_simt_kernel<Tin, 8>, grid, 32 * kSimtWarps, 0, stream, p);
   else if (pl <= 18)
-    attn_simt_kernel<Tin, 18><<<grid, 32 * kSimtWarps, 0, stream>>>(p);
+    return launch_pdl(attn_simt_kernel<Tin, 18>, grid, 32 * kSimtWarps, 0, stream, p);
   else
-    attn_simt_kernel<Tin, kMaxPerLane><<<grid, 32 * kSimtWarps, 0, stream>>>(p);
-  return launch_status();
+    return launch_pdl(attn_simt_kernel<Tin, kMaxPerLane>, grid, 32 * kSimtWarps, 0, stream, p);
 }
 
 int launch_attn_simt(const AttnParams& p, cudaStream_t stream) {

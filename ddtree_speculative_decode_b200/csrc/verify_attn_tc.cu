@@ -171,6 +171,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
+  pdl_wait();
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -548,6 +550,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
 // Merge split partials: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
 __global__ void __launch_bounds__(128) attn_combine_kernel(TcParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int rows_total = p.B * p.N * p.H;
   const int row = blockIdx.x;
   if (row >= rows_total) return;
@@ -686,11 +690,9 @@ int launch_attn_tc(const AttnParams& a, int64_t kv_rows, int max_cache_len, void
     attr_set = true;
   }
   const long long units = (long long)a.B * p.rowtiles * p.splits;
-  attn_tc_kernel<<<(unsigned)(2 * units), kThreads, kSmemAlloc, stream>>>(tq, tkv, p);
-  int st = launch_status();
+  int st = launch_pdl(attn_tc_kernel, (unsigned)(2 * units), kThreads, kSmemAlloc, stream, tq, tkv, p);
   if (st != DDT_OK || p.splits == 1) return st;
-  attn_combine_kernel<<<(unsigned)q_rows, 128, 0, stream>>>(p);
-  return launch_status();
+  return launch_pdl(attn_combine_kernel, (unsigned)q_rows, 128, 0, stream, p);
 }
 
 }  // namespace ddt

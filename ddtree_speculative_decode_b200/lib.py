@@ -233,7 +233,7 @@ def accept_compact(logits: torch.Tensor, node_tok: torch.Tensor, parent: torch.T
         out = alloc_accept(B, N, dev)
     need = accept_compact_workspace_size(B, N, V)
     if workspace is None:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)  # arrival counters start at 0
     row_elems = kv.shape[-1]
     st = load().ddt_accept_compact(_ptr(logits), _dt(logits), V, _ptr(node_tok), _ptr(parent), _ptr(n_nodes), B, N,
                                    _ptr(kv), _dt(kv), row_elems, n_layers, layer_stride_rows, _ptr(cache_off),

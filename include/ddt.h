@@ -203,7 +203,14 @@ DDT_API int ddt_verify_attn(const void* q, const void* kv, int64_t kv_rows, cons
  *   copied, cache_len unchanged). Requests with n_nodes[b] == 0 are skipped
  *   the same way with DDT_OK.
  * workspace: ddt_accept_compact_workspace_size(B, N, V) bytes, 256-byte
- *   aligned; contents on entry do not matter.
+ *   aligned. It starts with one arrival counter per request (rounded up to
+ *   256 bytes) that must be zero before the first call -- zero the buffer once
+ *   after allocating it; every call leaves the counters at zero again. The
+ *   rest holds one partial argmax key per (row, 16384-entry vocab chunk) and
+ *   may hold anything on entry. Calls that share a workspace must not overlap
+ *   on the GPU.
+ * Runs as one kernel: the CTA that reduces a request's last vocab chunk also
+ *   walks that request's tree and compacts its rows.
  */
 DDT_API size_t ddt_accept_compact_workspace_size(int B, int N, int V);
 

@@ -46,8 +46,9 @@ def test_status_strings_and_version(so):
 
 
 def test_workspace_queries(so):
-    # accept: one 8-byte key per (row, 16384-entry vocab chunk)
-    assert lib.accept_compact_workspace_size(1, 64, 163840) == 64 * 10 * 8
+    # accept: per-request counters (256-byte block) + one 8-byte key per (row, 16384-entry vocab chunk)
+    assert lib.accept_compact_workspace_size(1, 64, 163840) == 256 + 64 * 10 * 8
+    assert lib.accept_compact_workspace_size(65, 8, 16384) == 512 + 65 * 8 * 8
     assert lib.accept_compact_workspace_size(0, 64, 10) == 0
     assert so.ddt_verify_attn_workspace_size(1, 8, 4, 64, 16, 32, 0) == 0  # f32 path needs none
 
