@@ -19,11 +19,17 @@
 //    576-d rows through TMA), K-steps of 16 over 576 dims. PV: two MMAs with
 //    N = 256 output dims each (each CTA supplies 128 dims of the latent rows,
 //    read MN-major from the same TMA tiles layout), K = 256 keys.
-//  * Warp roles per CTA: warp 0 = TMA producer (both CTAs load their halves
-//    into their own shared memory, completion counted on the leader CTA's
-//    barrier), warp 1 = MMA issuer (leader CTA only; also TMEM allocator),
-//    warps 4..7 = softmax (TMEM lane quarter = warp % 4; thread = one query
-//    row x one half of the tile's keys / output dims).
+//  * Warp roles per CTA: warps 0 / 2 = TMA producers of the key ring and the
+//    value ring (both CTAs load their halves into their own shared memory,
+//    completion counted on the leader CTA's barriers), warps 1 / 3 = the QK
+//    and PV MMA issuers (leader CTA only; warp 1 also allocates TMEM),
+//    warps 4..11 = softmax (TMEM lane quarter = warp % 4, two warps per
+//    quarter; thread = one query row x one 64-key group of the tile, and one
+//    of the row's two 128-dim output accumulator blocks).
+//  * Two issuing threads because every mbarrier wait in an issuing thread
+//    stalls the tensor pipe for about as long as two MMAs (its issue queue
+//    is shallow); with QK and PV on separate threads and separate rings, one
+//    thread's waits hide behind the other's MMAs.
 //  * Online softmax in the base-2 domain; the running max is only moved (and
 //    the TMEM output rescaled) when it grows by more than 8, so P <= 256.
 //    P is rounded to bf16 into shared memory (K-major, 128-byte swizzle) and
@@ -51,32 +57,37 @@ using namespace sm100;
 constexpr int kDL = 512, kDR = 64, kDQK = 576;
 constexpr int kChunks = kDQK / 64;          // 9 column chunks of 64 (128 bytes)
 constexpr int kTileKeys = 256;              // keys per tile
-constexpr int kStages = 6;                  // ring stages
 constexpr int kStageBytes = 16384;          // 2 TMA boxes of 64 x 128 B
 constexpr int kBoxBytes = 8192;
 constexpr int kQBytes = kChunks * kBoxBytes;  // 73728
 constexpr int kPBytes = 4 * kBoxBytes;        // 64 rows x 256 keys bf16
 constexpr int kMaxW = 8;                      // mask words per row (N <= 256)
-constexpr int kThreads = 256;
+constexpr int kSoftmaxWarps = 8;               // warps 4..11, two per SM sub-partition
+constexpr int kThreads = 32 * (4 + kSoftmaxWarps);
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 // shared memory map (bytes from the 1024-aligned base)
+constexpr int kKStages = 3;                    // K ring (QK operand B)
+constexpr int kVStages = 3;                    // V ring (PV operand B)
 constexpr int kOffQ = 0;
-constexpr int kOffRing = kOffQ + kQBytes;
-constexpr int kOffP = kOffRing + kStages * kStageBytes;
+constexpr int kOffKRing = kOffQ + kQBytes;
+constexpr int kOffVRing = kOffKRing + kKStages * kStageBytes;
+constexpr int kOffP = kOffVRing + kVStages * kStageBytes;
 constexpr int kOffMisc = kOffP + kPBytes;
 // misc: barriers (8 B each)
-constexpr int kBarFull = 0;                   // [kStages] leader: TMA bytes of both CTAs
-constexpr int kBarEmpty = kBarFull + kStages;  // [kStages] each CTA: MMA done with stage
-constexpr int kBarQ = kBarEmpty + kStages;     // leader: Q bytes
-constexpr int kBarSFull = kBarQ + 1;           // [2] each CTA: S buffer written
-constexpr int kBarSEmpty = kBarSFull + 2;      // [2] leader: S buffer read (8 warps)
-constexpr int kBarPFull = kBarSEmpty + 2;      // leader: P written (8 warps)
-constexpr int kBarOFull = kBarPFull + 1;       // each CTA: PV finished
+constexpr int kBarKFull = 0;                     // [kKStages] leader: TMA bytes of both CTAs
+constexpr int kBarKEmpty = kBarKFull + kKStages; // [kKStages] each CTA: QK MMAs done with the stage
+constexpr int kBarVFull = kBarKEmpty + kKStages; // [kVStages]
+constexpr int kBarVEmpty = kBarVFull + kVStages; // [kVStages]
+constexpr int kBarQ = kBarVEmpty + kVStages;     // leader: Q bytes
+constexpr int kBarSFull = kBarQ + 1;             // [2] each CTA: S buffer written
+constexpr int kBarSEmpty = kBarSFull + 2;        // [2] leader: S buffer read (softmax warps of both CTAs)
+constexpr int kBarPFull = kBarSEmpty + 2;        // leader: P written (softmax warps of both CTAs)
+constexpr int kBarOFull = kBarPFull + 1;         // each CTA: PV finished
 constexpr int kNumBars = kBarOFull + 1;
-constexpr int kOffRed = kOffMisc + 256;                 // float [2 parity][2 half][64]
-constexpr int kOffLred = kOffRed + 2 * 2 * 64 * 4;      // float [2][64]
-constexpr int kOffMask = kOffLred + 2 * 64 * 4;         // uint32 [64][kMaxW]
+constexpr int kOffRed = kOffMisc + 256;                 // float [2 parity][4 groups][64]
+constexpr int kOffLred = kOffRed + 2 * 4 * 64 * 4;      // float [4][64]
+constexpr int kOffMask = kOffLred + 4 * 64 * 4;         // uint32 [64][kMaxW]
 constexpr int kOffTmem = kOffMask + 64 * kMaxW * 4;     // uint32
 constexpr int kSmemBytes = kOffTmem + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;           // slack for 1024 alignment
@@ -218,16 +229,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(kBarFull + s), 1);
-      mbar_init(bar(kBarEmpty + s), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);
     }
     mbar_init(bar(kBarQ), 1);
     mbar_init(bar(kBarSFull + 0), 1);
     mbar_init(bar(kBarSFull + 1), 1);
-    mbar_init(bar(kBarSEmpty + 0), 8);
-    mbar_init(bar(kBarSEmpty + 1), 8);
-    mbar_init(bar(kBarPFull), 8);
+    mbar_init(bar(kBarSEmpty + 0), 2 * kSoftmaxWarps);
+    mbar_init(bar(kBarSEmpty + 1), 2 * kSoftmaxWarps);
+    mbar_init(bar(kBarPFull), 2 * kSoftmaxWarps);
     mbar_init(bar(kBarOFull), 1);
     fence_mbar_init_cluster();
   }
@@ -255,27 +270,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmem);
   int* abort = p.abort;
 
-  if (warp == 0) {
-    // ============================================================ producer
-    if (lane == 0) {
-      const uint32_t full0 = map_to_rank(bar(kBarFull), 0);
+  // one ring of 16 KB stages per operand stream, each with its own producer
+  // thread and its own MMA-issuing thread: while one issuer waits on a
+  // barrier, the other keeps the tensor pipe fed
+  struct Ring {
+    int slot = 0;
+    uint32_t phase = 0;
+  };
+  if ((warp == 0 || warp == 2) && lane == 0) {
+    // ============================================================ producers
+    const bool kprod = warp == 0;
+    const int nst = kprod ? kKStages : kVStages;
+    const int off = kprod ? kOffKRing : kOffVRing;
+    const int fb0 = kprod ? kBarKFull : kBarVFull;
+    const int eb0 = kprod ? kBarKEmpty : kBarVEmpty;
+    const uint32_t full0 = map_to_rank(bar(fb0), 0);
+    Ring rg;
+    bool ok = true;
+    auto next_stage = [&](auto&& issue) {
+      if (!ok) return;
+      if (!mbar_wait(bar(eb0 + rg.slot), rg.phase ^ 1u, abort)) { ok = false; return; }
+      if (leader) mbar_arrive_expect_tx(bar(fb0 + rg.slot), 2u * kStageBytes);
+      issue(sbase + off + rg.slot * kStageBytes, full0 + 8u * (uint32_t)rg.slot);
+      if (++rg.slot == nst) { rg.slot = 0; rg.phase ^= 1u; }
+    };
+    if (kprod) {
+      // Q: this CTA's 64 rows x 9 chunks, then every tile's 9 key chunks
       const uint32_t q_bar = map_to_rank(bar(kBarQ), 0);
-      // Q: this CTA's 64 rows x 9 chunks
       if (leader) mbar_arrive_expect_tx(bar(kBarQ), 2u * kQBytes);
       const int qrow = u.b * req_rows + row0;
       for (int ch = 0; ch < kChunks; ++ch)
         tma_load_2d_pair(sbase + kOffQ + ch * kBoxBytes, &tm_q, ch * 64, qrow, q_bar);
-      int slot = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      auto next_stage = [&](auto&& issue) {
-        if (!ok) return;
-        if (!mbar_wait(bar(kBarEmpty + slot), phase ^ 1u, abort)) { ok = false; return; }
-        if (leader) mbar_arrive_expect_tx(bar(kBarFull + slot), 2u * kStageBytes);
-        issue(sbase + kOffRing + slot * kStageBytes, full0 + 8u * (uint32_t)slot);
-        if (++slot == kStages) { slot = 0; phase ^= 1u; }
-      };
-      auto load_k = [&](int t) {
+      for (int t = 0; t < u.T && ok; ++t) {
         const int tile0 = u.kb + t * kTileKeys;
         const int y0 = u.off_row + group_window(tile0 + 128 * (int)rank, u.nkeys);
         const int y1 = u.off_row + group_window(tile0 + 128 * (int)rank + 64, u.nkeys);
@@ -284,8 +310,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tma_load_2d_pair(dst, &tm_kv, ch * 64, y0, fb);
             tma_load_2d_pair(dst + kBoxBytes, &tm_kv, ch * 64, y1, fb);
           });
-      };
-      auto load_v = [&](int t) {
+      }
+    } else {
+      // every tile's value rows: two 128-dim blocks x four 64-key groups
+      for (int t = 0; t < u.T && ok; ++t) {
         const int tile0 = u.kb + t * kTileKeys;
         for (int j = 0; j < 2; ++j)
           for (int g = 0; g < 4; ++g) {
@@ -296,89 +324,84 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               tma_load_2d_pair(dst + kBoxBytes, &tm_kv, x + 64, y, fb);
             });
           }
-      };
-      load_k(0);
-      for (int t = 1; t < u.T; ++t) {
-        load_k(t);
-        load_v(t - 1);
       }
-      load_v(u.T - 1);
     }
-  } else if (warp == 1) {
-    // ============================================================ MMA issuer
-    if (leader && lane == 0) {
-      bool ok = mbar_wait(bar(kBarQ), 0, abort);
-      tc_fence_after();
-      int slot = 0;
-      uint32_t phase = 0;
-      auto take = [&]() -> bool {
-        if (!ok) return false;
-        if (!mbar_wait(bar(kBarFull + slot), phase, abort)) { ok = false; return false; }
-        tc_fence_after();
-        return true;
-      };
-      auto release = [&]() {
-        mma_commit_pair_mc(bar(kBarEmpty + slot), 0x3);
-        if (++slot == kStages) { slot = 0; phase ^= 1u; }
-      };
-      auto qk = [&](int t) {
+  } else if ((warp == 1 || warp == 3) && lane == 0 && leader) {
+    // ============================================================ MMA issuers
+    bool ok = true;
+    Ring rg;
+    // stage data comes from TMA (async proxy to async proxy): the mbarrier
+    // wait alone orders it before the MMAs, no tcgen05 fence needed
+    auto take = [&](int fb0) -> bool {
+      if (!ok) return false;
+      if (!mbar_wait(bar(fb0 + rg.slot), rg.phase, abort)) { ok = false; return false; }
+      return true;
+    };
+    if (warp == 1) {
+      // QK^T into the two S buffers
+      if (!mbar_wait(bar(kBarQ), 0, abort)) ok = false;
+      for (int t = 0; t < u.T && ok; ++t) {
         const int sb = t & 1;
         if (t >= 2) {
-          if (ok && !mbar_wait(bar(kBarSEmpty + sb), (uint32_t)(((t >> 1) + 1) & 1), abort)) ok = false;
+          if (!mbar_wait(bar(kBarSEmpty + sb), (uint32_t)(((t >> 1) + 1) & 1), abort)) { ok = false; break; }
           tc_fence_after();
         }
         const uint32_t d = tmem + (sb ? kColS1 : kColS0);
         for (int ch = 0; ch < kChunks; ++ch) {
-          if (!take()) return;
+          if (!take(kBarKFull)) break;
           const uint32_t a0 = sbase + kOffQ + ch * kBoxBytes;
-          const uint32_t b0 = sbase + kOffRing + slot * kStageBytes;
+          const uint32_t b0 = sbase + kOffKRing + rg.slot * kStageBytes;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_pair_ss(d, smem_desc_sw128(a0 + 32 * k, 16, 1024), smem_desc_sw128(b0 + 32 * k, 16, 1024),
-                        kIdescQK, (ch | k) != 0);
-          release();
+            mma_pair_ss(d, smem_desc_sw128(a0 + 32 * k, 16, 1024), smem_desc_sw128(b0 + 32 * k, 16, 1024), kIdescQK,
+                        (ch | k) != 0);
+          mma_commit_pair_mc(bar(kBarKEmpty + rg.slot), 0x3);
+          if (++rg.slot == kKStages) { rg.slot = 0; rg.phase ^= 1u; }
         }
-        mma_commit_pair_mc(bar(kBarSFull + sb), 0x3);
-      };
-      auto pv = [&](int t) {
-        if (ok && !mbar_wait(bar(kBarPFull), (uint32_t)(t & 1), abort)) ok = false;
+        if (ok) mma_commit_pair_mc(bar(kBarSFull + sb), 0x3);
+      }
+    } else {
+      // P.V into the two 128-column output blocks
+      for (int t = 0; t < u.T && ok; ++t) {
+        if (!mbar_wait(bar(kBarPFull), (uint32_t)(t & 1), abort)) { ok = false; break; }
         tc_fence_after();
-        for (int j = 0; j < 2; ++j) {
+        for (int j = 0; j < 2 && ok; ++j) {
           const uint32_t d = tmem + (j ? kColO1 : kColO0);
           for (int g = 0; g < 4; ++g) {
-            if (!take()) return;
+            if (!take(kBarVFull)) break;
             const uint32_t a0 = sbase + kOffP + g * kBoxBytes;
-            const uint32_t b0 = sbase + kOffRing + slot * kStageBytes;
+            const uint32_t b0 = sbase + kOffVRing + rg.slot * kStageBytes;
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               mma_pair_ss(d, smem_desc_sw128(a0 + 32 * k, 16, 1024), smem_desc_sw128(b0 + 2048 * k, kBoxBytes, 1024),
                           kIdescPV, (t > 0 || g > 0 || k > 0) ? 1u : 0u);
-            release();
+            mma_commit_pair_mc(bar(kBarVEmpty + rg.slot), 0x3);
+            if (++rg.slot == kVStages) { rg.slot = 0; rg.phase ^= 1u; }
           }
         }
-        mma_commit_pair_mc(bar(kBarOFull), 0x3);
-      };
-      if (ok) {
-        qk(0);
-        for (int t = 1; t < u.T && ok; ++t) {
-          qk(t);
-          pv(t - 1);
-        }
-        if (ok) pv(u.T - 1);
+        if (ok) mma_commit_pair_mc(bar(kBarOFull), 0x3);
       }
     }
   } else if (warp >= 4) {
     // ============================================================ softmax
+    // warp w reads TMEM lane quarter w % 4; lane l holds one row (l % 64) and
+    // one half of the tile's keys / output dims (l / 64); the two warps of a
+    // quarter split that half again (sub): each thread owns one 64-key group
+    // of S / P and one of the two 128-column output accumulators.
     const int q4 = warp & 3;
-    const int l = 32 * q4 + lane;        // TMEM lane
+    const int sub = (warp - 4) >> 2;
+    const int l = 32 * q4 + lane;          // TMEM lane
     const int rho = l & 63, eta = l >> 6;  // row within CTA, key / dim half
+    const int grp = 2 * eta + sub;         // 64-key group of the tile (= P chunk)
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16);
+    const uint32_t o_col = sub ? kColO1 : kColO0;
     const uint32_t* mw = s_mask + rho * kMaxW;
     float* red = reinterpret_cast<float*>(smem + kOffRed);
     float* lred = reinterpret_cast<float*>(smem + kOffLred);
     const uint32_t sempty0 = map_to_rank(bar(kBarSEmpty), 0);
     const uint32_t pfull0 = map_to_rank(bar(kBarPFull), 0);
-    unsigned char* prow = smem + kOffP + rho * 128;
+    unsigned char* pchunk = smem + kOffP + grp * kBoxBytes + rho * 128;
+    const float sl2 = p.scale_log2;
     float m_used = -INFINITY, lsum = 0.0f;
     bool ok = true;
     // every thread runs all T iterations (and so every named barrier) even
@@ -387,38 +410,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int sb = t & 1;
       if (ok && !mbar_wait(bar(kBarSFull + sb), (uint32_t)((t >> 1) & 1), abort)) ok = false;
       tc_fence_after();
-      float s[128];
+      float s[64];
       {
-        uint32_t r[32];
+        uint32_t r0[32], r1[32];
+        const uint32_t a = lane_addr + (sb ? kColS1 : kColS0) + 64 * sub;
+        tmem_ld32(a, r0);
+        tmem_ld32(a + 32, r1);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(lane_addr + (sb ? kColS1 : kColS0) + 32 * c, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[i]);
+        for (int i = 0; i < 32; ++i) {
+          s[i] = __uint_as_float(r0[i]);
+          s[32 + i] = __uint_as_float(r1[i]);
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(sempty0 + 8u * (uint32_t)sb);
-      // mask + scale + local max over this thread's 128 keys (2 groups of 64)
-      const int tile0 = u.kb + t * kTileKeys;
-      float mloc = -INFINITY;
+      if (lane == 0) {
+        if (leader) mbar_arrive_local(bar(kBarSEmpty + sb));
+        else mbar_arrive_cluster(sempty0 + 8u * (uint32_t)sb);
+      }
+      // visibility of this thread's 64 keys; the common case (all committed
+      // cache keys, none cut by the unit's range) needs no per-key work
+      const int g0 = u.kb + t * kTileKeys + 64 * grp;
+      const int kw = group_window(g0, u.nkeys);
+      const uint64_t vis = group_visibility(kw, g0, u.ke, u.L, mw, p.W);
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+      if (vis == ~0ull) {
 #pragma unroll
-      for (int gg = 0; gg < 2; ++gg) {
-        const int g0 = tile0 + 128 * eta + 64 * gg;
-        const int kw = group_window(g0, u.nkeys);
-        const uint64_t vis = group_visibility(kw, g0, u.ke, u.L, mw, p.W);
+        for (int c = 0; c < 64; c += 4) {
+          mx0 = fmaxf(mx0, s[c]);
+          mx1 = fmaxf(mx1, s[c + 1]);
+          mx2 = fmaxf(mx2, s[c + 2]);
+          mx3 = fmaxf(mx3, s[c + 3]);
+        }
+      } else {
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float v = ((vis >> c) & 1ull) ? s[64 * gg + c] * p.scale_log2 : -INFINITY;
-          s[64 * gg + c] = v;
-          mloc = fmaxf(mloc, v);
+          const float v = ((vis >> c) & 1ull) ? s[c] : -INFINITY;
+          s[c] = v;
+          if ((c & 3) == 0) mx0 = fmaxf(mx0, v);
+          if ((c & 3) == 1) mx1 = fmaxf(mx1, v);
+          if ((c & 3) == 2) mx2 = fmaxf(mx2, v);
+          if ((c & 3) == 3) mx3 = fmaxf(mx3, v);
         }
       }
-      red[(sb * 2 + eta) * 64 + rho] = mloc;
-      named_bar_sync(1, 128);
-      const float mtile = fmaxf(mloc, red[(sb * 2 + (eta ^ 1)) * 64 + rho]);
+      const float mloc = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;  // scale > 0 keeps the max
+      float* rt = red + sb * 4 * 64;
+      rt[grp * 64 + rho] = mloc;
+      named_bar_sync(1, 32 * kSoftmaxWarps);
+      const float mtile = fmaxf(fmaxf(rt[rho], rt[64 + rho]), fmaxf(rt[128 + rho], rt[192 + rho]));
       const float m_new = fmaxf(m_used, mtile);
       bool rescale = false;
       float alpha = 1.0f;
@@ -430,18 +470,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         rescale = true;
       }
       const float mref = (m_used == -INFINITY) ? 0.0f : m_used;
-      // probabilities, row sum, bf16 pack
-      uint32_t pk[64];
-      float part = 0.0f;
+      // probabilities (p = 2^(s * scale * log2e - m)), row sum, bf16 pack
+      uint32_t pk[32];
+      float ps0 = 0.0f, ps1 = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float p0 = exp2f(s[2 * i] - mref);
-        const float p1 = exp2f(s[2 * i + 1] - mref);
-        part += p0 + p1;
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = exp2f(fmaf(s[2 * i], sl2, -mref));
+        const float p1 = exp2f(fmaf(s[2 * i + 1], sl2, -mref));
+        ps0 += p0;
+        ps1 += p1;
         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk[i] = *reinterpret_cast<uint32_t*>(&h2);
       }
-      lsum = lsum * alpha + part;
+      lsum = lsum * alpha + (ps0 + ps1);
       // the P buffer and the output accumulator are free once PV(t-1) is done
       if (t > 0) {
         if (ok && !mbar_wait(bar(kBarOFull), (uint32_t)((t - 1) & 1), abort)) ok = false;
@@ -449,42 +490,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (rescale) {
 #pragma unroll 1
-        for (int j = 0; j < 2; ++j)
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            const uint32_t a = lane_addr + (j ? kColO1 : kColO0) + 32 * c;
-            tmem_ld32(a, r);
-            tmem_wait_ld();
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          const uint32_t a = lane_addr + o_col + 32 * c;
+          tmem_ld32(a, r);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(a, r);
-          }
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(a, r);
+        }
         tmem_wait_st();
       }
-      // P row: keys [128 eta, 128 eta + 128) = chunks 2 eta, 2 eta + 1, 128-byte swizzle
+      // P row segment: 64 keys = 8 x 16 bytes, 128-byte swizzle
 #pragma unroll
-      for (int gg = 0; gg < 2; ++gg) {
-        unsigned char* chunk = prow + (2 * eta + gg) * kBoxBytes;
-#pragma unroll
-        for (int u16 = 0; u16 < 8; ++u16) {
-          const int pos = u16 ^ (rho & 7);
-          uint4 v = make_uint4(pk[32 * gg + 4 * u16 + 0], pk[32 * gg + 4 * u16 + 1], pk[32 * gg + 4 * u16 + 2],
-                               pk[32 * gg + 4 * u16 + 3]);
-          *reinterpret_cast<uint4*>(chunk + pos * 16) = v;
-        }
+      for (int u16 = 0; u16 < 8; ++u16) {
+        const int pos = u16 ^ (rho & 7);
+        *reinterpret_cast<uint4*>(pchunk + pos * 16) =
+            make_uint4(pk[4 * u16 + 0], pk[4 * u16 + 1], pk[4 * u16 + 2], pk[4 * u16 + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(pfull0);
+      if (lane == 0) {
+        if (leader) mbar_arrive_local(bar(kBarPFull));
+        else mbar_arrive_cluster(pfull0);
+      }
     }
     // ---------------------------------------------------------- epilogue
     if (ok) ok = mbar_wait(bar(kBarOFull), (uint32_t)((u.T - 1) & 1), abort);
     tc_fence_after();
-    lred[eta * 64 + rho] = lsum;
-    named_bar_sync(1, 128);
-    const float ltot = lsum + lred[(eta ^ 1) * 64 + rho];
+    lred[grp * 64 + rho] = lsum;
+    named_bar_sync(1, 32 * kSoftmaxWarps);
+    const float ltot = (lred[rho] + lred[64 + rho]) + (lred[128 + rho] + lred[192 + rho]);
     const int rr = row0 + rho;
     const bool in_range = rr < req_rows;
     const bool real_row = ok && in_range && (rr / p.H) < u.n;
@@ -493,43 +530,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const size_t grow = (size_t)u.b * req_rows + rr;
     const float inv = !real_row ? 0.0f : ((p.splits == 1 && ltot > 0.0f) ? 1.0f / ltot : 1.0f);
 #pragma unroll 1
-    for (int j = 0; j < 2; ++j) {
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(lane_addr + (j ? kColO1 : kColO0) + 32 * c, r);
-        tmem_wait_ld();
-        if (!write_row) continue;
-        const int d0 = 256 * j + 128 * eta + 32 * c;  // first output dim of this chunk
-        if (p.splits > 1) {
-          float4* dst = reinterpret_cast<float4*>(p.part_o + ((size_t)u.split * rows_total + grow) * kDL + d0);
+    for (int c = 0; c < 4; ++c) {
+      uint32_t r[32];
+      tmem_ld32(lane_addr + o_col + 32 * c, r);
+      tmem_wait_ld();
+      if (!write_row) continue;
+      const int d0 = 256 * sub + 128 * eta + 32 * c;  // first output dim of this chunk
+      if (p.splits > 1) {
+        float4* dst = reinterpret_cast<float4*>(p.part_o + ((size_t)u.split * rows_total + grow) * kDL + d0);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                 __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-        } else if (p.out_dtype == DDT_F32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + grow * kDL + d0);
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                               __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+      } else if (p.out_dtype == DDT_F32) {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + grow * kDL + d0);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
-                                 __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + grow * kDL + d0);
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
+                               __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv);
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + grow * kDL + d0);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t w[4];
+        for (int i = 0; i < 4; ++i) {
+          uint32_t w[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[8 * i + 2 * k]) * inv,
-                                                        __uint_as_float(r[8 * i + 2 * k + 1]) * inv);
-              w[k] = *reinterpret_cast<uint32_t*>(&h2);
-            }
-            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int k = 0; k < 4; ++k) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[8 * i + 2 * k]) * inv,
+                                                      __uint_as_float(r[8 * i + 2 * k + 1]) * inv);
+            w[k] = *reinterpret_cast<uint32_t*>(&h2);
           }
+          dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
     }
-    if (write_row && eta == 0) {
+    if (write_row && grp == 0) {
       if (p.splits > 1) {
         p.part_ml[((size_t)u.split * rows_total + grow) * 2 + 0] = m_used;
         p.part_ml[((size_t)u.split * rows_total + grow) * 2 + 1] = ltot;
