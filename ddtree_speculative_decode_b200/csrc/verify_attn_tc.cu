@@ -18,11 +18,16 @@
 //  * Key tiles are 256 keys. QK: N = 256 keys (each CTA supplies 128 keys'
 //    576-d rows through TMA), K-steps of 16 over 576 dims. PV: two MMAs with
 //    N = 256 output dims each (each CTA supplies 128 dims of the latent rows,
-//    read MN-major from the same TMA tiles layout), K = 256 keys.
-//  * Warp roles per CTA: warps 0 / 2 = TMA producers of the key ring and the
-//    value ring (both CTAs load their halves into their own shared memory,
-//    completion counted on the leader CTA's barriers), warps 1 / 3 = the QK
-//    and PV MMA issuers (leader CTA only; warp 1 also allocates TMEM),
+//    read MN-major from the same TMA tile layout), K = 256 keys.
+//  * Both rings hand the tensor pipe 8 MMAs per stage release: a
+//    tcgen05.commit or an mbarrier wait in an issuing thread costs the pipe
+//    up to ~90 ns unless enough MMAs are queued around it.
+//  * Warp roles per CTA: warps 0 / 2 = TMA producers of the QK ring (query
+//    and key chunks; the query is re-streamed with every key tile so shared
+//    memory holds deeper rings) and of the value ring (both CTAs load their
+//    halves into their own shared memory, completion counted on the leader
+//    CTA's barriers), warps 1 / 3 = the QK and PV MMA issuers (leader CTA
+//    only; warp 1 also allocates TMEM),
 //    warps 4..11 = softmax (TMEM lane quarter = warp % 4, two warps per
 //    quarter; thread = one query row x one 64-key group of the tile, and one
 //    of the row's two 128-dim output accumulator blocks).
@@ -57,9 +62,7 @@ using namespace sm100;
 constexpr int kDL = 512, kDR = 64, kDQK = 576;
 constexpr int kChunks = kDQK / 64;          // 9 column chunks of 64 (128 bytes)
 constexpr int kTileKeys = 256;              // keys per tile
-constexpr int kStageBytes = 16384;          // 2 TMA boxes of 64 x 128 B
 constexpr int kBoxBytes = 8192;
-constexpr int kQBytes = kChunks * kBoxBytes;  // 73728
 constexpr int kPBytes = 4 * kBoxBytes;        // 64 rows x 256 keys bf16
 constexpr int kMaxW = 8;                      // mask words per row (N <= 256)
 constexpr int kSoftmaxWarps = 8;               // warps 4..11, two per SM sub-partition
@@ -67,23 +70,26 @@ constexpr int kThreads = 32 * (4 + kSoftmaxWarps);
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 // shared memory map (bytes from the 1024-aligned base)
-constexpr int kKStages = 3;                    // K ring (QK operand B)
-constexpr int kVStages = 3;                    // V ring (PV operand B)
-constexpr int kOffQ = 0;
-constexpr int kOffKRing = kOffQ + kQBytes;
-constexpr int kOffVRing = kOffKRing + kKStages * kStageBytes;
-constexpr int kOffP = kOffVRing + kVStages * kStageBytes;
+// QK ring: one stage = this CTA's Q chunk (64 rows x 64 dims, 8 KB) + K chunk
+// (128 keys x 64 dims, 16 KB); stages are released in pairs (8 MMAs / commit).
+// V ring: one stage = 64 keys x both 128-dim output blocks (4 boxes, 32 KB).
+constexpr int kKStages = 4;
+constexpr int kKStageBytes = 3 * kBoxBytes;    // 24 KB
+constexpr int kVStages = 2;
+constexpr int kVStageBytes = 4 * kBoxBytes;    // 32 KB
+constexpr int kOffKRing = 0;
+constexpr int kOffVRing = kOffKRing + kKStages * kKStageBytes;
+constexpr int kOffP = kOffVRing + kVStages * kVStageBytes;
 constexpr int kOffMisc = kOffP + kPBytes;
 // misc: barriers (8 B each)
-constexpr int kBarKFull = 0;                     // [kKStages] leader: TMA bytes of both CTAs
-constexpr int kBarKEmpty = kBarKFull + kKStages; // [kKStages] each CTA: QK MMAs done with the stage
-constexpr int kBarVFull = kBarKEmpty + kKStages; // [kVStages]
-constexpr int kBarVEmpty = kBarVFull + kVStages; // [kVStages]
-constexpr int kBarQ = kBarVEmpty + kVStages;     // leader: Q bytes
-constexpr int kBarSFull = kBarQ + 1;             // [2] each CTA: S buffer written
-constexpr int kBarSEmpty = kBarSFull + 2;        // [2] leader: S buffer read (softmax warps of both CTAs)
-constexpr int kBarPFull = kBarSEmpty + 2;        // leader: P written (softmax warps of both CTAs)
-constexpr int kBarOFull = kBarPFull + 1;         // each CTA: PV finished
+constexpr int kBarKFull = 0;                          // [kKStages / 2] leader: TMA bytes of a stage pair, both CTAs
+constexpr int kBarKEmpty = kBarKFull + kKStages / 2;  // [kKStages / 2] each CTA: QK MMAs done with a stage pair
+constexpr int kBarVFull = kBarKEmpty + kKStages / 2;  // [kVStages]
+constexpr int kBarVEmpty = kBarVFull + kVStages;      // [kVStages]
+constexpr int kBarSFull = kBarVEmpty + kVStages;      // [2] each CTA: S buffer written
+constexpr int kBarSEmpty = kBarSFull + 2;             // [2] leader: S buffer read (softmax warps of both CTAs)
+constexpr int kBarPFull = kBarSEmpty + 2;             // leader: P written (softmax warps of both CTAs)
+constexpr int kBarOFull = kBarPFull + 1;              // each CTA: PV finished
 constexpr int kNumBars = kBarOFull + 1;
 constexpr int kOffRed = kOffMisc + 256;                 // float [2 parity][4 groups][64]
 constexpr int kOffLred = kOffRed + 2 * 4 * 64 * 4;      // float [4][64]
@@ -92,6 +98,7 @@ constexpr int kOffTmem = kOffMask + 64 * kMaxW * 4;     // uint32
 constexpr int kSmemBytes = kOffTmem + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;           // slack for 1024 alignment
 static_assert(kNumBars * 8 <= 256, "barrier area");
+static_assert(kKStages % 2 == 0, "QK stages are released in pairs");
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
 // TMEM columns
@@ -229,7 +236,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kKStages; ++s) {
+    for (int s = 0; s < kKStages / 2; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
       mbar_init(bar(kBarKEmpty + s), 1);
     }
@@ -237,7 +244,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(bar(kBarVFull + s), 1);
       mbar_init(bar(kBarVEmpty + s), 1);
     }
-    mbar_init(bar(kBarQ), 1);
     mbar_init(bar(kBarSFull + 0), 1);
     mbar_init(bar(kBarSFull + 1), 1);
     mbar_init(bar(kBarSEmpty + 0), 2 * kSoftmaxWarps);
@@ -277,54 +283,73 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int slot = 0;
     uint32_t phase = 0;
   };
-  if ((warp == 0 || warp == 2) && lane == 0) {
-    // ============================================================ producers
-    const bool kprod = warp == 0;
-    const int nst = kprod ? kKStages : kVStages;
-    const int off = kprod ? kOffKRing : kOffVRing;
-    const int fb0 = kprod ? kBarKFull : kBarVFull;
-    const int eb0 = kprod ? kBarKEmpty : kBarVEmpty;
-    const uint32_t full0 = map_to_rank(bar(fb0), 0);
+  if (warp == 0 && lane == 0) {
+    // ============================================================ QK producer
+    // per tile and 64-dim chunk: this CTA's Q chunk and its 128 keys' chunk
+    const uint32_t full0 = map_to_rank(bar(kBarKFull), 0);
     Ring rg;
-    bool ok = true;
-    auto next_stage = [&](auto&& issue) {
-      if (!ok) return;
-      if (!mbar_wait(bar(eb0 + rg.slot), rg.phase ^ 1u, abort)) { ok = false; return; }
-      if (leader) mbar_arrive_expect_tx(bar(fb0 + rg.slot), 2u * kStageBytes);
-      issue(sbase + off + rg.slot * kStageBytes, full0 + 8u * (uint32_t)rg.slot);
-      if (++rg.slot == nst) { rg.slot = 0; rg.phase ^= 1u; }
-    };
-    if (kprod) {
-      // Q: this CTA's 64 rows x 9 chunks, then every tile's 9 key chunks
-      const uint32_t q_bar = map_to_rank(bar(kBarQ), 0);
-      if (leader) mbar_arrive_expect_tx(bar(kBarQ), 2u * kQBytes);
-      const int qrow = u.b * req_rows + row0;
-      for (int ch = 0; ch < kChunks; ++ch)
-        tma_load_2d_pair(sbase + kOffQ + ch * kBoxBytes, &tm_q, ch * 64, qrow, q_bar);
-      for (int t = 0; t < u.T && ok; ++t) {
-        const int tile0 = u.kb + t * kTileKeys;
-        const int y0 = u.off_row + group_window(tile0 + 128 * (int)rank, u.nkeys);
-        const int y1 = u.off_row + group_window(tile0 + 128 * (int)rank + 64, u.nkeys);
-        for (int ch = 0; ch < kChunks; ++ch)
-          next_stage([&](uint32_t dst, uint32_t fb) {
-            tma_load_2d_pair(dst, &tm_kv, ch * 64, y0, fb);
-            tma_load_2d_pair(dst + kBoxBytes, &tm_kv, ch * 64, y1, fb);
-          });
-      }
-    } else {
-      // every tile's value rows: two 128-dim blocks x four 64-key groups
-      for (int t = 0; t < u.T && ok; ++t) {
-        const int tile0 = u.kb + t * kTileKeys;
-        for (int j = 0; j < 2; ++j)
-          for (int g = 0; g < 4; ++g) {
-            const int y = u.off_row + group_window(tile0 + 64 * g, u.nkeys);
-            const int x = 256 * j + 128 * (int)rank;
-            next_stage([&](uint32_t dst, uint32_t fb) {
-              tma_load_2d_pair(dst, &tm_kv, x, y, fb);
-              tma_load_2d_pair(dst + kBoxBytes, &tm_kv, x + 64, y, fb);
-            });
+    const int qrow = u.b * req_rows + row0;
+    for (int t = 0; t < u.T; ++t) {
+      const int tile0 = u.kb + t * kTileKeys;
+      const int y0 = u.off_row + group_window(tile0 + 128 * (int)rank, u.nkeys);
+      const int y1 = u.off_row + group_window(tile0 + 128 * (int)rank + 64, u.nkeys);
+      bool ok = true;
+      for (int ch = 0; ch < kChunks; ++ch) {
+        if ((rg.slot & 1) == 0) {
+          if (!mbar_wait(bar(kBarKEmpty + (rg.slot >> 1)), rg.phase ^ 1u, abort)) {
+            ok = false;
+            break;
           }
+          // one barrier per stage pair; the pair is always filled completely
+          // (the last pair of the unit may get a duplicate stage, see below)
+          if (leader) mbar_arrive_expect_tx(bar(kBarKFull + (rg.slot >> 1)), 4u * kKStageBytes);
+        }
+        const uint32_t dst = sbase + kOffKRing + rg.slot * kKStageBytes;
+        const uint32_t fb = full0 + 8u * (uint32_t)(rg.slot >> 1);
+        tma_load_2d_pair(dst, &tm_q, ch * 64, qrow, fb);
+        tma_load_2d_pair(dst + kBoxBytes, &tm_kv, ch * 64, y0, fb);
+        tma_load_2d_pair(dst + 2 * kBoxBytes, &tm_kv, ch * 64, y1, fb);
+        if (++rg.slot == kKStages) { rg.slot = 0; rg.phase ^= 1u; }
       }
+      if (!ok) break;
+    }
+    if (rg.slot & 1) {
+      // odd number of stages: complete the last pair's byte count with a
+      // repeat of the last Q box + key boxes (never consumed)
+      const int tile0 = u.kb + (u.T - 1) * kTileKeys;
+      const int y0 = u.off_row + group_window(tile0 + 128 * (int)rank, u.nkeys);
+      const int y1 = u.off_row + group_window(tile0 + 128 * (int)rank + 64, u.nkeys);
+      const uint32_t dst = sbase + kOffKRing + rg.slot * kKStageBytes;
+      const uint32_t fb = full0 + 8u * (uint32_t)(rg.slot >> 1);
+      tma_load_2d_pair(dst, &tm_q, (kChunks - 1) * 64, qrow, fb);
+      tma_load_2d_pair(dst + kBoxBytes, &tm_kv, (kChunks - 1) * 64, y0, fb);
+      tma_load_2d_pair(dst + 2 * kBoxBytes, &tm_kv, (kChunks - 1) * 64, y1, fb);
+    }
+  } else if (warp == 2 && lane == 0) {
+    // ============================================================ V producer
+    // per tile and 64-key group: this CTA's two 128-dim value blocks
+    const uint32_t full0 = map_to_rank(bar(kBarVFull), 0);
+    Ring rg;
+    const int x = 128 * (int)rank;
+    for (int t = 0; t < u.T; ++t) {
+      const int tile0 = u.kb + t * kTileKeys;
+      bool ok = true;
+      for (int g = 0; g < 4; ++g) {
+        if (!mbar_wait(bar(kBarVEmpty + rg.slot), rg.phase ^ 1u, abort)) {
+          ok = false;
+          break;
+        }
+        if (leader) mbar_arrive_expect_tx(bar(kBarVFull + rg.slot), 2u * kVStageBytes);
+        const int y = u.off_row + group_window(tile0 + 64 * g, u.nkeys);
+        const uint32_t dst = sbase + kOffVRing + rg.slot * kVStageBytes;
+        const uint32_t fb = full0 + 8u * (uint32_t)rg.slot;
+        tma_load_2d_pair(dst, &tm_kv, x, y, fb);
+        tma_load_2d_pair(dst + kBoxBytes, &tm_kv, x + 64, y, fb);
+        tma_load_2d_pair(dst + 2 * kBoxBytes, &tm_kv, x + 256, y, fb);
+        tma_load_2d_pair(dst + 3 * kBoxBytes, &tm_kv, x + 320, y, fb);
+        if (++rg.slot == kVStages) { rg.slot = 0; rg.phase ^= 1u; }
+      }
+      if (!ok) break;
     }
   } else if ((warp == 1 || warp == 3) && lane == 0 && leader) {
     // ============================================================ MMA issuers
@@ -332,14 +357,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     Ring rg;
     // stage data comes from TMA (async proxy to async proxy): the mbarrier
     // wait alone orders it before the MMAs, no tcgen05 fence needed
-    auto take = [&](int fb0) -> bool {
-      if (!ok) return false;
-      if (!mbar_wait(bar(fb0 + rg.slot), rg.phase, abort)) { ok = false; return false; }
-      return true;
-    };
     if (warp == 1) {
-      // QK^T into the two S buffers
-      if (!mbar_wait(bar(kBarQ), 0, abort)) ok = false;
+      // Q.K^T into the two S buffers
       for (int t = 0; t < u.T && ok; ++t) {
         const int sb = t & 1;
         if (t >= 2) {
@@ -348,14 +367,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         const uint32_t d = tmem + (sb ? kColS1 : kColS0);
         for (int ch = 0; ch < kChunks; ++ch) {
-          if (!take(kBarKFull)) break;
-          const uint32_t a0 = sbase + kOffQ + ch * kBoxBytes;
-          const uint32_t b0 = sbase + kOffKRing + rg.slot * kStageBytes;
+          if ((rg.slot & 1) == 0 && !mbar_wait(bar(kBarKFull + (rg.slot >> 1)), rg.phase, abort)) { ok = false; break; }
+          const uint32_t a0 = sbase + kOffKRing + rg.slot * kKStageBytes;
+          const uint32_t b0 = a0 + kBoxBytes;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_pair_ss(d, smem_desc_sw128(a0 + 32 * k, 16, 1024), smem_desc_sw128(b0 + 32 * k, 16, 1024), kIdescQK,
                         (ch | k) != 0);
-          mma_commit_pair_mc(bar(kBarKEmpty + rg.slot), 0x3);
+          if (rg.slot & 1) mma_commit_pair_mc(bar(kBarKEmpty + (rg.slot >> 1)), 0x3);
           if (++rg.slot == kKStages) { rg.slot = 0; rg.phase ^= 1u; }
         }
         if (ok) mma_commit_pair_mc(bar(kBarSFull + sb), 0x3);
@@ -365,19 +384,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int t = 0; t < u.T && ok; ++t) {
         if (!mbar_wait(bar(kBarPFull), (uint32_t)(t & 1), abort)) { ok = false; break; }
         tc_fence_after();
-        for (int j = 0; j < 2 && ok; ++j) {
-          const uint32_t d = tmem + (j ? kColO1 : kColO0);
-          for (int g = 0; g < 4; ++g) {
-            if (!take(kBarVFull)) break;
-            const uint32_t a0 = sbase + kOffP + g * kBoxBytes;
-            const uint32_t b0 = sbase + kOffVRing + rg.slot * kStageBytes;
+        for (int g = 0; g < 4; ++g) {
+          if (!mbar_wait(bar(kBarVFull + rg.slot), rg.phase, abort)) { ok = false; break; }
+          const uint32_t a0 = sbase + kOffP + g * kBoxBytes;
+          const uint32_t b0 = sbase + kOffVRing + rg.slot * kVStageBytes;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const uint32_t d = tmem + (j ? kColO1 : kColO0);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              mma_pair_ss(d, smem_desc_sw128(a0 + 32 * k, 16, 1024), smem_desc_sw128(b0 + 2048 * k, kBoxBytes, 1024),
-                          kIdescPV, (t > 0 || g > 0 || k > 0) ? 1u : 0u);
-            mma_commit_pair_mc(bar(kBarVEmpty + rg.slot), 0x3);
-            if (++rg.slot == kVStages) { rg.slot = 0; rg.phase ^= 1u; }
+              mma_pair_ss(d, smem_desc_sw128(a0 + 32 * k, 16, 1024),
+                          smem_desc_sw128(b0 + 2 * j * kBoxBytes + 2048 * k, kBoxBytes, 1024), kIdescPV,
+                          (t > 0 || g > 0 || k > 0) ? 1u : 0u);
           }
+          mma_commit_pair_mc(bar(kBarVEmpty + rg.slot), 0x3);
+          if (++rg.slot == kVStages) { rg.slot = 0; rg.phase ^= 1u; }
         }
         if (ok) mma_commit_pair_mc(bar(kBarOFull), 0x3);
       }
