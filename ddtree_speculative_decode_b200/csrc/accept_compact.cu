@@ -20,6 +20,8 @@
 //    copying rows in increasing j is already read-before-write per byte; the
 //    CTA still stages groups of rows in registers behind a barrier so many rows
 //    are in flight at once.
+#include <mutex>
+
 #include "ddt_kernels.cuh"
 
 namespace ddt {
@@ -292,6 +294,52 @@ int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream) 
   const unsigned grid = (unsigned)p.chunks * (unsigned)(p.B * p.N);
   if (p.logits_dtype == DDT_BF16) return launch_pdl(accept_kernel<true>, grid, kArgmaxThreads, 0, stream, p);
   return launch_pdl(accept_kernel<false>, grid, kArgmaxThreads, 0, stream, p);
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant: the same kernel, with its scratch (per-request
+// arrival counters + partial argmax keys) in a fixed device array that is part
+// of the loaded library instead of a caller-provided workspace.
+// ---------------------------------------------------------------------------
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB on every device that loads the library
+static __device__ __align__(256) unsigned char g_accept_scratch[kNoAllocScratchBytes];
+
+size_t accept_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+// Device address of g_accept_scratch, looked up once per device (with that
+// device current). Host code must not hand the symbol itself to a kernel: on
+// the host it names a stand-in, not device memory.
+static void* noalloc_scratch_ptr(int* status) {
+  static std::mutex mu;
+  static void* ptrs[128] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) {
+    *status = DDT_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_accept_scratch) != cudaSuccess || ptr == nullptr) {
+      *status = DDT_ERR_CUDA;
+      return nullptr;
+    }
+    ptrs[dev] = ptr;
+  }
+  *status = DDT_OK;
+  return ptrs[dev];
+}
+
+int launch_accept_compact_noalloc(AcceptParams p, cudaStream_t stream) {
+  if (accept_workspace_bytes(p.B, p.N, p.V) > kNoAllocScratchBytes) return DDT_ERR_UNSUPPORTED;
+  int st = DDT_OK;
+  void* scratch = noalloc_scratch_ptr(&st);
+  if (st != DDT_OK) return st;
+  // the counters must start at zero; the array keeps whatever the last call
+  // (on any stream) left there, so clear them on this call's stream first
+  if (cudaMemsetAsync(scratch, 0, counter_bytes(p.B), stream) != cudaSuccess) return DDT_ERR_CUDA;
+  return launch_accept_compact(p, scratch, stream);
 }
 
 }  // namespace ddt

@@ -134,4 +134,47 @@ int ddt_accept_compact(const void* logits, int logits_dtype, int V, const int32_
   return ddt::launch_accept_compact(p, workspace, stream);
 }
 
+int ddt_accept_compact_noalloc(const void* logits, int logits_dtype, int V, const int32_t* node_tok,
+                               const int32_t* parent, const int32_t* n_nodes, int B, int N, void* kv, int kv_dtype,
+                               int row_elems, int n_layers, int64_t layer_stride_rows, const int64_t* cache_off,
+                               int32_t* cache_len, const int32_t* cache_cap, int32_t* am, int32_t* acc_len,
+                               int32_t* acc_nodes, int32_t* out_tok, int32_t* bonus, int32_t* dev_status,
+                               cudaStream_t stream) {
+  if (!logits || !node_tok || !parent || !n_nodes || !kv || !cache_off || !cache_len || !cache_cap || !acc_len ||
+      !acc_nodes || !out_tok || !bonus)
+    return DDT_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || N > 1024 || V < 1 || row_elems < 1 || n_layers < 1 || layer_stride_rows < 0)
+    return DDT_ERR_INVALID_ARG;
+  if (n_layers > 1 && layer_stride_rows < 1) return DDT_ERR_INVALID_ARG;
+  if ((logits_dtype != DDT_F32 && logits_dtype != DDT_BF16) || (kv_dtype != DDT_F32 && kv_dtype != DDT_BF16))
+    return DDT_ERR_INVALID_ARG;
+  const int elt = kv_dtype == DDT_F32 ? 4 : 2;
+  const long long row_bytes = (long long)row_elems * elt;
+  if (row_bytes % 4 != 0 || row_bytes > (1 << 20)) return DDT_ERR_INVALID_ARG;
+  if (!ddt::aligned(kv, 4)) return DDT_ERR_INVALID_ARG;
+  ddt::AcceptParams p{};
+  p.logits = logits;
+  p.logits_dtype = logits_dtype;
+  p.V = V;
+  p.node_tok = node_tok;
+  p.parent = parent;
+  p.n_nodes = n_nodes;
+  p.B = B;
+  p.N = N;
+  p.kv = static_cast<unsigned char*>(kv);
+  p.row_bytes = (int)row_bytes;
+  p.n_layers = n_layers;
+  p.layer_stride_bytes = layer_stride_rows * row_bytes;
+  p.cache_off = cache_off;
+  p.cache_len = cache_len;
+  p.cache_cap = cache_cap;
+  p.am = am;
+  p.acc_len = acc_len;
+  p.acc_nodes = acc_nodes;
+  p.out_tok = out_tok;
+  p.bonus = bonus;
+  p.dev_status = dev_status;
+  return ddt::launch_accept_compact_noalloc(p, stream);
+}
+
 }  // extern "C"

@@ -51,6 +51,8 @@ struct AcceptParams {
 };
 size_t accept_workspace_bytes(int B, int N, int V);
 int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream);
+size_t accept_noalloc_scratch_bytes();
+int launch_accept_compact_noalloc(AcceptParams p, cudaStream_t stream);
 
 // ---- verify attention -------------------------------------------------------
 struct AttnParams {

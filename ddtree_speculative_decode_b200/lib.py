@@ -28,6 +28,7 @@ EXPORTS = (
     "ddt_verify_attn",
     "ddt_accept_compact_workspace_size",
     "ddt_accept_compact",
+    "ddt_accept_compact_noalloc",
 )
 
 _lib = None
@@ -66,6 +67,9 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.ddt_accept_compact.restype = i32
     lib.ddt_accept_compact.argtypes = [vp, i32, i32, vp, vp, vp, i32, i32, vp, i32, i32, i32, i64, vp, vp, vp,
                                        vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.ddt_accept_compact_noalloc.restype = i32
+    lib.ddt_accept_compact_noalloc.argtypes = [vp, i32, i32, vp, vp, vp, i32, i32, vp, i32, i32, i32, i64, vp, vp,
+                                               vp, vp, vp, vp, vp, vp, vp, vp]
     if path is None:
         _lib = lib
     return lib
@@ -250,3 +254,30 @@ def alloc_accept(B: int, N: int, device) -> dict:
     return {"am": torch.empty(B, N, **i32), "acc_len": torch.empty(B, **i32),
             "acc_nodes": torch.empty(B, N, **i32), "out_tok": torch.empty(B, N, **i32),
             "bonus": torch.empty(B, **i32), "status": torch.empty(B, **i32)}
+
+
+def accept_compact_noalloc(logits: torch.Tensor, node_tok: torch.Tensor, parent: torch.Tensor,
+                           n_nodes: torch.Tensor, kv: torch.Tensor, cache_off: torch.Tensor, cache_len: torch.Tensor,
+                           cache_cap: torch.Tensor, n_layers: int = 1, layer_stride_rows: int = 0,
+                           out: Optional[dict] = None, stream=None) -> dict:
+    """ddt_accept_compact_noalloc: the same step as accept_compact, for callers
+    that cannot allocate device memory; its scratch is a fixed array inside
+    libddt.so (shared by all calls, so calls must not overlap on the GPU)."""
+    B, N, V = logits.shape
+    _check(logits, "logits", (torch.float32, torch.bfloat16))
+    _check(node_tok, "node_tok", torch.int32, (B, N))
+    _check(parent, "parent", torch.int32, (B, N))
+    _check(n_nodes, "n_nodes", torch.int32, (B,))
+    _check(kv, "kv", (torch.float32, torch.bfloat16))
+    _check(cache_off, "cache_off", torch.int64, (B,))
+    _check(cache_len, "cache_len", torch.int32, (B,))
+    _check(cache_cap, "cache_cap", torch.int32, (B,))
+    if out is None:
+        out = alloc_accept(B, N, logits.device)
+    st = load().ddt_accept_compact_noalloc(_ptr(logits), _dt(logits), V, _ptr(node_tok), _ptr(parent), _ptr(n_nodes),
+                                           B, N, _ptr(kv), _dt(kv), kv.shape[-1], n_layers, layer_stride_rows,
+                                           _ptr(cache_off), _ptr(cache_len), _ptr(cache_cap), _ptr(out["am"]),
+                                           _ptr(out["acc_len"]), _ptr(out["acc_nodes"]), _ptr(out["out_tok"]),
+                                           _ptr(out["bonus"]), _ptr(out["status"]), _stream(stream))
+    _raise("ddt_accept_compact_noalloc", st)
+    return out

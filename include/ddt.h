@@ -222,6 +222,39 @@ DDT_API int ddt_accept_compact(const void* logits, int logits_dtype, int V, cons
                        int32_t* bonus, int32_t* dev_status, void* workspace,
                        size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * ddt_accept_compact_noalloc -- ddt_accept_compact without a workspace.
+ *
+ * No counterpart in the paper: this is a convenience of this library. Some
+ * callers cannot allocate device memory at the point where they verify a
+ * tree -- for example code that is only handed fixed, pre-reserved buffers by
+ * the host application, or a latency-critical decode loop that must not call
+ * cudaMalloc (which can synchronise the device). This entry point takes the
+ * same arguments as ddt_accept_compact minus the workspace and allocates
+ * nothing: its scratch (per-request arrival counters and the partial argmax
+ * keys) lives in one fixed 4 MiB array inside the library, which every GPU
+ * that loads the library keeps until the process exits.
+ *
+ * Limit: ddt_accept_compact_workspace_size(B, N, V) must be at most 4 MiB
+ *   (e.g. B 64 x N 256 x V 163840 needs 1.3 MiB); larger calls return
+ *   DDT_ERR_UNSUPPORTED without launching anything.
+ * Set-up: the first call on each device looks up the array's device address
+ *   (with that device current); make that first call before any stream
+ *   capture.
+ * Sharing: every call on every stream uses the same array, which keeps what
+ *   the last call left in it. Each call first clears the counters it needs on
+ *   its own stream; calls that overlap on the GPU race on the array and give
+ *   wrong results, so serialise them (one stream, or events).
+ * Everything else -- definition, layouts, outputs, device status -- is as for
+ * ddt_accept_compact.
+ */
+DDT_API int ddt_accept_compact_noalloc(const void* logits, int logits_dtype, int V, const int32_t* node_tok,
+                                       const int32_t* parent, const int32_t* n_nodes, int B, int N, void* kv,
+                                       int kv_dtype, int row_elems, int n_layers, int64_t layer_stride_rows,
+                                       const int64_t* cache_off, int32_t* cache_len, const int32_t* cache_cap,
+                                       int32_t* am, int32_t* acc_len, int32_t* acc_nodes, int32_t* out_tok,
+                                       int32_t* bonus, int32_t* dev_status, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -67,3 +67,15 @@ def test_host_validation_without_gpu(so):
     assert st == lib.DDT_ERR_INVALID_ARG
     st = so.ddt_accept_compact(p, 0, 10, p, p, p, 1, 4, p, 0, 8, 1, 0, p, p, p, p, p, p, p, p, p, p, 0, None)
     assert st == lib.DDT_ERR_INVALID_ARG  # workspace too small
+
+
+def test_noalloc_accept_rejects_sizes_beyond_its_array(so):
+    # 64 x 1024 rows x 10 vocab chunks of 8-byte keys = 5.2 MiB > the 4 MiB array:
+    # rejected on the host before anything touches the GPU
+    p = ctypes.c_void_p(256)
+    st = so.ddt_accept_compact_noalloc(p, 1, 163840, p, p, p, 64, 1024, p, 1, 576, 1, 0, p, p, p, p, p, p, p, p, p,
+                                       None)
+    assert st == lib.DDT_ERR_UNSUPPORTED
+    st = so.ddt_accept_compact_noalloc(None, 1, 163840, p, p, p, 1, 64, p, 1, 576, 1, 0, p, p, p, p, p, p, p, p, p,
+                                       None)
+    assert st == lib.DDT_ERR_INVALID_ARG
