@@ -305,7 +305,7 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
     pk = peaks()
     achieved = flops / (attn_ms / 1e3) / 1e12
     peak = pk["bf16_tflops_sustained"]
-    launches_per_step = (1 + attn_launches(shape) + 2)
+    launches_per_step = 1 + attn_launches(shape) + 1  # build, attention, accept (memcpy of cache_len excluded)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
@@ -331,9 +331,8 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
 
 
 def attn_launches(shape: synth.Shape) -> int:
-    from ddtree_speculative_decode_b200 import lib
-    return 2 if lib.verify_attn_workspace_size(shape.B, shape.N, shape.H, shape.d_l, shape.d_r, max(shape.L),
-                                               _tdtype(shape)) > 0 else 1
+    """The verify attention is one launch (split partials merge in-kernel)."""
+    return 1
 
 
 def _tdtype(shape):

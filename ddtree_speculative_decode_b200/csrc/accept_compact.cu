@@ -70,21 +70,31 @@ __global__ void __launch_bounds__(kArgmaxThreads) accept_kernel(AcceptParams p) 
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int e = base + u * kArgmaxThreads + threadIdx.x;
-          if (e < nvec) r[u] = __ldcs(s4 + e);
+          r[u] = e < nvec ? __ldcs(s4 + e) : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
         }
+        // pass 1: the thread's largest value (packed bf16 max, -inf padding)
+        __nv_bfloat162 m2 = __halves2bfloat162(__ushort_as_bfloat16(0xff80), __ushort_as_bfloat16(0xff80));
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-          const int e = base + u * kArgmaxThreads + threadIdx.x;
-          if (e < nvec) {
-            const uint32_t w[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
+          const uint32_t w[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              const int idx = v0 + e * 8 + 2 * t;
-              best = umax64(best, pack_key(__uint_as_float(w[t] << 16), idx));
-              best = umax64(best, pack_key(__uint_as_float(w[t] & 0xffff0000u), idx + 1));
-            }
+          for (int t = 0; t < 4; ++t) m2 = __hmax2(m2, *reinterpret_cast<const __nv_bfloat162*>(&w[t]));
+        }
+        const float mx = fmaxf(__low2float(m2), __high2float(m2));
+        // pass 2: its lowest index (values compare as floats, so -0 == +0)
+        int first = 0x7fffffff;
+#pragma unroll
+        for (int u = U - 1; u >= 0; --u) {
+          const int e = base + u * kArgmaxThreads + threadIdx.x;
+          const uint32_t w[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
+#pragma unroll
+          for (int t = 3; t >= 0; --t) {
+            const int idx = v0 + e * 8 + 2 * t;
+            if (e < nvec && __uint_as_float(w[t] & 0xffff0000u) == mx) first = idx + 1;
+            if (e < nvec && __uint_as_float(w[t] << 16) == mx) first = idx;
           }
         }
+        if (first != 0x7fffffff) best = umax64(best, pack_key(mx, first));
       }
       for (int v = v0 + nvec * 8 + threadIdx.x; v < v1; v += kArgmaxThreads)
         best = umax64(best, pack_key(bf16_bits_to_float(src[v]), v));
@@ -146,6 +156,8 @@ __device__ __noinline__ void walk_compact_body(const AcceptParams& p, int b) {
   const int n = p.n_nodes[b];
   __shared__ int32_t s_am[kMaxN];
   __shared__ int32_t s_path[kMaxN];
+  __shared__ int32_t s_par[kMaxN];
+  __shared__ int32_t s_tok[kMaxN];
   __shared__ int s_a;
   __shared__ int s_skip;
 
@@ -156,25 +168,35 @@ __device__ __noinline__ void walk_compact_body(const AcceptParams& p, int b) {
     s_skip = (n <= 0 || st != DDT_OK);
     if (p.dev_status) p.dev_status[b] = st;
   }
-  // fold partial argmax keys
-  for (int i = threadIdx.x; i < N; i += kWalkThreads) {
-    int a = -1;
+  // fold partial argmax keys: 4 threads per row, each over a strided subset
+  // of the chunks, then a 4-lane shuffle reduce
+  for (int i0 = 0; i0 < N; i0 += kWalkThreads / 4) {
+    const int i = i0 + (threadIdx.x >> 2);
+    const int sub = threadIdx.x & 3;
+    unsigned long long m = 0ull;
     if (i < n) {
       const unsigned long long* pk = p.partial + ((size_t)b * N + i) * p.chunks;
-      unsigned long long m = 0ull;
-      for (int c = 0; c < p.chunks; ++c) m = umax64(m, __ldcg(pk + c));
-      a = static_cast<int>(~static_cast<uint32_t>(m & 0xffffffffull));
+      for (int c = sub; c < p.chunks; c += 4) m = umax64(m, __ldcg(pk + c));
     }
-    s_am[i] = a;
-    if (p.am) p.am[(size_t)b * N + i] = a;
+    m = umax64(m, __shfl_xor_sync(DDT_FULL_MASK, m, 1));
+    m = umax64(m, __shfl_xor_sync(DDT_FULL_MASK, m, 2));
+    if (sub == 0 && i < N) {
+      const int a = i < n ? static_cast<int>(~static_cast<uint32_t>(m & 0xffffffffull)) : -1;
+      s_am[i] = a;
+      if (p.am) p.am[(size_t)b * N + i] = a;
+    }
+  }
+  for (int i = threadIdx.x; i < n; i += kWalkThreads) {
+    s_par[i] = p.parent[(size_t)b * N + i];
+    s_tok[i] = p.node_tok[(size_t)b * N + i];
   }
   __syncthreads();
   const bool skip = s_skip;
   // greedy walk on warp 0
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
-    const int32_t* par = p.parent + (size_t)b * N;
-    const int32_t* tk = p.node_tok + (size_t)b * N;
+    const int32_t* par = s_par;
+    const int32_t* tk = s_tok;
     int a = 0;
     if (!skip) {
       int curn = 0;

@@ -261,25 +261,78 @@ __global__ void __launch_bounds__(32) build_tree_kernel(BuildParams p) {
 }
 
 
-// Same search with the frontier in registers: slot f lives in lane f % 32,
-// register f / 32 (SPL = slots per lane, N <= 32 * SPL). A pop then needs no
-// shared-memory traffic: each lane scans its own registers, the winner's entry
-// is broadcast with shuffles, and only the owner lanes of the (at most two)
-// updated slots write.
+// ---------------------------------------------------------------------------
+// Sorted-frontier variant (the default for N <= 256).
+//
+// The frontier is kept sorted across the warp: entry f lives in lane f % 32,
+// register f / 32, and entry 0 is the best. A pop is "take entry 0"; its (at
+// most two) successors are merged into the remaining entries in one step:
+// two ballots count how many remaining entries beat each successor, which
+// fixes every lane's source (old f+1, old f, old f-1 or a successor), and one
+// shuffle per word moves the entries. Entries that can no longer be popped
+// (beyond the number of pops left) are dropped, which keeps the frontier
+// within min(pops + 1, N - 1 - pops) <= 32 * SPL entries for N <= 64 * SPL.
+//
+// An entry is six 32-bit words: A = order key of the score << 32 | (127 -
+// depth) (larger is better when scores or depths differ), the packed rank
+// tuple k (smaller is better when A ties), aux = last rank << 16 | parent
+// node, and the parent's score ps (for the next sibling's score). The score
+// itself is recovered exactly from A.
+// ---------------------------------------------------------------------------
+struct FEntry {
+  uint64_t A, k;
+  uint32_t aux;
+  float ps;
+};
+
+__device__ __forceinline__ bool fbetter(const FEntry& a, const FEntry& b) {
+  return a.A > b.A || (a.A == b.A && a.k < b.k);
+}
+
+__device__ __forceinline__ float order_key_to_float(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+__device__ __forceinline__ uint64_t entry_key(float sc, int d) {
+  return (static_cast<uint64_t>(float_order_key(sc)) << 32) | static_cast<uint32_t>(127 - d);
+}
+
+__device__ __forceinline__ FEntry fshfl(const FEntry& e, int src) {
+  FEntry o;
+  o.A = __shfl_sync(DDT_FULL_MASK, e.A, src);
+  o.k = __shfl_sync(DDT_FULL_MASK, e.k, src);
+  o.aux = __shfl_sync(DDT_FULL_MASK, e.aux, src);
+  o.ps = __shfl_sync(DDT_FULL_MASK, e.ps, src);
+  return o;
+}
+
+__device__ __forceinline__ FEntry fsel(bool c, const FEntry& a, const FEntry& b) {
+  FEntry o;
+  o.A = c ? a.A : b.A;
+  o.k = c ? a.k : b.k;
+  o.aux = c ? a.aux : b.aux;
+  o.ps = c ? a.ps : b.ps;
+  return o;
+}
+
 template <int SPL>
-__global__ void __launch_bounds__(32) build_tree_reg_kernel(BuildParams p) {
+__global__ void __launch_bounds__(32) build_tree_sorted_kernel(BuildParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   pdl_wait();
   pdl_launch_dependents();
   const int b = blockIdx.x;
   const int lane = threadIdx.x;
-  const int N = p.N, D = p.D, K = p.K, W = p.W;
+  const int N = p.N, D = p.D, K = p.K, W = p.W, bpl = p.bpl;
   int32_t* n_parent = reinterpret_cast<int32_t*>(smem_raw);
-  float* lp = reinterpret_cast<float*>(smem_raw + (size_t)N * 4);
-  int32_t* tk = reinterpret_cast<int32_t*>(smem_raw + (size_t)N * 4 + (size_t)D * K * 4);
+  int32_t* n_dep = n_parent + N;
+  int32_t* n_tok = n_dep + N;
+  float* n_sc = reinterpret_cast<float*>(n_tok + N);
+  float* lp = n_sc + N;
+  int32_t* tk = reinterpret_cast<int32_t*>(lp + D * K);
+  const int L = p.cache_len[b];
+  const int root = p.root_tok[b];
   const bool bad = load_drafter(p, b, lp, tk, lane);
 
-  const int L = p.cache_len[b];
   int32_t* o_tok = p.node_tok + (size_t)b * N;
   int32_t* o_par = p.parent + (size_t)b * N;
   int32_t* o_dep = p.depth + (size_t)b * N;
@@ -289,107 +342,87 @@ __global__ void __launch_bounds__(32) build_tree_reg_kernel(BuildParams p) {
 
   int n = 0;
   if (!bad) {
-    float f_sc[SPL], f_ps[SPL];
-    int f_d[SPL], f_r[SPL], f_p[SPL];
-    uint64_t f_k[SPL];
+    FEntry fr[SPL];
 #pragma unroll
-    for (int q = 0; q < SPL; ++q) {
-      f_sc[q] = 0.0f; f_ps[q] = 0.0f; f_d[q] = 0; f_r[q] = 0; f_p[q] = 0; f_k[q] = 0ull;
-    }
+    for (int q = 0; q < SPL; ++q) fr[q] = FEntry{0ull, 0ull, 0u, 0.0f};
     if (lane == 0) {
-      o_tok[0] = p.root_tok[b];
-      o_par[0] = -1;
-      o_dep[0] = 0;
-      o_pos[0] = L;
-      o_sc[0] = 0.0f;
+      fr[0].A = entry_key(__fadd_rn(0.0f, lp[0]), 1);  // rank 0 at depth 1, parent = root
       n_parent[0] = -1;
-      f_sc[0] = __fadd_rn(0.0f, lp[0]);  // rank 0 at depth 1
-      f_d[0] = 1;
+      n_dep[0] = 0;
+      n_tok[0] = root;
+      n_sc[0] = 0.0f;
     }
     int fsize = (N > 1) ? 1 : 0;
     n = 1;
     while (n < N && fsize > 0) {
-      // lane-local best over this lane's slots
-      int bj = -1;
-      float bs = 0.0f;
-      int bd = 0;
-      uint64_t bk = 0ull;
+      // pop entry 0 (lane 0, register 0)
+      const FEntry w = fshfl(fr[0], 0);
+      const int wd = 127 - static_cast<int>(static_cast<uint32_t>(w.A));
+      const float wsc = order_key_to_float(static_cast<uint32_t>(w.A >> 32));
+      const int wr = static_cast<int>(w.aux >> 16), wpar = static_cast<int>(w.aux & 0xffffu);
+      const int i = n;
+      // successors: first child (rank 0 one level down) and next sibling
+      const bool has_c = wd < D, has_s = wr + 1 < K;
+      const float lc = lp[has_c ? wd * K : 0];
+      const float ls = lp[has_s ? (wd - 1) * K + wr + 1 : 0];
+      const FEntry c{entry_key(__fadd_rn(wsc, lc), wd + 1), w.k << bpl, static_cast<uint32_t>(i), wsc};
+      const FEntry sb{entry_key(__fadd_rn(w.ps, ls), wd), w.k + 1ull, w.aux + 0x10000u, w.ps};
+      if (lane == 0) {
+        n_parent[i] = wpar;
+        n_dep[i] = wd;
+        n_tok[i] = tk[(wd - 1) * K + wr];
+        n_sc[i] = wsc;
+      }
+      const int ns = (int)has_c + (int)has_s;
+      const bool c_first = has_c && (!has_s || fbetter(c, sb));
+      const FEntry s0 = fsel(c_first, c, sb);
+      const FEntry s1 = fsel(c_first, sb, c);
+      // ranks of the successors among the remaining entries (old 1 .. fsize-1)
+      int p0 = 0, p1 = 0;
 #pragma unroll
       for (int q = 0; q < SPL; ++q) {
-        if (32 * q + lane < fsize && (bj < 0 || better(f_sc[q], f_d[q], f_k[q], bs, bd, bk))) {
-          bj = q; bs = f_sc[q]; bd = f_d[q]; bk = f_k[q];
+        const int f = 32 * q + lane;
+        const bool valid = f >= 1 && f < fsize;
+        p0 += __popc(__ballot_sync(DDT_FULL_MASK, valid && fbetter(fr[q], s0)));
+        p1 += __popc(__ballot_sync(DDT_FULL_MASK, valid && fbetter(fr[q], s1)));
+      }
+      if (ns == 0) p0 = 32 * SPL;  // every entry moves up by one
+      // merge: new entry f comes from old f + 1 (f < p0), s0 (f == p0), old f
+      // (between the successors), s1 (f == p1 + 1) or old f - 1 (after both)
+      FEntry nf[SPL];
+#pragma unroll
+      for (int q = 0; q < SPL; ++q) {
+        const int f = 32 * q + lane;
+        const int delta = 1 - (f > p0 ? 1 : 0) - ((ns == 2 && f > p1 + 1) ? 1 : 0);
+        const int src = (lane + delta) & 31;
+        FEntry v = fshfl(fr[q], src);
+        if (q + 1 < SPL) {  // lane 31 moving up reads lane 0 of the next register
+          const FEntry t = fshfl(fr[q + 1 < SPL ? q + 1 : q], src);
+          v = fsel(lane == 31 && delta == 1, t, v);
         }
-      }
-      const int wl = warp_winner(bj >= 0, bs, bd, bk, lane);
-      // the winner's remaining fields
-      float ps_l = 0.0f;
-      int r_l = 0, p_l = 0;
-#pragma unroll
-      for (int q = 0; q < SPL; ++q)
-        if (q == bj) { ps_l = f_ps[q]; r_l = f_r[q]; p_l = f_p[q]; }
-      const int wj = __shfl_sync(DDT_FULL_MASK, bj, wl);
-      const float sc = __shfl_sync(DDT_FULL_MASK, bs, wl);
-      const int dd = __shfl_sync(DDT_FULL_MASK, bd, wl);
-      const uint64_t kk = __shfl_sync(DDT_FULL_MASK, bk, wl);
-      const float psc = __shfl_sync(DDT_FULL_MASK, ps_l, wl);
-      const int rr = __shfl_sync(DDT_FULL_MASK, r_l, wl);
-      const int pp = __shfl_sync(DDT_FULL_MASK, p_l, wl);
-      const int slot = 32 * wj + wl;
-      const int i = n;
-      if (lane == wl) {
-        o_tok[i] = tk[(dd - 1) * K + rr];
-        o_par[i] = pp;
-        o_dep[i] = dd;
-        o_pos[i] = L + dd;
-        o_sc[i] = sc;
-        n_parent[i] = pp;
-      }
-      const bool has_child = dd < D;
-      const bool has_sib = rr + 1 < K;
-      if (has_child && lane == wl) {  // first child takes the popped slot
-        const float cs = __fadd_rn(sc, lp[dd * K]);
-#pragma unroll
-        for (int q = 0; q < SPL; ++q)
-          if (q == wj) { f_sc[q] = cs; f_ps[q] = sc; f_d[q] = dd + 1; f_r[q] = 0; f_p[q] = i; f_k[q] = kk << p.bpl; }
-      }
-      if (has_sib) {  // next sibling: the popped slot, or a new one at the end
-        const int t = has_child ? fsize : slot;
-        if (lane == (t & 31)) {
-          const float ss = __fadd_rn(psc, lp[(dd - 1) * K + rr + 1]);
-          const int tj = t >> 5;
-#pragma unroll
-          for (int q = 0; q < SPL; ++q)
-            if (q == tj) { f_sc[q] = ss; f_ps[q] = psc; f_d[q] = dd; f_r[q] = rr + 1; f_p[q] = pp; f_k[q] = kk + 1ull; }
+        if (q > 0) {  // lane 0 moving down reads lane 31 of the previous register
+          const FEntry t = fshfl(fr[q > 0 ? q - 1 : q], src);
+          v = fsel(lane == 0 && delta == -1, t, v);
         }
-        if (has_child) ++fsize;
+        v = fsel(f == p0, s0, v);
+        v = fsel(ns == 2 && f == p1 + 1, s1, v);
+        nf[q] = v;
       }
-      if (!has_child && !has_sib) {  // remove the popped slot: move the last entry into it
-        const int last = fsize - 1;
-        if (last != slot) {
-          const int ll = last & 31, lj = last >> 5;
-          float m_sc = 0.0f, m_ps = 0.0f;
-          int m_d = 0, m_r = 0, m_p = 0;
-          uint64_t m_k = 0ull;
 #pragma unroll
-          for (int q = 0; q < SPL; ++q)
-            if (q == lj) { m_sc = f_sc[q]; m_ps = f_ps[q]; m_d = f_d[q]; m_r = f_r[q]; m_p = f_p[q]; m_k = f_k[q]; }
-          m_sc = __shfl_sync(DDT_FULL_MASK, m_sc, ll);
-          m_ps = __shfl_sync(DDT_FULL_MASK, m_ps, ll);
-          m_d = __shfl_sync(DDT_FULL_MASK, m_d, ll);
-          m_r = __shfl_sync(DDT_FULL_MASK, m_r, ll);
-          m_p = __shfl_sync(DDT_FULL_MASK, m_p, ll);
-          m_k = __shfl_sync(DDT_FULL_MASK, m_k, ll);
-          if (lane == wl) {
-#pragma unroll
-            for (int q = 0; q < SPL; ++q)
-              if (q == wj) { f_sc[q] = m_sc; f_ps[q] = m_ps; f_d[q] = m_d; f_r[q] = m_r; f_p[q] = m_p; f_k[q] = m_k; }
-          }
-        }
-        --fsize;
-      }
+      for (int q = 0; q < SPL; ++q) fr[q] = nf[q];
       ++n;
+      // entries that can still be popped: N - n more pops at most
+      fsize = min(min(fsize - 1 + ns, N - n), 32 * SPL);
     }
     __syncwarp();
+    // outputs (coalesced) and ancestor masks
+    for (int j = lane; j < n; j += 32) {
+      o_tok[j] = n_tok[j];
+      o_par[j] = n_parent[j];
+      o_dep[j] = n_dep[j];
+      o_pos[j] = L + n_dep[j];
+      o_sc[j] = n_sc[j];
+    }
     write_masks(o_mask, W, n, n_parent, lane);
   }
   write_pads(o_tok, o_par, o_dep, o_pos, o_sc, o_mask, W, n, N, lane);
@@ -400,21 +433,20 @@ __global__ void __launch_bounds__(32) build_tree_reg_kernel(BuildParams p) {
 }
 
 template <int SPL>
-static int launch_reg(const BuildParams& p, cudaStream_t stream) {
-  const size_t smem = (size_t)p.N * 4 + (size_t)p.D * p.K * 8;
+static int launch_sorted(const BuildParams& p, cudaStream_t stream) {
+  const size_t smem = (size_t)p.N * 16 + (size_t)p.D * p.K * 8;
   if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(build_tree_reg_kernel<SPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(build_tree_sorted_kernel<SPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
       return DDT_ERR_CUDA;
   }
-  return launch_pdl(build_tree_reg_kernel<SPL>, (unsigned)p.B, 32, smem, stream, p);
+  return launch_pdl(build_tree_sorted_kernel<SPL>, (unsigned)p.B, 32, smem, stream, p);
 }
 
 int launch_build_tree(const BuildParams& p, cudaStream_t stream) {
-  if (p.N <= 32) return launch_reg<1>(p, stream);
-  if (p.N <= 64) return launch_reg<2>(p, stream);
-  if (p.N <= 128) return launch_reg<4>(p, stream);
-  if (p.N <= 256) return launch_reg<8>(p, stream);
+  if (p.N <= 64) return launch_sorted<1>(p, stream);
+  if (p.N <= 128) return launch_sorted<2>(p, stream);
+  if (p.N <= 256) return launch_sorted<4>(p, stream);
   const size_t smem = build_smem_bytes(p.N, p.D, p.K);
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(build_tree_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

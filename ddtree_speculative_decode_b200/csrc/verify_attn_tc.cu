@@ -43,13 +43,15 @@
 //    are loaded from a window that ends at that key (never outside the
 //    request's finite rows) and the duplicated keys are masked.
 //  * A request's keys can be split into several units (flash-decoding); each
-//    split writes unnormalised fp32 partials (O, running max, sum) and a small
-//    combine kernel merges them. With one split the kernel writes the final
-//    output and lse directly.
+//    split writes unnormalised fp32 partials (O, running max, sum) and counts
+//    its arrival per (row tile, CTA half); the split that arrives last merges
+//    the partials into the final output. With one split the kernel writes the
+//    final output and lse directly.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstring>
 
 #include "ddt_kernels.cuh"
 #include "sm100_ptx.cuh"
@@ -62,6 +64,7 @@ using namespace sm100;
 constexpr int kDL = 512, kDR = 64, kDQK = 576;
 constexpr int kChunks = kDQK / 64;          // 9 column chunks of 64 (128 bytes)
 constexpr int kTileKeys = 256;              // keys per tile
+constexpr int kMaxSplits = 16;  // key splits per request at most
 constexpr int kBoxBytes = 8192;
 constexpr int kPBytes = 4 * kBoxBytes;        // 64 rows x 256 keys bf16
 constexpr int kMaxW = 8;                      // mask words per row (N <= 256)
@@ -90,7 +93,8 @@ constexpr int kBarSFull = kBarVEmpty + kVStages;      // [2] each CTA: S buffer 
 constexpr int kBarSEmpty = kBarSFull + 2;             // [2] leader: S buffer read (softmax warps of both CTAs)
 constexpr int kBarPFull = kBarSEmpty + 2;             // leader: P written (softmax warps of both CTAs)
 constexpr int kBarOFull = kBarPFull + 1;              // each CTA: PV finished
-constexpr int kNumBars = kBarOFull + 1;
+constexpr int kBarEpi = kBarOFull + 1;                // [4] each CTA: epilogue tile loads, one per 32-dim chunk
+constexpr int kNumBars = kBarEpi + 4;
 constexpr int kOffRed = kOffMisc + 256;                 // float [2 parity][4 groups][64]
 constexpr int kOffLred = kOffRed + 2 * 4 * 64 * 4;      // float [4][64]
 constexpr int kOffMask = kOffLred + 4 * 64 * 4;         // uint32 [64][kMaxW]
@@ -100,6 +104,14 @@ constexpr int kSmemAlloc = kSmemBytes + 1024;           // slack for 1024 alignm
 static_assert(kNumBars * 8 <= 256, "barrier area");
 static_assert(kKStages % 2 == 0, "QK stages are released in pairs");
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
+
+// epilogue staging (reuses the rings once the last MMA has completed): the
+// CTA's 64 rows x 512 dims as 128-byte-wide boxes of 64 rows, 128B-swizzled,
+// fp32 (16 boxes, 128 KB) at kOffStage32 and bf16 (8 boxes, 64 KB) at
+// kOffStage16
+constexpr int kOffStage32 = 0;
+constexpr int kOffStage16 = 16 * kBoxBytes;
+static_assert(kOffStage16 + 8 * kBoxBytes <= kOffMisc, "epilogue staging fits in the rings");
 
 // TMEM columns
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 384;
@@ -121,6 +133,7 @@ struct TcParams {
   float* lse;
   float* part_o;     // [splits][B*N*H][512]
   float* part_ml;    // [splits][B*N*H][2]
+  unsigned* counter; // [B * rowtiles * 2][2] per (row tile, CTA half): splits done, partials published; zero between calls
   int* abort;
 };
 
@@ -129,6 +142,8 @@ struct UnitInfo {
   int off_row;       // first pool row of the request (fits int: checked on host)
   int L, n, nkeys;
   int kb, ke, T;     // key range [kb, ke) of this unit, T tiles
+  int active;        // splits of this request that get keys (splits [0, active))
+  bool pad_tile;     // every row of the row tile is a pad row
 };
 
 __device__ __forceinline__ UnitInfo unit_info(const TcParams& p, int unit) {
@@ -148,9 +163,11 @@ __device__ __forceinline__ UnitInfo unit_info(const TcParams& p, int unit) {
   u.T = t1 - t0;
   u.kb = t0 * kTileKeys;
   u.ke = min(u.nkeys, t1 * kTileKeys);
+  u.active = per > 0 ? (tiles + per - 1) / per : 0;
   // a row tile whose first node is already a pad node has nothing to compute
   const int first_node = (u.rt * 128) / p.H;
-  if (u.n <= 0 || first_node >= u.n) u.T = 0;
+  u.pad_tile = u.n <= 0 || first_node >= u.n;
+  if (u.pad_tile) u.T = 0;
   return u;
 }
 
@@ -184,8 +201,15 @@ __device__ __forceinline__ uint64_t group_visibility(int kw, int g0, int kend, i
   return range & (cache | mask_bits64(mw, W, kw - L));
 }
 
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv, TcParams p) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                   const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_part, TcParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -204,28 +228,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   // ---------------------------------------------------------------- empty unit
   if (u.T == 0) {
-    // no keys for these rows: partials get (m = -inf, l = 0, O = 0); with a
-    // single split the rows are pad rows (written as zeros / -inf)
+    // a split past the last one that gets keys has nothing to do; a row tile
+    // of pad rows only is written (zeros, lse -inf) by split 0
+    if (!u.pad_tile || u.split != 0) return;
     for (int r = threadIdx.x; r < 64; r += kThreads) {
       const int rr = row0 + r;
       if (rr >= req_rows) continue;
       const size_t grow = (size_t)u.b * req_rows + rr;
-      if (p.splits > 1) {
-        p.part_ml[((size_t)u.split * rows_total + grow) * 2 + 0] = -INFINITY;
-        p.part_ml[((size_t)u.split * rows_total + grow) * 2 + 1] = 0.0f;
-      } else if (p.lse) {
-        p.lse[grow] = -INFINITY;
-      }
+      if (p.lse) p.lse[grow] = -INFINITY;
     }
     for (int e = threadIdx.x; e < 64 * (kDL / 4); e += kThreads) {
       const int r = e / (kDL / 4), c4 = e % (kDL / 4);
       const int rr = row0 + r;
       if (rr >= req_rows) continue;
       const size_t grow = (size_t)u.b * req_rows + rr;
-      if (p.splits > 1) {
-        reinterpret_cast<float4*>(p.part_o + ((size_t)u.split * rows_total + grow) * kDL)[c4] =
-            make_float4(0.f, 0.f, 0.f, 0.f);
-      } else if (p.out_dtype == DDT_F32) {
+      if (p.out_dtype == DDT_F32) {
         reinterpret_cast<float4*>(static_cast<float*>(p.out) + grow * kDL)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
       } else {
         reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out) + grow * kDL)[c4] = make_uint2(0u, 0u);
@@ -250,6 +267,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(bar(kBarSEmpty + 1), 2 * kSoftmaxWarps);
     mbar_init(bar(kBarPFull), 2 * kSoftmaxWarps);
     mbar_init(bar(kBarOFull), 1);
+    for (int c = 0; c < 4; ++c) mbar_init(bar(kBarEpi + c), 1);
     fence_mbar_init_cluster();
   }
   if (warp == 0 && lane == 0) {
@@ -538,59 +556,225 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
     // ---------------------------------------------------------- epilogue
+    // O goes from TMEM through swizzled shared-memory boxes to global memory
+    // by TMA tile stores, one group of boxes per 32-dim chunk so that staging
+    // and storing overlap (rows past the request are clipped by the map).
+    //
+    // Several key splits: the split that finishes its keys last for these 64
+    // rows is the merger. It skips its own partial, waits (bounded) until
+    // the other splits -- all already past their keys -- have published
+    // theirs, loads them by TMA and merges them into its own O in TMEM:
+    //   O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
     if (ok) ok = mbar_wait(bar(kBarOFull), (uint32_t)((u.T - 1) & 1), abort);
     tc_fence_after();
     lred[grp * 64 + rho] = lsum;
-    named_bar_sync(1, 32 * kSoftmaxWarps);
-    const float ltot = (lred[rho] + lred[64 + rho]) + (lred[128 + rho] + lred[192 + rho]);
     const int rr = row0 + rho;
     const bool in_range = rr < req_rows;
-    const bool real_row = ok && in_range && (rr / p.H) < u.n;
-    // single split: pad rows of a computed tile are written as zeros
-    const bool write_row = p.splits > 1 ? real_row : in_range;
+    const bool multi = u.active > 1;  // this unit's O is one split's partial
     const size_t grow = (size_t)u.b * req_rows + rr;
-    const float inv = !real_row ? 0.0f : ((p.splits == 1 && ltot > 0.0f) ? 1.0f / ltot : 1.0f);
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      uint32_t r[32];
-      tmem_ld32(lane_addr + o_col + 32 * c, r);
-      tmem_wait_ld();
-      if (!write_row) continue;
-      const int d0 = 256 * sub + 128 * eta + 32 * c;  // first output dim of this chunk
-      if (p.splits > 1) {
-        float4* dst = reinterpret_cast<float4*>(p.part_o + ((size_t)u.split * rows_total + grow) * kDL + d0);
+    const uint32_t sw = (uint32_t)(rho & 7);
+    const bool f32_out = p.out_dtype == DDT_F32;
+    int* s_flag = reinterpret_cast<int*>(smem + kOffTmem + 4);
+    unsigned* cnt = multi ? p.counter + (((size_t)u.b * p.rowtiles + u.rt) * 2 + rank) * 2 : nullptr;
+    if (multi && threadIdx.x == 128) {
+      const bool last = atomicAdd(cnt, 1u) == (unsigned)(u.active - 1);
+      if (last) cnt[0] = 0u;
+      *s_flag = last ? 1 : 0;
+    }
+    named_bar_sync(1, 32 * kSoftmaxWarps);
+    const bool merger = multi && *s_flag != 0;
+    const float ltot = (lred[rho] + lred[64 + rho]) + (lred[128 + rho] + lred[192 + rho]);
+    const bool real_row = ok && in_range && (rr / p.H) < u.n;
+    const float m_own = real_row ? m_used : -INFINITY;
+    // 32 values of this thread's row, dims d0.., into the fp32 or bf16 staging
+    auto stage_chunk = [&](int d0, const float* f, bool f32) {
+      if (f32) {
+        unsigned char* row = smem + kOffStage32 + (d0 >> 5) * kBoxBytes + rho * 128;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                               __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-      } else if (p.out_dtype == DDT_F32) {
-        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + grow * kDL + d0);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
-                               __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv);
+          *reinterpret_cast<float4*>(row + (((uint32_t)i ^ sw) << 4)) =
+              make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
       } else {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + grow * kDL + d0);
+        unsigned char* row = smem + kOffStage16 + (d0 >> 6) * kBoxBytes + rho * 128;
+        const int i0 = (d0 & 63) >> 3;  // 16-byte chunk of the first value
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           uint32_t w[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[8 * i + 2 * k]) * inv,
-                                                      __uint_as_float(r[8 * i + 2 * k + 1]) * inv);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(f[8 * i + 2 * k], f[8 * i + 2 * k + 1]);
             w[k] = *reinterpret_cast<uint32_t*>(&h2);
           }
-          dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(row + (((uint32_t)(i0 + i) ^ sw) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-    }
-    if (write_row && grp == 0) {
-      if (p.splits > 1) {
-        p.part_ml[((size_t)u.split * rows_total + grow) * 2 + 0] = m_used;
-        p.part_ml[((size_t)u.split * rows_total + grow) * 2 + 1] = ltot;
-      } else if (p.lse) {
-        p.lse[grow] = (real_row && ltot > 0.0f) ? (m_used + log2f(ltot)) * 0.6931471805599453f : -INFINITY;
+    };
+    // after chunk c is staged by every thread: one thread stores the boxes it
+    // completed. kind 0: this split's partial (fp32), 1: final fp32, 2: final
+    // bf16 (a bf16 box holds two chunks: stored after odd c)
+    auto store_chunk = [&](int c, int kind) {
+      if (kind == 2 && !(c & 1)) return;
+      fence_proxy_async_smem();
+      named_bar_sync(1, 32 * kSoftmaxWarps);
+      if (threadIdx.x == 128) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (kind == 0) {
+            const int j = 4 * q + c;
+            tma_store_4d(&tm_part, sbase + kOffStage32 + j * kBoxBytes, 32 * j, row0, u.b, u.split);
+          } else if (kind == 1) {
+            const int j = 4 * q + c;
+            tma_store_3d(&tm_out, sbase + kOffStage32 + j * kBoxBytes, 32 * j, row0, u.b);
+          } else {
+            const int j = 2 * q + (c >> 1);
+            tma_store_3d(&tm_out, sbase + kOffStage16 + j * kBoxBytes, 64 * j, row0, u.b);
+          }
+        }
+        bulk_commit();
       }
+    };
+    // TMA loads of split s2's partial rows into the fp32 staging, one barrier per chunk
+    auto load_partial = [&](int s2) {
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        mbar_arrive_expect_tx(bar(kBarEpi + c), 4u * kBoxBytes);
+        for (int q = 0; q < 4; ++q) {
+          const int j = 4 * q + c;
+          tma_load_4d(sbase + kOffStage32 + j * kBoxBytes, &tm_part, 32 * j, row0, u.b, s2, bar(kBarEpi + c));
+        }
+      }
+    };
+    if (!merger) {
+      // the final output (one split) or this split's partial
+      const int kind = multi ? 0 : (f32_out ? 1 : 2);
+      const float inv = !real_row ? 0.0f : ((!multi && ltot > 0.0f) ? 1.0f / ltot : 1.0f);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(lane_addr + o_col + 32 * c, r);
+        tmem_wait_ld();
+        float f[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(r[i]) * inv;
+        stage_chunk(256 * sub + 128 * eta + 32 * c, f, kind != 2);
+        store_chunk(c, kind);
+      }
+      if (grp == 0 && in_range) {
+        if (multi) {
+          *reinterpret_cast<float2*>(p.part_ml + ((size_t)u.split * rows_total + grow) * 2) = make_float2(m_own, ltot);
+        } else if (p.lse) {
+          p.lse[grow] = (real_row && ltot > 0.0f) ? (m_used + log2f(ltot)) * 0.6931471805599453f : -INFINITY;
+        }
+      }
+      if (multi) {
+        // publish: partial rows (TMA, complete) and (m, l) before the count
+        if (threadIdx.x == 128) {
+          bulk_wait_all();
+          fence_proxy_async_global();
+        }
+        __threadfence();
+        named_bar_sync(1, 32 * kSoftmaxWarps);
+        if (threadIdx.x == 128) atomicAdd(cnt + 1, 1u);
+      } else if (threadIdx.x == 128) {
+        bulk_wait_read_all();
+      }
+    } else {
+      // ---- merger
+      int* s_ok = s_flag;
+      if (threadIdx.x == 128) {
+        bool pub = true;
+        if (ld_acquire_gpu(cnt + 1) != (unsigned)(u.active - 1)) {
+          const uint64_t t0 = global_timer_ns();
+          while (ld_acquire_gpu(cnt + 1) != (unsigned)(u.active - 1)) {
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+              atomicExch(abort, 1);
+              pub = false;
+              break;
+            }
+          }
+        }
+        if (pub) cnt[1] = 0u;
+        __threadfence();
+        fence_proxy_async_global();
+        *s_ok = pub ? 1 : 0;
+        if (pub) load_partial(u.split == 0 ? 1 : 0);
+      }
+      named_bar_sync(1, 32 * kSoftmaxWarps);
+      const bool pub = *s_ok != 0;
+      if (!pub) ok = false;
+      float M = m_own;
+      if (in_range && pub)
+        for (int s2 = 0; s2 < u.active; ++s2)
+          if (s2 != u.split) M = fmaxf(M, __ldcg(p.part_ml + ((size_t)s2 * rows_total + grow) * 2));
+      const float w_own = m_own == -INFINITY ? 0.0f : exp2f(m_own - M);
+      float den = w_own * ltot;
+      const int nother = u.active - 1;
+      int step = 0;
+      for (int s2 = 0; s2 < u.active && pub; ++s2) {
+        if (s2 == u.split) continue;
+        float w_s = 0.0f;
+        if (in_range) {
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml) + (size_t)s2 * rows_total + grow);
+          w_s = ml.x == -INFINITY ? 0.0f : exp2f(ml.x - M);
+          den += w_s * ml.y;
+        }
+        const bool last = step == nother - 1;
+        const float dinv = den > 0.0f ? 1.0f / den : 0.0f;
+        const float wo = step == 0 ? w_own : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          if (!mbar_wait_own(bar(kBarEpi + c), (uint32_t)(step & 1), abort)) ok = false;
+          const int d0 = 256 * sub + 128 * eta + 32 * c;
+          uint32_t r[32];
+          tmem_ld32(lane_addr + o_col + 32 * c, r);
+          tmem_wait_ld();
+          const unsigned char* row = smem + kOffStage32 + (d0 >> 5) * kBoxBytes + rho * 128;
+          float f[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 v = *reinterpret_cast<const float4*>(row + (((uint32_t)i ^ sw) << 4));
+            f[4 * i] = fmaf(w_s, v.x, __uint_as_float(r[4 * i]) * wo);
+            f[4 * i + 1] = fmaf(w_s, v.y, __uint_as_float(r[4 * i + 1]) * wo);
+            f[4 * i + 2] = fmaf(w_s, v.z, __uint_as_float(r[4 * i + 2]) * wo);
+            f[4 * i + 3] = fmaf(w_s, v.w, __uint_as_float(r[4 * i + 3]) * wo);
+          }
+          if (last) {
+            const bool keep = real_row && ok;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) f[i] = keep ? f[i] * dinv : 0.0f;
+            stage_chunk(d0, f, f32_out);  // fp32: in place of the values just read
+            store_chunk(c, f32_out ? 1 : 2);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(f[i]);
+            tmem_st32(lane_addr + o_col + 32 * c, r);
+          }
+        }
+        if (!last) {
+          tmem_wait_st();
+          named_bar_sync(1, 32 * kSoftmaxWarps);  // staging read by all before the next loads
+          if (threadIdx.x == 128) {
+            int nx = s2 + 1;
+            if (nx == u.split) ++nx;
+            load_partial(nx);
+          }
+        }
+        ++step;
+      }
+      if (!pub) {
+        // timed out waiting for the other splits: zeros
+        float f[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) f[i] = 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          stage_chunk(256 * sub + 128 * eta + 32 * c, f, f32_out);
+          store_chunk(c, f32_out ? 1 : 2);
+        }
+      }
+      if (grp == 0 && in_range && p.lse)
+        p.lse[grow] = (real_row && ok && den > 0.0f) ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
+      if (threadIdx.x == 128) bulk_wait_read_all();
     }
   }
   // ---------------------------------------------------------------- teardown
@@ -601,44 +785,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem, 512);
   }
-}
-
-// Merge split partials: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
-__global__ void __launch_bounds__(128) attn_combine_kernel(TcParams p) {
-  pdl_wait();
-  pdl_launch_dependents();
-  const int rows_total = p.B * p.N * p.H;
-  const int row = blockIdx.x;
-  if (row >= rows_total) return;
-  const int b = row / (p.N * p.H);
-  const int node = (row / p.H) % p.N;
-  const bool real_row = node < p.n_nodes[b];
-  float M = -INFINITY;
-  for (int s = 0; s < p.splits; ++s) M = fmaxf(M, p.part_ml[((size_t)s * rows_total + row) * 2]);
-  float wsum = 0.0f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int c4 = threadIdx.x;  // 128 threads x 4 dims
-  if (real_row && M != -INFINITY) {
-    for (int s = 0; s < p.splits; ++s) {
-      const float m = p.part_ml[((size_t)s * rows_total + row) * 2];
-      if (m == -INFINITY) continue;
-      const float w = exp2f(m - M);
-      wsum += w * p.part_ml[((size_t)s * rows_total + row) * 2 + 1];
-      const float4 o = reinterpret_cast<const float4*>(p.part_o + ((size_t)s * rows_total + row) * kDL)[c4];
-      acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
-    }
-  }
-  const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
-  acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
-  if (p.out_dtype == DDT_F32) {
-    reinterpret_cast<float4*>(static_cast<float*>(p.out) + (size_t)row * kDL)[c4] = acc;
-  } else {
-    __nv_bfloat162 a = __floats2bfloat162_rn(acc.x, acc.y), bq = __floats2bfloat162_rn(acc.z, acc.w);
-    reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out) + (size_t)row * kDL)[c4] =
-        make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&bq));
-  }
-  if (p.lse && threadIdx.x == 0)
-    p.lse[row] = (real_row && wsum > 0.0f) ? (M + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
 }
 
 // ---------------------------------------------------------------------------
@@ -670,6 +816,24 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t rows) {
   return r == CUDA_SUCCESS;
 }
 
+// [outer...][req_rows][512] row-major output-like tensor (f32 or bf16) with
+// 128-byte x 64-row boxes, 128B-swizzled; rank 3 (B) or 4 (splits, B).
+static bool make_out_map(CUtensorMap* m, void* base, bool f32, int rank, uint64_t req_rows, uint64_t B,
+                         uint64_t splits) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t es = f32 ? 4 : 2;
+  cuuint64_t dims[4] = {(cuuint64_t)kDL, (cuuint64_t)req_rows, (cuuint64_t)B, (cuuint64_t)splits};
+  cuuint64_t strides[3] = {(cuuint64_t)(kDL * es), (cuuint64_t)(req_rows * kDL * es),
+                           (cuuint64_t)(B * req_rows * kDL * es)};
+  cuuint32_t box[4] = {(cuuint32_t)(128 / es), 64, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, base,
+                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // number of key splits: minimise an estimate of the makespan over 74 CTA pairs
 static int choose_splits(int B, int N, int H, int max_cache_len) {
   const int rowtiles = (N * H + 127) / 128;
@@ -678,7 +842,7 @@ static int choose_splits(int B, int N, int H, int max_cache_len) {
   const int slots = 74;
   int best = 1;
   double best_t = 1e30;
-  for (int s = 1; s <= std::min(16, std::max(1, tiles)); ++s) {
+  for (int s = 1; s <= std::min(kMaxSplits, std::max(1, tiles)); ++s) {
     const int per = (tiles + s - 1) / s;
     const long units = (long)units1 * s;
     const long waves = (units + slots - 1) / slots;
@@ -696,12 +860,17 @@ bool tc_attn_supported(int d_l, int d_r, int in_dtype) {
   return in_dtype == DDT_BF16 && d_l == tc::kDL && d_r == tc::kDR;
 }
 
+static size_t counter_bytes(int B, int N, int H) {
+  const size_t rowtiles = ((size_t)N * H + 127) / 128;
+  return ((size_t)B * rowtiles * 2 * 2 * 4 + 255) / 256 * 256;
+}
+
 size_t tc_attn_workspace_bytes(int B, int N, int H, int max_cache_len) {
   const int s = tc::choose_splits(B, N, H, max_cache_len);
   size_t bytes = tc::ws_header();
   if (s > 1) {
     const size_t rows = (size_t)B * N * H;
-    bytes += (size_t)s * rows * tc::kDL * 4 + (size_t)s * rows * 2 * 4;
+    bytes += counter_bytes(B, N, H) + (size_t)s * rows * tc::kDL * 4 + (size_t)s * rows * 2 * 4;
   }
   return bytes;
 }
@@ -734,8 +903,10 @@ int launch_attn_tc(const AttnParams& a, int64_t kv_rows, int max_cache_len, void
   p.abort = reinterpret_cast<int*>(ws);
   if (p.splits > 1) {
     const size_t rows = (size_t)a.B * a.N * a.H;
-    p.part_o = reinterpret_cast<float*>(ws + ws_header());
-    p.part_ml = reinterpret_cast<float*>(ws + ws_header() + (size_t)p.splits * rows * kDL * 4);
+    const size_t cb = counter_bytes(a.B, a.N, a.H);
+    p.counter = reinterpret_cast<unsigned*>(ws + ws_header());
+    p.part_o = reinterpret_cast<float*>(ws + ws_header() + cb);
+    p.part_ml = reinterpret_cast<float*>(ws + ws_header() + cb + (size_t)p.splits * rows * kDL * 4);
   }
   if (workspace_bytes < tc_attn_workspace_bytes(a.B, a.N, a.H, max_cache_len)) return DDT_ERR_INVALID_ARG;
   static bool attr_set = false;
@@ -744,10 +915,14 @@ int launch_attn_tc(const AttnParams& a, int64_t kv_rows, int max_cache_len, void
       return DDT_ERR_CUDA;
     attr_set = true;
   }
+  CUtensorMap tout, tpart;
+  memset(&tpart, 0, sizeof(tpart));
+  if (!make_out_map(&tout, a.out, a.out_dtype == DDT_F32, 3, (uint64_t)a.N * a.H, (uint64_t)a.B, 1)) return DDT_ERR_CUDA;
+  if (p.splits > 1 &&
+      !make_out_map(&tpart, p.part_o, true, 4, (uint64_t)a.N * a.H, (uint64_t)a.B, (uint64_t)p.splits))
+    return DDT_ERR_CUDA;
   const long long units = (long long)a.B * p.rowtiles * p.splits;
-  int st = launch_pdl(attn_tc_kernel, (unsigned)(2 * units), kThreads, kSmemAlloc, stream, tq, tkv, p);
-  if (st != DDT_OK || p.splits == 1) return st;
-  return launch_pdl(attn_combine_kernel, (unsigned)q_rows, 128, 0, stream, p);
+  return launch_pdl(attn_tc_kernel, (unsigned)(2 * units), kThreads, kSmemAlloc, stream, tq, tkv, tout, tpart, p);
 }
 
 }  // namespace ddt

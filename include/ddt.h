@@ -158,8 +158,12 @@ DDT_API int ddt_build_tree(const float* logp, const int32_t* tok, const int32_t*
  *   (zero the buffer once after allocating it). Every wait inside the bf16
  *   kernel is bounded (about 2 s); if one expires the kernel stores
  *   DDT_ERR_TIMEOUT there and returns, and later calls with that workspace
- *   return at once until the caller zeroes it again. The rest of the
- *   workspace holds per-split partial results; its contents do not matter.
+ *   return at once until the caller zeroes it again. When the launch splits
+ *   the keys (the size above 256), the next bytes are per-row-tile arrival
+ *   counters that must also start at zero; each call leaves them at zero
+ *   (except after a timeout: zero the whole workspace then). The rest holds
+ *   per-split partial results; its contents do not matter. Calls that share
+ *   a workspace must not overlap in time.
  * Errors: DDT_ERR_INVALID_ARG (nulls, sizes, workspace too small or
  *   misaligned, kv / q not 16-byte aligned for bf16), DDT_ERR_UNSUPPORTED.
  */
