@@ -305,7 +305,7 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
     pk = peaks()
     achieved = flops / (attn_ms / 1e3) / 1e12
     peak = pk["bf16_tflops_sustained"]
-    launches_per_step = 1 + attn_launches(shape) + 1  # build, attention, accept (memcpy of cache_len excluded)
+    launches_per_step = 1 + attn_launches(shape) + 2  # build, attention, accept argmax + walk (cache_len memcpy excluded)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,

@@ -8,26 +8,44 @@
 // post-verify compaction; "ddtree_speculative_decode_test_capstone", section
 // "What the Test Validated": the bonus token).
 //
-// One launch:
-//  * Every (row, vocab-chunk) pair is one CTA that streams its 16-byte
-//    vectors once and reduces them to one packed 64-bit key (order-preserving
-//    value bits << 32 | ~index): the max key is the largest logit at its
-//    lowest index. Partial keys go to the workspace.
-//  * The CTA that finishes a request's last chunk (a per-request arrival
-//    counter in the workspace; it resets the counter to zero for the next call)
-//    folds the partial keys into am[], walks the tree with warp ballots, then
-//    copies the accepted rows. path[j] >= j and the path is increasing, so
-//    copying rows in increasing j is already read-before-write per byte; the
-//    CTA still stages groups of rows in registers behind a barrier so many rows
-//    are in flight at once.
+// Two launches:
+//  * accept_argmax_kernel streams the logits once with coalesced 16-byte
+//    loads, eight in flight per lane, 32 warps per SM. Work is cut into
+//    slices of 2048 entries of one row, and every warp owns a contiguous
+//    range of slices, so it folds a row's slices itself and publishes one
+//    packed 64-bit key per row segment with a fire-and-forget atomic max
+//    (key = order-preserving value bits << 32 | ~index: the max key is the
+//    largest logit at its lowest index). A lane only searches for an index
+//    when a batch beats its running maximum, so the common batch costs one
+//    packed max per two values.
+//  * accept_walk_kernel, one CTA per request (launched programmatically: it
+//    stages the tree while the argmax runs), turns the row keys into am[],
+//    finds every node's accepted child (the lowest-index child whose token is
+//    the node's argmax) with shared-memory atomics, chases the path from the
+//    root, writes the outputs, copies the accepted rows and clears the row
+//    keys for the next call. path[j] >= j and the path is increasing, so
+//    copying rows in increasing j is already read-before-write per byte; rows
+//    are still staged in registers behind a barrier so that many are in
+//    flight at once.
+#include <algorithm>
 #include <mutex>
 
 #include "ddt_kernels.cuh"
 
 namespace ddt {
 
-constexpr int kArgmaxThreads = 256;
-constexpr int kArgmaxChunk = 16384;  // vocab entries per CTA
+constexpr int kSliceVec = 8;                      // 16-byte loads per lane per slice
+constexpr int kArgmaxThreads = 512;
+constexpr int kArgmaxCtasPerSm = 2;
+constexpr int kWalkThreads = 512;
+constexpr int kMaxN = 1024;
+constexpr int kStageVec = 4;                      // 16-byte vectors per thread per copy round
+
+template <bool kBF16>
+struct SliceCfg {
+  static constexpr int kPer = kBF16 ? 8 : 4;                // values per 16-byte vector
+  static constexpr int kElems = 32 * kSliceVec * kPer;      // values per slice
+};
 
 __device__ __forceinline__ unsigned long long pack_key(float v, int idx) {
   return (static_cast<unsigned long long>(float_order_key(v)) << 32) |
@@ -38,284 +56,269 @@ __device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsig
   return a > b ? a : b;
 }
 
-__device__ __noinline__ void walk_compact_body(const AcceptParams& p, int b);
-
-template <bool kBF16>
-__global__ void __launch_bounds__(kArgmaxThreads) accept_kernel(AcceptParams p) {
-  pdl_wait();
-  pdl_launch_dependents();
-  const int row = blockIdx.x / p.chunks;  // b * N + i
-  const int chunk = blockIdx.x - row * p.chunks;
-  const int b = row / p.N;
-  const int i = row - b * p.N;
-  const int n = p.n_nodes[b];
-  if (i >= n) {
-    // an empty tree has no argmax CTAs: one CTA writes its (skipped) outputs
-    if (n <= 0 && i == 0 && chunk == 0) walk_compact_body(p, b);
-    return;
-  }
-  const int v0 = chunk * kArgmaxChunk;
-  const int v1 = min(p.V, v0 + kArgmaxChunk);
-  unsigned long long best = 0ull;
-  if (kBF16) {
-    const uint16_t* src = static_cast<const uint16_t*>(p.logits) + (size_t)row * p.V;
-    // 8 bf16 per 16-byte vector when the row start is 16-byte aligned
-    const bool vec = ((reinterpret_cast<uintptr_t>(src + v0) & 15u) == 0);
-    if (vec) {
-      const int nvec = (v1 - v0) >> 3;
-      const uint4* s4 = reinterpret_cast<const uint4*>(src + v0);
-      constexpr int U = 8;
-      for (int base = 0; base < nvec; base += kArgmaxThreads * U) {
-        uint4 r[U];
+__device__ __forceinline__ unsigned long long warp_max64(unsigned long long k) {
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int e = base + u * kArgmaxThreads + threadIdx.x;
-          r[u] = e < nvec ? __ldcs(s4 + e) : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
-        }
-        // pass 1: the thread's largest value (packed bf16 max, -inf padding)
-        __nv_bfloat162 m2 = __halves2bfloat162(__ushort_as_bfloat16(0xff80), __ushort_as_bfloat16(0xff80));
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const uint32_t w[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
-#pragma unroll
-          for (int t = 0; t < 4; ++t) m2 = __hmax2(m2, *reinterpret_cast<const __nv_bfloat162*>(&w[t]));
-        }
-        const float mx = fmaxf(__low2float(m2), __high2float(m2));
-        // pass 2: its lowest index (values compare as floats, so -0 == +0)
-        int first = 0x7fffffff;
-#pragma unroll
-        for (int u = U - 1; u >= 0; --u) {
-          const int e = base + u * kArgmaxThreads + threadIdx.x;
-          const uint32_t w[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
-#pragma unroll
-          for (int t = 3; t >= 0; --t) {
-            const int idx = v0 + e * 8 + 2 * t;
-            if (e < nvec && __uint_as_float(w[t] & 0xffff0000u) == mx) first = idx + 1;
-            if (e < nvec && __uint_as_float(w[t] << 16) == mx) first = idx;
-          }
-        }
-        if (first != 0x7fffffff) best = umax64(best, pack_key(mx, first));
-      }
-      for (int v = v0 + nvec * 8 + threadIdx.x; v < v1; v += kArgmaxThreads)
-        best = umax64(best, pack_key(bf16_bits_to_float(src[v]), v));
-    } else {
-      for (int v = v0 + threadIdx.x; v < v1; v += kArgmaxThreads)
-        best = umax64(best, pack_key(bf16_bits_to_float(src[v]), v));
-    }
-  } else {
-    const float* src = static_cast<const float*>(p.logits) + (size_t)row * p.V;
-    const bool vec = ((reinterpret_cast<uintptr_t>(src + v0) & 15u) == 0);
-    if (vec) {
-      const int nvec = (v1 - v0) >> 2;
-      const float4* s4 = reinterpret_cast<const float4*>(src + v0);
-      for (int e = threadIdx.x; e < nvec; e += kArgmaxThreads) {
-        const float4 r = __ldcs(s4 + e);
-        const int idx = v0 + e * 4;
-        best = umax64(best, pack_key(r.x, idx));
-        best = umax64(best, pack_key(r.y, idx + 1));
-        best = umax64(best, pack_key(r.z, idx + 2));
-        best = umax64(best, pack_key(r.w, idx + 3));
-      }
-      for (int v = v0 + nvec * 4 + threadIdx.x; v < v1; v += kArgmaxThreads)
-        best = umax64(best, pack_key(src[v], v));
-    } else {
-      for (int v = v0 + threadIdx.x; v < v1; v += kArgmaxThreads)
-        best = umax64(best, pack_key(src[v], v));
-    }
-  }
-  // block reduce: warp shuffles, then one value per warp through shared memory
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) best = umax64(best, __shfl_xor_sync(DDT_FULL_MASK, best, o));
-  __shared__ unsigned long long wbest[kArgmaxThreads / 32];
-  if ((threadIdx.x & 31) == 0) wbest[threadIdx.x >> 5] = best;
-  __syncthreads();
-  __shared__ int s_last;
-  if (threadIdx.x == 0) {
-    unsigned long long m = wbest[0];
-#pragma unroll
-    for (int w = 1; w < kArgmaxThreads / 32; ++w) m = umax64(m, wbest[w]);
-    p.partial[(size_t)row * p.chunks + chunk] = m;
-    __threadfence();
-    const unsigned prev = atomicAdd(p.counter + b, 1u);
-    s_last = (prev == (unsigned)(n * p.chunks - 1));
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  walk_compact_body(p, b);
-  if (threadIdx.x == 0) p.counter[b] = 0u;
+  for (int o = 16; o > 0; o >>= 1) k = umax64(k, __shfl_xor_sync(DDT_FULL_MASK, k, o));
+  return k;
 }
 
-constexpr int kWalkThreads = 256;
-constexpr int kMaxN = 1024;
-constexpr int kStageRows = 16;  // rows staged per copy round
-constexpr int kStageVec = 8;    // 16-byte vectors per thread per round (256 * 8 * 16 B = 32 KB)
+// Value t (0..kPer-1) of a 16-byte vector.
+template <bool kBF16>
+__device__ __forceinline__ float vec_val(const uint4& r, int t) {
+  const uint32_t w = t < (kBF16 ? 2 : 1) ? r.x : t < (kBF16 ? 4 : 2) ? r.y : t < (kBF16 ? 6 : 3) ? r.z : r.w;
+  if (!kBF16) return __uint_as_float(w);
+  return __uint_as_float((t & 1) ? (w & 0xffff0000u) : (w << 16));
+}
 
-__device__ __noinline__ void walk_compact_body(const AcceptParams& p, int b) {
-  const int N = p.N;
-  const int n = p.n_nodes[b];
+template <bool kBF16>
+__global__ void __launch_bounds__(kArgmaxThreads) accept_argmax_kernel(AcceptParams p) {
+  using C = SliceCfg<kBF16>;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const long long gw = ((long long)blockIdx.x * kArgmaxThreads + threadIdx.x) >> 5;
+  const long long nw = ((long long)gridDim.x * kArgmaxThreads) >> 5;
+  const int spr = (p.V + C::kElems - 1) / C::kElems;  // slices per row
+  const long long slices = (long long)p.B * p.N * spr;
+  const long long s_begin = slices * gw / nw, s_end = slices * (gw + 1) / nw;
+  const size_t esz = kBF16 ? 2 : 4;
+  int cur_row = -1;
+  float best_v = -INFINITY;   // this lane's running max of cur_row and its lowest index
+  int best_i = -1;
+  auto flush = [&]() {
+    const unsigned long long k = warp_max64(best_i < 0 ? 0ull : pack_key(best_v, best_i));
+    if (lane == 0 && k != 0ull) atomicMax(p.rowkey + cur_row, k);  // result unused: no wait
+  };
+  for (long long sl = s_begin; sl < s_end; ++sl) {
+    const int r = (int)(sl / spr), c = (int)(sl - (long long)r * spr);
+    const int b = r / p.N, i = r - b * p.N;
+    if (i >= __ldg(p.n_nodes + b)) continue;
+    if (r != cur_row) {
+      if (cur_row >= 0) flush();
+      cur_row = r;
+      best_v = -INFINITY;
+      best_i = -1;
+    }
+    const int v0 = c * C::kElems;
+    const int cnt = min(C::kElems, p.V - v0);
+    const unsigned char* row = static_cast<const unsigned char*>(p.logits) + ((size_t)r * p.V + v0) * esz;
+    if (p.tma) {  // 16-byte aligned rows: cnt is a multiple of kPer
+      const int nvec = cnt / C::kPer;
+      uint4 v[kSliceVec];
+#pragma unroll
+      for (int k = 0; k < kSliceVec; ++k) {
+        const int e = lane + 32 * k;
+        v[k] = e < nvec ? __ldcs(reinterpret_cast<const uint4*>(row) + e)
+                        : (kBF16 ? make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u)
+                                 : make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u));
+      }
+      // tree-shaped maximum (short dependency chains)
+      float m;
+      if (kBF16) {
+        auto h = [](uint32_t w) { return *reinterpret_cast<const __nv_bfloat162*>(&w); };
+        __nv_bfloat162 mk[kSliceVec];
+#pragma unroll
+        for (int k = 0; k < kSliceVec; ++k)
+          mk[k] = __hmax2(__hmax2(h(v[k].x), h(v[k].y)), __hmax2(h(v[k].z), h(v[k].w)));
+#pragma unroll
+        for (int w = kSliceVec / 2; w > 0; w >>= 1)
+#pragma unroll
+          for (int k = 0; k < w; ++k) mk[k] = __hmax2(mk[k], mk[k + w]);
+        m = fmaxf(__low2float(mk[0]), __high2float(mk[0]));
+      } else {
+        float mk[kSliceVec];
+#pragma unroll
+        for (int k = 0; k < kSliceVec; ++k)
+          mk[k] = fmaxf(fmaxf(__uint_as_float(v[k].x), __uint_as_float(v[k].y)),
+                        fmaxf(__uint_as_float(v[k].z), __uint_as_float(v[k].w)));
+#pragma unroll
+        for (int w = kSliceVec / 2; w > 0; w >>= 1)
+#pragma unroll
+          for (int k = 0; k < w; ++k) mk[k] = fmaxf(mk[k], mk[k + w]);
+        m = mk[0];
+      }
+      const bool has_real = lane < nvec;
+      if (has_real && (m > best_v || best_i < 0)) {
+        // lowest real index holding m (values compare as floats: -0 == +0)
+        int first = -1;
+#pragma unroll
+        for (int k = kSliceVec - 1; k >= 0; --k) {
+          const int e = lane + 32 * k;
+#pragma unroll
+          for (int t = C::kPer - 1; t >= 0; --t)
+            if (e < nvec && vec_val<kBF16>(v[k], t) == m) first = v0 + e * C::kPer + t;
+        }
+        best_v = m;
+        best_i = first;
+      }
+    } else {
+      for (int t = lane; t < cnt; t += 32) {
+        const float x = kBF16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(row)[t])
+                              : reinterpret_cast<const float*>(row)[t];
+        if (x > best_v || best_i < 0) { best_v = x; best_i = v0 + t; }
+      }
+    }
+  }
+  if (cur_row >= 0) flush();
+}
+
+// Request epilogue: one CTA per request.
+__global__ void __launch_bounds__(kWalkThreads) accept_walk_kernel(AcceptParams p) {
   __shared__ int32_t s_am[kMaxN];
+  __shared__ int32_t s_child[kMaxN];
   __shared__ int32_t s_path[kMaxN];
   __shared__ int32_t s_par[kMaxN];
   __shared__ int32_t s_tok[kMaxN];
-  __shared__ int s_a;
-  __shared__ int s_skip;
-
-  if (threadIdx.x == 0) {
+  __shared__ int s_misc[3];
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int N = p.N;
+  // The tree and the cache bookkeeping are inputs the argmax kernel does not
+  // write, and this grid starts only after that kernel has waited for all
+  // earlier work: stage them before waiting for the argmax.
+  const int n = p.n_nodes[b];
+  for (int i = tid; i < n; i += kWalkThreads) {
+    s_par[i] = p.parent[(size_t)b * N + i];
+    s_tok[i] = p.node_tok[(size_t)b * N + i];
+    s_child[i] = 0x7fffffff;
+  }
+  if (tid == 0) {
     int st = DDT_OK;
     const int L = p.cache_len[b];
     if (n > 0 && (int64_t)L + n > (int64_t)p.cache_cap[b]) st = DDT_ERR_CAPACITY;
-    s_skip = (n <= 0 || st != DDT_OK);
+    s_misc[0] = (n <= 0 || st != DDT_OK);
     if (p.dev_status) p.dev_status[b] = st;
   }
-  // fold partial argmax keys: 4 threads per row, each over a strided subset
-  // of the chunks, then a 4-lane shuffle reduce
-  for (int i0 = 0; i0 < N; i0 += kWalkThreads / 4) {
-    const int i = i0 + (threadIdx.x >> 2);
-    const int sub = threadIdx.x & 3;
-    unsigned long long m = 0ull;
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int i = tid; i < N; i += kWalkThreads) {
+    int a = -1;
     if (i < n) {
-      const unsigned long long* pk = p.partial + ((size_t)b * N + i) * p.chunks;
-      for (int c = sub; c < p.chunks; c += 4) m = umax64(m, __ldcg(pk + c));
-    }
-    m = umax64(m, __shfl_xor_sync(DDT_FULL_MASK, m, 1));
-    m = umax64(m, __shfl_xor_sync(DDT_FULL_MASK, m, 2));
-    if (sub == 0 && i < N) {
-      const int a = i < n ? static_cast<int>(~static_cast<uint32_t>(m & 0xffffffffull)) : -1;
+      const unsigned long long k = p.rowkey[(size_t)b * N + i];
+      p.rowkey[(size_t)b * N + i] = 0ull;  // zero for the next call
+      a = static_cast<int>(~static_cast<uint32_t>(k & 0xffffffffull));
       s_am[i] = a;
-      if (p.am) p.am[(size_t)b * N + i] = a;
     }
-  }
-  for (int i = threadIdx.x; i < n; i += kWalkThreads) {
-    s_par[i] = p.parent[(size_t)b * N + i];
-    s_tok[i] = p.node_tok[(size_t)b * N + i];
+    if (p.am) p.am[(size_t)b * N + i] = a;
   }
   __syncthreads();
-  const bool skip = s_skip;
-  // greedy walk on warp 0
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    const int32_t* par = s_par;
-    const int32_t* tk = s_tok;
-    int a = 0;
+  const bool skip = s_misc[0] != 0;
+  // accepted child of every node: the lowest-index child whose token is the
+  // node's argmax (children have larger indices than their parent)
+  if (!skip)
+    for (int j = 1 + tid; j < n; j += kWalkThreads) {
+      const int pp = s_par[j];
+      if (pp >= 0 && pp < j && s_tok[j] == s_am[pp]) atomicMin(&s_child[pp], j);
+    }
+  __syncthreads();
+  if (tid == 0) {
+    int a = 0, cur = 0;
+    s_path[0] = 0;
     if (!skip) {
-      int curn = 0;
-      if (lane == 0) s_path[0] = 0;
       for (;;) {
-        const int want = s_am[curn];
-        int found = -1;
-        // children have larger indices than their parent
-        for (int base = curn + 1; base < n && found < 0; base += 32) {
-          const int c = base + lane;
-          const bool hit = c < n && par[c] == curn && tk[c] == want;
-          const uint32_t bal = __ballot_sync(DDT_FULL_MASK, hit);
-          if (bal) found = base + __ffs(bal) - 1;
-        }
-        if (found < 0) break;
-        ++a;
-        if (lane == 0) s_path[a] = found;
-        curn = found;
+        const int c = s_child[cur];
+        if (c >= n) break;  // none
+        s_path[++a] = c;
+        cur = c;
       }
     }
-    if (lane == 0) s_a = a;
+    s_misc[1] = a;
+    s_misc[2] = skip ? -1 : s_am[cur];
   }
   __syncthreads();
-  const int a = s_a;
-  // outputs
-  for (int j = threadIdx.x; j < N; j += kWalkThreads) {
+  const int a = s_misc[1];
+  const int bonus = s_misc[2];
+  for (int j = tid; j < N; j += kWalkThreads) {
     const bool in = !skip && j <= a;
     p.acc_nodes[(size_t)b * N + j] = in ? s_path[j] : -1;
     int t = -1;
-    if (in) t = (j < a) ? p.node_tok[(size_t)b * N + s_path[j + 1]] : s_am[s_path[a]];
+    if (in) t = (j < a) ? s_tok[s_path[j + 1]] : bonus;
     p.out_tok[(size_t)b * N + j] = t;
   }
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     p.acc_len[b] = skip ? 0 : a;
-    p.bonus[b] = skip ? -1 : s_am[s_path[a]];
+    p.bonus[b] = bonus;
   }
   if (skip) return;
   // compaction: rows path[0..a] -> L + 0..a on every layer
   const int L = p.cache_len[b];
   const int rows = a + 1;
   const int64_t base_row = p.cache_off[b] + L;
-  const bool v16 = (p.row_bytes % 16 == 0) &&
-                   ((reinterpret_cast<uintptr_t>(p.kv) & 15u) == 0) && (p.layer_stride_bytes % 16 == 0);
-  for (int layer = 0; layer < p.n_layers; ++layer) {
-    unsigned char* lbase = p.kv + layer * p.layer_stride_bytes + base_row * p.row_bytes;
-    if (v16) {
-      const int vpr = p.row_bytes / 16;  // vectors per row
-      for (int r0 = 0; r0 < rows; r0 += kStageRows) {
-        const int nr = min(kStageRows, rows - r0);
-        const int total = nr * vpr;
-        for (int t0 = 0; t0 < total; t0 += kWalkThreads * kStageVec) {
-          uint4 buf[kStageVec];
+  const bool v16 = (p.row_bytes % 16 == 0) && ((reinterpret_cast<uintptr_t>(p.kv) & 15u) == 0) &&
+                   (p.layer_stride_bytes % 16 == 0);
+  const int vb = v16 ? 16 : 4;         // bytes per vector
+  const int vpr = p.row_bytes / vb;    // vectors per row
+  const int per_layer = rows * vpr;
+  const long long total = (long long)per_layer * p.n_layers;
+  for (long long t0 = 0; t0 < total; t0 += (long long)kWalkThreads * kStageVec) {
+    uint4 buf[kStageVec];
 #pragma unroll
-          for (int u = 0; u < kStageVec; ++u) {
-            const int e = t0 + u * kWalkThreads + threadIdx.x;
-            if (e < total) {
-              const int rr = e / vpr, cc = e - rr * vpr;
-              buf[u] = reinterpret_cast<const uint4*>(lbase + (size_t)s_path[r0 + rr] * p.row_bytes)[cc];
-            }
-          }
-          __syncthreads();
-#pragma unroll
-          for (int u = 0; u < kStageVec; ++u) {
-            const int e = t0 + u * kWalkThreads + threadIdx.x;
-            if (e < total) {
-              const int rr = e / vpr, cc = e - rr * vpr;
-              reinterpret_cast<uint4*>(lbase + (size_t)(r0 + rr) * p.row_bytes)[cc] = buf[u];
-            }
-          }
-          __syncthreads();
-        }
-      }
-    } else {
-      const int wpr = p.row_bytes / 4;
-      for (int r0 = 0; r0 < rows; r0 += kStageRows) {
-        const int nr = min(kStageRows, rows - r0);
-        const int total = nr * wpr;
-        for (int t0 = 0; t0 < total; t0 += kWalkThreads * kStageVec) {
-          uint32_t buf[kStageVec];
-#pragma unroll
-          for (int u = 0; u < kStageVec; ++u) {
-            const int e = t0 + u * kWalkThreads + threadIdx.x;
-            if (e < total) {
-              const int rr = e / wpr, cc = e - rr * wpr;
-              buf[u] = reinterpret_cast<const uint32_t*>(lbase + (size_t)s_path[r0 + rr] * p.row_bytes)[cc];
-            }
-          }
-          __syncthreads();
-#pragma unroll
-          for (int u = 0; u < kStageVec; ++u) {
-            const int e = t0 + u * kWalkThreads + threadIdx.x;
-            if (e < total) {
-              const int rr = e / wpr, cc = e - rr * wpr;
-              reinterpret_cast<uint32_t*>(lbase + (size_t)(r0 + rr) * p.row_bytes)[cc] = buf[u];
-            }
-          }
-          __syncthreads();
-        }
+    for (int u = 0; u < kStageVec; ++u) {
+      const long long e = t0 + u * kWalkThreads + tid;
+      if (e < total) {
+        const int layer = (int)(e / per_layer);
+        const int rem = (int)(e - (long long)layer * per_layer);
+        const int rr = rem / vpr, cc = rem - rr * vpr;
+        const unsigned char* src =
+            p.kv + layer * p.layer_stride_bytes + (base_row + s_path[rr]) * p.row_bytes + (size_t)cc * vb;
+        if (v16) buf[u] = *reinterpret_cast<const uint4*>(src);
+        else buf[u].x = *reinterpret_cast<const uint32_t*>(src);
       }
     }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kStageVec; ++u) {
+      const long long e = t0 + u * kWalkThreads + tid;
+      if (e < total) {
+        const int layer = (int)(e / per_layer);
+        const int rem = (int)(e - (long long)layer * per_layer);
+        const int rr = rem / vpr, cc = rem - rr * vpr;
+        unsigned char* dst = p.kv + layer * p.layer_stride_bytes + (base_row + rr) * p.row_bytes + (size_t)cc * vb;
+        if (v16) *reinterpret_cast<uint4*>(dst) = buf[u];
+        else *reinterpret_cast<uint32_t*>(dst) = buf[u].x;
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  if (threadIdx.x == 0) p.cache_len[b] = L + rows;
+  if (tid == 0) p.cache_len[b] = L + rows;
 }
 
-static size_t counter_bytes(int B) { return ((size_t)B * 4 + 255) / 256 * 256; }
+static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+static size_t header_bytes() { return 256; }
+static size_t zeroed_bytes(int B, int N) { return header_bytes() + round256((size_t)B * N * 8); }
 
 size_t accept_workspace_bytes(int B, int N, int V) {
-  const size_t chunks = (size_t)ceil_div(V, kArgmaxChunk);
-  return counter_bytes(B) + (size_t)B * N * chunks * sizeof(unsigned long long);
+  (void)V;
+  return zeroed_bytes(B, N);
+}
+
+static int sm_count() {
+  static int counts[128] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+  if (counts[dev] == 0) {
+    int c = 0;
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
+    counts[dev] = c;
+  }
+  return counts[dev];
 }
 
 int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream) {
-  p.chunks = ceil_div(p.V, kArgmaxChunk);
-  p.counter = static_cast<unsigned*>(workspace);
-  p.partial = reinterpret_cast<unsigned long long*>(static_cast<unsigned char*>(workspace) + counter_bytes(p.B));
-  const unsigned grid = (unsigned)p.chunks * (unsigned)(p.B * p.N);
-  if (p.logits_dtype == DDT_BF16) return launch_pdl(accept_kernel<true>, grid, kArgmaxThreads, 0, stream, p);
-  return launch_pdl(accept_kernel<false>, grid, kArgmaxThreads, 0, stream, p);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  p.abort = reinterpret_cast<int*>(ws);
+  p.rowkey = reinterpret_cast<unsigned long long*>(ws + header_bytes());
+  const size_t esz = p.logits_dtype == DDT_BF16 ? 2 : 4;
+  p.tma = (reinterpret_cast<uintptr_t>(p.logits) % 16 == 0) && (((size_t)p.V * esz) % 16 == 0);
+  const int elems = p.logits_dtype == DDT_BF16 ? SliceCfg<true>::kElems : SliceCfg<false>::kElems;
+  const long long slices = (long long)p.B * p.N * ceil_div(p.V, elems);
+  const long long warps = std::max(1LL, std::min<long long>(slices, (long long)sm_count() * kArgmaxCtasPerSm *
+                                                                        (kArgmaxThreads / 32)));
+  const unsigned grid = (unsigned)((warps + kArgmaxThreads / 32 - 1) / (kArgmaxThreads / 32));
+  const int st = p.logits_dtype == DDT_BF16
+                     ? launch_pdl(accept_argmax_kernel<true>, grid, kArgmaxThreads, 0, stream, p)
+                     : launch_pdl(accept_argmax_kernel<false>, grid, kArgmaxThreads, 0, stream, p);
+  if (st != DDT_OK) return st;
+  return launch_pdl(accept_walk_kernel, (unsigned)p.B, kWalkThreads, 0, stream, p);
 }
 
 // ---------------------------------------------------------------------------
@@ -358,9 +361,10 @@ int launch_accept_compact_noalloc(AcceptParams p, cudaStream_t stream) {
   int st = DDT_OK;
   void* scratch = noalloc_scratch_ptr(&st);
   if (st != DDT_OK) return st;
-  // the counters must start at zero; the array keeps whatever the last call
-  // (on any stream) left there, so clear them on this call's stream first
-  if (cudaMemsetAsync(scratch, 0, counter_bytes(p.B), stream) != cudaSuccess) return DDT_ERR_CUDA;
+  // the status word and row keys must start at zero; the array keeps
+  // whatever the last call (on any stream) left there, so clear them on this
+  // call's stream first
+  if (cudaMemsetAsync(scratch, 0, zeroed_bytes(p.B, p.N), stream) != cudaSuccess) return DDT_ERR_CUDA;
   return launch_accept_compact(p, scratch, stream);
 }
 

@@ -45,9 +45,10 @@ struct AcceptParams {
   int32_t* out_tok;
   int32_t* bonus;
   int32_t* dev_status;
-  unsigned long long* partial;  // [B*N][chunks] packed (value, ~index) keys
-  unsigned* counter;            // [B] chunk arrivals per request (zero between calls)
+  int* abort;                   // workspace status word (DDT_ERR_TIMEOUT after an expired wait)
+  unsigned long long* rowkey;   // [B*N] packed (value, ~index) row maxima (zero between calls)
   int chunks;
+  int tma;                      // logits rows stream by bulk copies (16-byte aligned rows)
 };
 size_t accept_workspace_bytes(int B, int N, int V);
 int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream);

@@ -207,14 +207,17 @@ DDT_API int ddt_verify_attn(const void* q, const void* kv, int64_t kv_rows, cons
  *   copied, cache_len unchanged). Requests with n_nodes[b] == 0 are skipped
  *   the same way with DDT_OK.
  * workspace: ddt_accept_compact_workspace_size(B, N, V) bytes, 256-byte
- *   aligned. It starts with one arrival counter per request (rounded up to
- *   256 bytes) that must be zero before the first call -- zero the buffer once
- *   after allocating it; every call leaves the counters at zero again. The
- *   rest holds one partial argmax key per (row, 16384-entry vocab chunk) and
- *   may hold anything on entry. Calls that share a workspace must not overlap
- *   on the GPU.
- * Runs as one kernel: the CTA that reduces a request's last vocab chunk also
- *   walks that request's tree and compacts its rows.
+ *   aligned: a 256-byte status word, then one 8-byte running argmax key per
+ *   row (B * N, rounded up to 256 bytes). All of it must be zero before the
+ *   first call -- zero the buffer once after allocating it; every call
+ *   leaves it at zero again. Every wait inside the kernels is bounded (about
+ *   2 s); if one expires the status word holds DDT_ERR_TIMEOUT and the
+ *   outputs are not valid (zero the workspace before reusing it). Calls that
+ *   share a workspace must not overlap on the GPU.
+ * Runs as two kernels: the logits stream through shared memory by bulk
+ *   copies on at most one CTA per SM (row maxima by 64-bit atomic max), then
+ *   one CTA per request finds each node's accepted child, walks the path and
+ *   compacts the rows.
  */
 DDT_API size_t ddt_accept_compact_workspace_size(int B, int N, int V);
 
@@ -235,12 +238,13 @@ DDT_API int ddt_accept_compact(const void* logits, int logits_dtype, int V, cons
  * the host application, or a latency-critical decode loop that must not call
  * cudaMalloc (which can synchronise the device). This entry point takes the
  * same arguments as ddt_accept_compact minus the workspace and allocates
- * nothing: its scratch (per-request arrival counters and the partial argmax
- * keys) lives in one fixed 4 MiB array inside the library, which every GPU
+ * nothing: its scratch (status word and per-row argmax keys) lives in one
+ * fixed 4 MiB array inside the library, which every GPU
  * that loads the library keeps until the process exits.
  *
  * Limit: ddt_accept_compact_workspace_size(B, N, V) must be at most 4 MiB
- *   (e.g. B 64 x N 256 x V 163840 needs 1.3 MiB); larger calls return
+ *   (e.g. B 64 x N 256 needs 0.13 MiB, B 512 x N 1024 needs 4.0 MiB + 256 B
+ *   and is rejected); larger calls return
  *   DDT_ERR_UNSUPPORTED without launching anything.
  * Set-up: the first call on each device looks up the array's device address
  *   (with that device current); make that first call before any stream

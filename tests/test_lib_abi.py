@@ -45,10 +45,20 @@ def test_status_strings_and_version(so):
     assert lib.version() >= 100
 
 
+def _r256(x):
+    return (x + 255) // 256 * 256
+
+
+def _accept_ws(B, N, V):
+    """The layout ddt.h documents: a 256-byte status word, then one 8-byte
+    running argmax key per row, rounded up to 256 bytes."""
+    return 256 + _r256(B * N * 8)
+
+
 def test_workspace_queries(so):
-    # accept: per-request counters (256-byte block) + one 8-byte key per (row, 16384-entry vocab chunk)
-    assert lib.accept_compact_workspace_size(1, 64, 163840) == 256 + 64 * 10 * 8
-    assert lib.accept_compact_workspace_size(65, 8, 16384) == 512 + 65 * 8 * 8
+    assert lib.accept_compact_workspace_size(1, 64, 163840) == _accept_ws(1, 64, 163840) == 256 + 512
+    assert lib.accept_compact_workspace_size(65, 8, 16384) == _accept_ws(65, 8, 16384)
+    assert lib.accept_compact_workspace_size(64, 256, 163840) < 4 << 20  # fits the no-alloc scratch
     assert lib.accept_compact_workspace_size(0, 64, 10) == 0
     assert so.ddt_verify_attn_workspace_size(1, 8, 4, 64, 16, 32, 0) == 0  # f32 path needs none
 
@@ -70,10 +80,11 @@ def test_host_validation_without_gpu(so):
 
 
 def test_noalloc_accept_rejects_sizes_beyond_its_array(so):
-    # 64 x 1024 rows x 10 vocab chunks of 8-byte keys = 5.2 MiB > the 4 MiB array:
+    # 512 x 1024 rows of 8-byte keys + the 256-byte status word > the 4 MiB array:
     # rejected on the host before anything touches the GPU
     p = ctypes.c_void_p(256)
-    st = so.ddt_accept_compact_noalloc(p, 1, 163840, p, p, p, 64, 1024, p, 1, 576, 1, 0, p, p, p, p, p, p, p, p, p,
+    assert lib.accept_compact_workspace_size(512, 1024, 163840) > 4 << 20
+    st = so.ddt_accept_compact_noalloc(p, 1, 163840, p, p, p, 512, 1024, p, 1, 576, 1, 0, p, p, p, p, p, p, p, p, p,
                                        None)
     assert st == lib.DDT_ERR_UNSUPPORTED
     st = so.ddt_accept_compact_noalloc(None, 1, 163840, p, p, p, 1, 64, p, 1, 576, 1, 0, p, p, p, p, p, p, p, p, p,
