@@ -273,44 +273,41 @@ __global__ void __launch_bounds__(32) build_tree_kernel(BuildParams p) {
 // (beyond the number of pops left) are dropped, which keeps the frontier
 // within min(pops + 1, N - 1 - pops) <= 32 * SPL entries for N <= 64 * SPL.
 //
-// An entry is six 32-bit words: A = order key of the score << 32 | (127 -
-// depth) (larger is better when scores or depths differ), the packed rank
-// tuple k (smaller is better when A ties), aux = last rank << 16 | parent
-// node, and the parent's score ps (for the next sibling's score). The score
-// itself is recovered exactly from A.
+// An entry is five 32-bit words: hi = order key of the score (scores are
+// <= 0, so the key is the complement of the bits of score + 0, which maps -0
+// to +0; larger is better), aux = (127 - depth) << 24 | last rank << 16 |
+// parent node, the packed rank tuple k (two words; smaller is better when
+// score and depth tie) and the parent's score ps (for the next sibling). The
+// score itself is recovered exactly from hi. Comparisons are branch-free.
 // ---------------------------------------------------------------------------
 struct FEntry {
-  uint64_t A, k;
-  uint32_t aux;
+  uint32_t hi, aux;
+  uint64_t k;
   float ps;
 };
 
 __device__ __forceinline__ bool fbetter(const FEntry& a, const FEntry& b) {
-  return a.A > b.A || (a.A == b.A && a.k < b.k);
+  const uint32_t da = a.aux >> 24, db = b.aux >> 24;
+  return (a.hi > b.hi) | ((a.hi == b.hi) & ((da > db) | ((da == db) & (a.k < b.k))));
 }
 
-__device__ __forceinline__ float order_key_to_float(uint32_t u) {
-  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
-}
-
-__device__ __forceinline__ uint64_t entry_key(float sc, int d) {
-  return (static_cast<uint64_t>(float_order_key(sc)) << 32) | static_cast<uint32_t>(127 - d);
-}
+__device__ __forceinline__ uint32_t score_key(float sc) { return ~__float_as_uint(__fadd_rn(sc, 0.0f)); }
+__device__ __forceinline__ float key_score(uint32_t hi) { return __uint_as_float(~hi); }
 
 __device__ __forceinline__ FEntry fshfl(const FEntry& e, int src) {
   FEntry o;
-  o.A = __shfl_sync(DDT_FULL_MASK, e.A, src);
-  o.k = __shfl_sync(DDT_FULL_MASK, e.k, src);
+  o.hi = __shfl_sync(DDT_FULL_MASK, e.hi, src);
   o.aux = __shfl_sync(DDT_FULL_MASK, e.aux, src);
+  o.k = __shfl_sync(DDT_FULL_MASK, e.k, src);
   o.ps = __shfl_sync(DDT_FULL_MASK, e.ps, src);
   return o;
 }
 
 __device__ __forceinline__ FEntry fsel(bool c, const FEntry& a, const FEntry& b) {
   FEntry o;
-  o.A = c ? a.A : b.A;
-  o.k = c ? a.k : b.k;
+  o.hi = c ? a.hi : b.hi;
   o.aux = c ? a.aux : b.aux;
+  o.k = c ? a.k : b.k;
   o.ps = c ? a.ps : b.ps;
   return o;
 }
@@ -324,9 +321,8 @@ __global__ void __launch_bounds__(32) build_tree_sorted_kernel(BuildParams p) {
   const int lane = threadIdx.x;
   const int N = p.N, D = p.D, K = p.K, W = p.W, bpl = p.bpl;
   int32_t* n_parent = reinterpret_cast<int32_t*>(smem_raw);
-  int32_t* n_dep = n_parent + N;
-  int32_t* n_tok = n_dep + N;
-  float* n_sc = reinterpret_cast<float*>(n_tok + N);
+  int32_t* n_dr = n_parent + N;  // depth << 8 | last rank
+  float* n_sc = reinterpret_cast<float*>(n_dr + N);
   float* lp = n_sc + N;
   int32_t* tk = reinterpret_cast<int32_t*>(lp + D * K);
   const int L = p.cache_len[b];
@@ -344,12 +340,12 @@ __global__ void __launch_bounds__(32) build_tree_sorted_kernel(BuildParams p) {
   if (!bad) {
     FEntry fr[SPL];
 #pragma unroll
-    for (int q = 0; q < SPL; ++q) fr[q] = FEntry{0ull, 0ull, 0u, 0.0f};
+    for (int q = 0; q < SPL; ++q) fr[q] = FEntry{0u, 0u, 0ull, 0.0f};
     if (lane == 0) {
-      fr[0].A = entry_key(__fadd_rn(0.0f, lp[0]), 1);  // rank 0 at depth 1, parent = root
+      fr[0].hi = score_key(__fadd_rn(0.0f, lp[0]));  // rank 0 at depth 1, parent = root
+      fr[0].aux = (127u - 1u) << 24;
       n_parent[0] = -1;
-      n_dep[0] = 0;
-      n_tok[0] = root;
+      n_dr[0] = 0;
       n_sc[0] = 0.0f;
     }
     int fsize = (N > 1) ? 1 : 0;
@@ -357,24 +353,21 @@ __global__ void __launch_bounds__(32) build_tree_sorted_kernel(BuildParams p) {
     while (n < N && fsize > 0) {
       // pop entry 0 (lane 0, register 0)
       const FEntry w = fshfl(fr[0], 0);
-      const int wd = 127 - static_cast<int>(static_cast<uint32_t>(w.A));
-      const float wsc = order_key_to_float(static_cast<uint32_t>(w.A >> 32));
-      const int wr = static_cast<int>(w.aux >> 16), wpar = static_cast<int>(w.aux & 0xffffu);
+      const int wd = 127 - static_cast<int>(w.aux >> 24);
+      const int wr = static_cast<int>((w.aux >> 16) & 0xffu), wpar = static_cast<int>(w.aux & 0xffffu);
+      const float wsc = key_score(w.hi);
       const int i = n;
       // successors: first child (rank 0 one level down) and next sibling
       const bool has_c = wd < D, has_s = wr + 1 < K;
       const float lc = lp[has_c ? wd * K : 0];
       const float ls = lp[has_s ? (wd - 1) * K + wr + 1 : 0];
-      const FEntry c{entry_key(__fadd_rn(wsc, lc), wd + 1), w.k << bpl, static_cast<uint32_t>(i), wsc};
-      const FEntry sb{entry_key(__fadd_rn(w.ps, ls), wd), w.k + 1ull, w.aux + 0x10000u, w.ps};
-      if (lane == 0) {
-        n_parent[i] = wpar;
-        n_dep[i] = wd;
-        n_tok[i] = tk[(wd - 1) * K + wr];
-        n_sc[i] = wsc;
-      }
+      const FEntry c{score_key(__fadd_rn(wsc, lc)), ((uint32_t)(126 - wd) << 24) | (uint32_t)i, w.k << bpl, wsc};
+      const FEntry sb{score_key(__fadd_rn(w.ps, ls)), w.aux + 0x10000u, w.k + 1ull, w.ps};
+      if (lane == 0) n_parent[i] = wpar;
+      if (lane == 0) n_dr[i] = (wd << 8) | wr;
+      if (lane == 0) n_sc[i] = wsc;
       const int ns = (int)has_c + (int)has_s;
-      const bool c_first = has_c && (!has_s || fbetter(c, sb));
+      const bool c_first = has_c & (!has_s | fbetter(c, sb));
       const FEntry s0 = fsel(c_first, c, sb);
       const FEntry s1 = fsel(c_first, sb, c);
       // ranks of the successors among the remaining entries (old 1 .. fsize-1)
@@ -382,9 +375,9 @@ __global__ void __launch_bounds__(32) build_tree_sorted_kernel(BuildParams p) {
 #pragma unroll
       for (int q = 0; q < SPL; ++q) {
         const int f = 32 * q + lane;
-        const bool valid = f >= 1 && f < fsize;
-        p0 += __popc(__ballot_sync(DDT_FULL_MASK, valid && fbetter(fr[q], s0)));
-        p1 += __popc(__ballot_sync(DDT_FULL_MASK, valid && fbetter(fr[q], s1)));
+        const bool valid = (f >= 1) & (f < fsize);
+        p0 += __popc(__ballot_sync(DDT_FULL_MASK, valid & fbetter(fr[q], s0)));
+        p1 += __popc(__ballot_sync(DDT_FULL_MASK, valid & fbetter(fr[q], s1)));
       }
       if (ns == 0) p0 = 32 * SPL;  // every entry moves up by one
       // merge: new entry f comes from old f + 1 (f < p0), s0 (f == p0), old f
@@ -417,10 +410,12 @@ __global__ void __launch_bounds__(32) build_tree_sorted_kernel(BuildParams p) {
     __syncwarp();
     // outputs (coalesced) and ancestor masks
     for (int j = lane; j < n; j += 32) {
-      o_tok[j] = n_tok[j];
+      const int dr = n_dr[j];
+      const int d = dr >> 8;
+      o_tok[j] = j == 0 ? root : tk[(d - 1) * K + (dr & 0xff)];
       o_par[j] = n_parent[j];
-      o_dep[j] = n_dep[j];
-      o_pos[j] = L + n_dep[j];
+      o_dep[j] = d;
+      o_pos[j] = L + d;
       o_sc[j] = n_sc[j];
     }
     write_masks(o_mask, W, n, n_parent, lane);
@@ -434,7 +429,7 @@ __global__ void __launch_bounds__(32) build_tree_sorted_kernel(BuildParams p) {
 
 template <int SPL>
 static int launch_sorted(const BuildParams& p, cudaStream_t stream) {
-  const size_t smem = (size_t)p.N * 16 + (size_t)p.D * p.K * 8;
+  const size_t smem = (size_t)p.N * 12 + (size_t)p.D * p.K * 8;
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(build_tree_sorted_kernel<SPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
