@@ -42,6 +42,29 @@ L2_BYTES = 126 * 1024 * 1024
 # ---------------------------------------------------------------------------
 
 
+def profiled_traffic(shape: synth.Shape):
+    """DRAM bytes (read + write) of one verify-attention launch from the ncu
+    capture summarised in profiles/attn_tc_<workload>.md, or None when there is
+    no capture of this workload or the kernel sources changed since it was
+    taken (the summary records their sha256)."""
+    import hashlib
+    import re
+    tag = {"kimi-1req-L4096-N64": "kimi-1req"}.get(shape.name)
+    path = os.path.join(ROOT, "profiles", f"attn_tc_{tag}.md") if tag else None
+    if not path or not os.path.exists(path):
+        return None
+    text = open(path).read()
+    for fname, digest in re.findall(r"^\s+(\S+\.cuh?)\s+([0-9a-f]{64})\s*$", text, re.M):
+        src = os.path.join(ROOT, "ddtree_speculative_decode_b200", "csrc", fname)
+        if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != digest:
+            return None
+    rd = re.search(r"\| dram__bytes_read\.sum \| ([0-9.]+) MB \|", text)
+    wr = re.search(r"\| dram__bytes_write\.sum \| ([0-9.]+) (MB|B)", text)
+    if not rd or not wr:
+        return None
+    return float(rd.group(1)) * 1e6 + float(wr.group(1)) * (1e6 if wr.group(2) == "MB" else 1.0)
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -314,7 +337,7 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
                                       "l2": f"{n_sets} rotating input sets of {set_bytes / 2**20:.1f} MiB "
                                             f"(> 2x 126 MiB L2)"}),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": profiled_traffic(shape),
                      "kernel": "ddt_verify_attn", "peak_kind": f"bf16 dense, sustained, {pk['source']}"},
         "stages_ms": {"build_tree": build_ms, "verify_attn": attn_ms, "accept_compact": accept_ms},
         "accept_hbm": {"achieved_gbs": acc_bytes / (accept_ms / 1e3) / 1e9, "peak_gbs": pk["hbm_gbs"],
