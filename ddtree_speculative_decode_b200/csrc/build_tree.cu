@@ -427,6 +427,162 @@ __global__ void __launch_bounds__(32) build_tree_sorted_kernel(BuildParams p) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Packed-key variant of the sorted frontier, used when the rank tuples of
+// every entry that can exist fit 25 bits (bpl * min(D, N) <= 25, e.g. K 8 x
+// D 8): the whole order is then one 64-bit integer,
+//   key = score key << 32 | (127 - depth) << 25 | (2^25 - 1 - k),
+// larger is better, and an entry is four words (key, rank << 16 | parent,
+// parent's score). Same pop / merge as build_tree_sorted_kernel.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kKMask = (1u << 25) - 1u;
+
+struct PEntry {
+  uint64_t key;
+  uint32_t aux;
+  float ps;
+};
+
+__device__ __forceinline__ PEntry pshfl(const PEntry& e, int src) {
+  PEntry o;
+  o.key = __shfl_sync(DDT_FULL_MASK, e.key, src);
+  o.aux = __shfl_sync(DDT_FULL_MASK, e.aux, src);
+  o.ps = __shfl_sync(DDT_FULL_MASK, e.ps, src);
+  return o;
+}
+
+__device__ __forceinline__ PEntry psel(bool c, const PEntry& a, const PEntry& b) {
+  PEntry o;
+  o.key = c ? a.key : b.key;
+  o.aux = c ? a.aux : b.aux;
+  o.ps = c ? a.ps : b.ps;
+  return o;
+}
+
+__device__ __forceinline__ uint64_t packed_key(float sc, int d, uint32_t k) {
+  return (static_cast<uint64_t>(score_key(sc)) << 32) | (static_cast<uint64_t>(127 - d) << 25) |
+         static_cast<uint64_t>(kKMask - k);
+}
+
+template <int SPL>
+__global__ void __launch_bounds__(32) build_tree_packed_kernel(BuildParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int b = blockIdx.x;
+  const int lane = threadIdx.x;
+  const int N = p.N, D = p.D, K = p.K, W = p.W, bpl = p.bpl;
+  int32_t* n_parent = reinterpret_cast<int32_t*>(smem_raw);
+  int32_t* n_dr = n_parent + N;  // depth << 8 | last rank
+  float* n_sc = reinterpret_cast<float*>(n_dr + N);
+  float* lp = n_sc + N;
+  int32_t* tk = reinterpret_cast<int32_t*>(lp + D * K);
+  const int L = p.cache_len[b];
+  const int root = p.root_tok[b];
+  const bool bad = load_drafter(p, b, lp, tk, lane);
+
+  int32_t* o_tok = p.node_tok + (size_t)b * N;
+  int32_t* o_par = p.parent + (size_t)b * N;
+  int32_t* o_dep = p.depth + (size_t)b * N;
+  int32_t* o_pos = p.pos + (size_t)b * N;
+  float* o_sc = p.score + (size_t)b * N;
+  uint32_t* o_mask = p.mask + (size_t)b * N * W;
+
+  int n = 0;
+  if (!bad) {
+    PEntry fr[SPL];
+#pragma unroll
+    for (int q = 0; q < SPL; ++q) fr[q] = PEntry{0ull, 0u, 0.0f};
+    if (lane == 0) {
+      fr[0].key = packed_key(__fadd_rn(0.0f, lp[0]), 1, 0u);  // rank 0 at depth 1, parent = root
+      n_parent[0] = -1;
+      n_dr[0] = 0;
+      n_sc[0] = 0.0f;
+    }
+    int fsize = (N > 1) ? 1 : 0;
+    n = 1;
+    while (n < N && fsize > 0) {
+      const PEntry w = pshfl(fr[0], 0);
+      const int wd = 127 - static_cast<int>((w.key >> 25) & 0x7fu);
+      const uint32_t wk = kKMask - static_cast<uint32_t>(w.key & kKMask);
+      const float wsc = key_score(static_cast<uint32_t>(w.key >> 32));
+      const int wr = static_cast<int>(w.aux >> 16), wpar = static_cast<int>(w.aux & 0xffffu);
+      const int i = n;
+      const bool has_c = wd < D, has_s = wr + 1 < K;
+      const float lc = lp[has_c ? wd * K : 0];
+      const float ls = lp[has_s ? (wd - 1) * K + wr + 1 : 0];
+      const PEntry c{packed_key(__fadd_rn(wsc, lc), wd + 1, wk << bpl), static_cast<uint32_t>(i), wsc};
+      const PEntry sb{packed_key(__fadd_rn(w.ps, ls), wd, wk + 1u), w.aux + 0x10000u, w.ps};
+      if (lane == 0) n_parent[i] = wpar;
+      if (lane == 0) n_dr[i] = (wd << 8) | wr;
+      if (lane == 0) n_sc[i] = wsc;
+      const int ns = (int)has_c + (int)has_s;
+      const bool c_first = has_c & (!has_s | (c.key > sb.key));
+      const PEntry s0 = psel(c_first, c, sb);
+      const PEntry s1 = psel(c_first, sb, c);
+      int p0 = 0, p1 = 0;
+#pragma unroll
+      for (int q = 0; q < SPL; ++q) {
+        const int f = 32 * q + lane;
+        const bool valid = (f >= 1) & (f < fsize);
+        p0 += __popc(__ballot_sync(DDT_FULL_MASK, valid & (fr[q].key > s0.key)));
+        p1 += __popc(__ballot_sync(DDT_FULL_MASK, valid & (fr[q].key > s1.key)));
+      }
+      if (ns == 0) p0 = 32 * SPL;
+      PEntry nf[SPL];
+#pragma unroll
+      for (int q = 0; q < SPL; ++q) {
+        const int f = 32 * q + lane;
+        const int delta = 1 - (f > p0 ? 1 : 0) - ((ns == 2 && f > p1 + 1) ? 1 : 0);
+        const int src = (lane + delta) & 31;
+        PEntry v = pshfl(fr[q], src);
+        if (q + 1 < SPL) {
+          const PEntry t = pshfl(fr[q + 1 < SPL ? q + 1 : q], src);
+          v = psel(lane == 31 && delta == 1, t, v);
+        }
+        if (q > 0) {
+          const PEntry t = pshfl(fr[q > 0 ? q - 1 : q], src);
+          v = psel(lane == 0 && delta == -1, t, v);
+        }
+        v = psel(f == p0, s0, v);
+        v = psel(ns == 2 && f == p1 + 1, s1, v);
+        nf[q] = v;
+      }
+#pragma unroll
+      for (int q = 0; q < SPL; ++q) fr[q] = nf[q];
+      ++n;
+      fsize = min(min(fsize - 1 + ns, N - n), 32 * SPL);
+    }
+    __syncwarp();
+    for (int j = lane; j < n; j += 32) {
+      const int dr = n_dr[j];
+      const int d = dr >> 8;
+      o_tok[j] = j == 0 ? root : tk[(d - 1) * K + (dr & 0xff)];
+      o_par[j] = n_parent[j];
+      o_dep[j] = d;
+      o_pos[j] = L + d;
+      o_sc[j] = n_sc[j];
+    }
+    write_masks(o_mask, W, n, n_parent, lane);
+  }
+  write_pads(o_tok, o_par, o_dep, o_pos, o_sc, o_mask, W, n, N, lane);
+  if (lane == 0) {
+    p.n_nodes[b] = n;
+    if (p.dev_status) p.dev_status[b] = bad ? DDT_ERR_INPUT : DDT_OK;
+  }
+}
+
+template <int SPL>
+static int launch_packed(const BuildParams& p, cudaStream_t stream) {
+  const size_t smem = (size_t)p.N * 12 + (size_t)p.D * p.K * 8;
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(build_tree_packed_kernel<SPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return DDT_ERR_CUDA;
+  }
+  return launch_pdl(build_tree_packed_kernel<SPL>, (unsigned)p.B, 32, smem, stream, p);
+}
+
 template <int SPL>
 static int launch_sorted(const BuildParams& p, cudaStream_t stream) {
   const size_t smem = (size_t)p.N * 12 + (size_t)p.D * p.K * 8;
@@ -439,6 +595,12 @@ static int launch_sorted(const BuildParams& p, cudaStream_t stream) {
 }
 
 int launch_build_tree(const BuildParams& p, cudaStream_t stream) {
+  // every entry that can exist has depth <= min(D, N): its rank tuple needs
+  // bpl bits per level
+  const bool packed = (long long)p.bpl * (p.D < p.N ? p.D : p.N) <= 25;
+  if (packed && p.N <= 64) return launch_packed<1>(p, stream);
+  if (packed && p.N <= 128) return launch_packed<2>(p, stream);
+  if (packed && p.N <= 256) return launch_packed<4>(p, stream);
   if (p.N <= 64) return launch_sorted<1>(p, stream);
   if (p.N <= 128) return launch_sorted<2>(p, stream);
   if (p.N <= 256) return launch_sorted<4>(p, stream);
