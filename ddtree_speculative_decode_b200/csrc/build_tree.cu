@@ -363,9 +363,11 @@ __global__ void __launch_bounds__(32) build_tree_sorted_kernel(BuildParams p) {
       const float ls = lp[has_s ? (wd - 1) * K + wr + 1 : 0];
       const FEntry c{score_key(__fadd_rn(wsc, lc)), ((uint32_t)(126 - wd) << 24) | (uint32_t)i, w.k << bpl, wsc};
       const FEntry sb{score_key(__fadd_rn(w.ps, ls)), w.aux + 0x10000u, w.k + 1ull, w.ps};
-      if (lane == 0) n_parent[i] = wpar;
-      if (lane == 0) n_dr[i] = (wd << 8) | wr;
-      if (lane == 0) n_sc[i] = wsc;
+      // node record: warp-uniform values stored by every lane (one wavefront
+      // each, no divergent branch)
+      n_parent[i] = wpar;
+      n_dr[i] = (wd << 8) | wr;
+      n_sc[i] = wsc;
       const int ns = (int)has_c + (int)has_s;
       const bool c_first = has_c & (!has_s | fbetter(c, sb));
       const FEntry s0 = fsel(c_first, c, sb);
@@ -513,9 +515,11 @@ __global__ void __launch_bounds__(32) build_tree_packed_kernel(BuildParams p) {
       const float ls = lp[has_s ? (wd - 1) * K + wr + 1 : 0];
       const PEntry c{packed_key(__fadd_rn(wsc, lc), wd + 1, wk << bpl), static_cast<uint32_t>(i), wsc};
       const PEntry sb{packed_key(__fadd_rn(w.ps, ls), wd, wk + 1u), w.aux + 0x10000u, w.ps};
-      if (lane == 0) n_parent[i] = wpar;
-      if (lane == 0) n_dr[i] = (wd << 8) | wr;
-      if (lane == 0) n_sc[i] = wsc;
+      // node record: warp-uniform values stored by every lane (one wavefront
+      // each, no divergent branch)
+      n_parent[i] = wpar;
+      n_dr[i] = (wd << 8) | wr;
+      n_sc[i] = wsc;
       const int ns = (int)has_c + (int)has_s;
       const bool c_first = has_c & (!has_s | (c.key > sb.key));
       const PEntry s0 = psel(c_first, c, sb);
