@@ -265,20 +265,23 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
     acc_bytes = float(t_host["n_nodes"].sum()) * shape.V * (2 if bf else 4)
 
     def step(s, ev=None):
-        cl.copy_(cl0, non_blocking=True)
+        st = torch.cuda.current_stream(dev)  # the capture stream while a graph is recorded
+        # restore cache_len (the accept advances it) with a small kernel rather
+        # than a memcpy, which would break the chain of programmatic launches
+        torch.add(cl0, 0, out=cl)
         if ev is not None:
-            ev[0].record(stream)
-        lib.build_tree(logp, tok, root, cl, N, out=tree, stream=stream)
+            ev[0].record(st)
+        lib.build_tree(logp, tok, root, cl, N, out=tree, stream=st)
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record(st)
         lib.verify_attn(s["q"], s["kv"], off, cl, tree["mask"], tree["n_nodes"], shape.d_l, shape.d_r, shape.scale,
-                        maxL, out=out, lse=lse, workspace=ws_attn, stream=stream)
+                        maxL, out=out, lse=lse, workspace=ws_attn, stream=st)
         if ev is not None:
-            ev[2].record(stream)
+            ev[2].record(st)
         lib.accept_compact(s["logits"], tree["node_tok"], tree["parent"], tree["n_nodes"], s["kv"], off, cl, cap,
-                           out=acc, workspace=ws_acc, stream=stream)
+                           out=acc, workspace=ws_acc, stream=st)
         if ev is not None:
-            ev[3].record(stream)
+            ev[3].record(st)
 
     # ---- warm-up ---------------------------------------------------------------
     uuid = None
@@ -292,10 +295,28 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
     for w in range(args.warmup):
         step(sets[w % n_sets])
     torch.cuda.synchronize()
+    # one CUDA graph per input set holds one whole step (the library's launches
+    # keep their programmatic-launch edges), so the timed loop is not bound by
+    # Python's per-call cost; --no-graph times plain calls instead
+    graphs = None
+    if args.graph:
+        try:
+            graphs = []
+            for k in range(n_sets):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    step(sets[k])
+                graphs.append(g)
+            for k in range(max(3, n_sets)):
+                graphs[k % n_sets].replay()
+            torch.cuda.synchronize()
+        except Exception as e:  # capture unsupported here: fall back to plain calls
+            print(f"graph capture failed ({e}); timing plain calls", file=sys.stderr)
+            graphs = None
+            torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     # ---- timed region: exactly K steps ------------------------------------------
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
@@ -303,13 +324,23 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
         dist.barrier()
     t_start.record(stream)
     for k in range(args.steps):
-        step(sets[k % n_sets], evs[k])
+        if graphs is not None:
+            graphs[k % n_sets].replay()
+        else:
+            step(sets[k % n_sets])
     t_end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
     clocks = sampler.stop()
+    # ---- per-stage breakdown (a separate pass: events between the kernels
+    # would cut their programmatic overlap inside the timed region) ----------------
+    n_stage = min(args.steps, 300)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_stage)]
+    for k in range(n_stage):
+        step(sets[k % n_sets], evs[k])
+    torch.cuda.synchronize()
     build_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     accept_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
@@ -347,6 +378,7 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
         "gpu_launches": launches_per_step * args.steps,
         "e2e": e2e,
         "clocks": clocks,
+        "timed_loop": "cuda-graph replays of the step" if graphs is not None else "plain library calls",
     }
     if args.cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(args, shape, x, logits_h, t_host)
@@ -447,6 +479,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--ref-nodes", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="time plain library calls instead of CUDA-graph replays of the step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
