@@ -157,18 +157,26 @@ __device__ __forceinline__ UnitInfo unit_info(const TcParams& p, int unit) {
   u.n = p.n_nodes[u.b];
   u.nkeys = u.L + u.n;
   const int tiles = (u.nkeys + kTileKeys - 1) / kTileKeys;
-  const int per = (tiles + p.splits - 1) / p.splits;
-  const int t0 = min(tiles, u.split * per);
-  const int t1 = min(tiles, t0 + per);
+  // splits get floor or ceil(tiles / splits) tiles, the larger shares last
+  // (where the request's ragged last tile is); splits past `tiles` get none
+  u.active = min(p.splits, tiles);
+  const int t0 = u.split < u.active ? (int)((long long)u.split * tiles / u.active) : tiles;
+  const int t1 = u.split < u.active ? (int)((long long)(u.split + 1) * tiles / u.active) : tiles;
   u.T = t1 - t0;
   u.kb = t0 * kTileKeys;
   u.ke = min(u.nkeys, t1 * kTileKeys);
-  u.active = per > 0 ? (tiles + per - 1) / per : 0;
   // a row tile whose first node is already a pad node has nothing to compute
   const int first_node = (u.rt * 128) / p.H;
   u.pad_tile = u.n <= 0 || first_node >= u.n;
   if (u.pad_tile) u.T = 0;
   return u;
+}
+
+// 64-key groups of the unit's tile t that hold at least one key of the unit
+// (the last tile of a request can be ragged: P.V skips its empty groups)
+__device__ __forceinline__ int live_groups(const UnitInfo& u, int t) {
+  const int tile0 = u.kb + t * kTileKeys;
+  return min(4, (u.ke - tile0 + 63) / 64);
 }
 
 // first pool row (relative to the request) that key group g0 is loaded from:
@@ -352,7 +360,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int t = 0; t < u.T; ++t) {
       const int tile0 = u.kb + t * kTileKeys;
       bool ok = true;
-      for (int g = 0; g < 4; ++g) {
+      const int ng = live_groups(u, t);
+      for (int g = 0; g < ng; ++g) {
         if (!mbar_wait(bar(kBarVEmpty + rg.slot), rg.phase ^ 1u, abort)) {
           ok = false;
           break;
@@ -402,7 +411,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int t = 0; t < u.T && ok; ++t) {
         if (!mbar_wait(bar(kBarPFull), (uint32_t)(t & 1), abort)) { ok = false; break; }
         tc_fence_after();
-        for (int g = 0; g < 4; ++g) {
+        const int ng = live_groups(u, t);
+        for (int g = 0; g < ng; ++g) {
           if (!mbar_wait(bar(kBarVFull + rg.slot), rg.phase, abort)) { ok = false; break; }
           const uint32_t a0 = sbase + kOffP + g * kBoxBytes;
           const uint32_t b0 = sbase + kOffVRing + rg.slot * kVStageBytes;
