@@ -94,7 +94,9 @@ constexpr int kBarSEmpty = kBarSFull + 2;             // [2] leader: S buffer re
 constexpr int kBarPFull = kBarSEmpty + 2;             // leader: P written (softmax warps of both CTAs)
 constexpr int kBarOFull = kBarPFull + 1;              // each CTA: PV finished
 constexpr int kBarEpi = kBarOFull + 1;                // [4] each CTA: epilogue tile loads, one per 32-dim chunk
-constexpr int kNumBars = kBarEpi + 4;
+constexpr int kBarXReady = kBarEpi + 4;               // each CTA: the other split's CTA of these rows is done with its MMAs
+constexpr int kBarXData = kBarXReady + 1;             // each CTA: the other split's partial has landed here (bulk copy)
+constexpr int kNumBars = kBarXData + 1;
 constexpr int kOffRed = kOffMisc + 256;                 // float [2 parity][4 groups][64]
 constexpr int kOffLred = kOffRed + 2 * 4 * 64 * 4;      // float [4][64]
 constexpr int kOffMask = kOffLred + 4 * 64 * 4;         // uint32 [64][kMaxW]
@@ -127,6 +129,7 @@ struct TcParams {
   int B, N, H, W;
   float scale_log2;  // scale * log2(e)
   int splits;
+  int csize;         // CTAs per cluster: 2 (one pair), or 4 (both key splits of a row tile, splits == 2)
   int rowtiles;      // per request: ceil(N * H / 128)
   int out_dtype;
   void* out;
@@ -215,7 +218,7 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   return v;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                    const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_part, TcParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -224,9 +227,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   pdl_wait();
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
+  // A CTA pair (ranks 2k, 2k + 1 of the cluster) runs one unit with the
+  // 2-CTA MMA; a cluster of 4 holds both key splits of one row tile, so the
+  // splits merge through distributed shared memory.
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t rank = crank & 1u;    // CTA within its pair
+  const uint32_t pbase = crank & ~1u;  // cluster rank of the pair's leader CTA
   const bool leader = rank == 0;
-  const int unit = blockIdx.x >> 1;
+  const uint16_t pmask = (uint16_t)(0x3u << pbase);
+  const int unit = p.csize == 4 ? (int)((blockIdx.x >> 2) * 2 + (crank >> 1)) : (int)(blockIdx.x >> 1);
   const UnitInfo u = unit_info(p, unit);
   const int rows_total = p.B * p.N * p.H;
   const int req_rows = p.N * p.H;
@@ -235,28 +244,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) -> uint32_t { return sbase + kOffMisc + 8u * (uint32_t)i; };
 
   // ---------------------------------------------------------------- empty unit
-  if (u.T == 0) {
-    // a split past the last one that gets keys has nothing to do; a row tile
-    // of pad rows only is written (zeros, lse -inf) by split 0
-    if (!u.pad_tile || u.split != 0) return;
-    for (int r = threadIdx.x; r < 64; r += kThreads) {
-      const int rr = row0 + r;
-      if (rr >= req_rows) continue;
-      const size_t grow = (size_t)u.b * req_rows + rr;
-      if (p.lse) p.lse[grow] = -INFINITY;
-    }
-    for (int e = threadIdx.x; e < 64 * (kDL / 4); e += kThreads) {
-      const int r = e / (kDL / 4), c4 = e % (kDL / 4);
-      const int rr = row0 + r;
-      if (rr >= req_rows) continue;
-      const size_t grow = (size_t)u.b * req_rows + rr;
-      if (p.out_dtype == DDT_F32) {
-        reinterpret_cast<float4*>(static_cast<float*>(p.out) + grow * kDL)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
-      } else {
-        reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out) + grow * kDL)[c4] = make_uint2(0u, 0u);
+  // a split past the last one that gets keys has nothing to do; a row tile of
+  // pad rows only is written (zeros, lse -inf) by split 0. In a 4-CTA cluster
+  // an idle pair still takes part in the cluster-wide barriers below.
+  const bool idle = u.T == 0;
+  if (idle) {
+    if (u.pad_tile && u.split == 0) {
+      for (int r = threadIdx.x; r < 64; r += kThreads) {
+        const int rr = row0 + r;
+        if (rr >= req_rows) continue;
+        const size_t grow = (size_t)u.b * req_rows + rr;
+        if (p.lse) p.lse[grow] = -INFINITY;
+      }
+      for (int e = threadIdx.x; e < 64 * (kDL / 4); e += kThreads) {
+        const int r = e / (kDL / 4), c4 = e % (kDL / 4);
+        const int rr = row0 + r;
+        if (rr >= req_rows) continue;
+        const size_t grow = (size_t)u.b * req_rows + rr;
+        if (p.out_dtype == DDT_F32) {
+          reinterpret_cast<float4*>(static_cast<float*>(p.out) + grow * kDL)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+          reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out) + grow * kDL)[c4] = make_uint2(0u, 0u);
+        }
       }
     }
-    return;
+    if (p.csize == 2) return;
   }
 
   // ---------------------------------------------------------------- setup
@@ -276,6 +288,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(bar(kBarPFull), 2 * kSoftmaxWarps);
     mbar_init(bar(kBarOFull), 1);
     for (int c = 0; c < 4; ++c) mbar_init(bar(kBarEpi + c), 1);
+    mbar_init(bar(kBarXReady), kSoftmaxWarps);
+    mbar_init(bar(kBarXData), 1);
     fence_mbar_init_cluster();
   }
   if (warp == 0 && lane == 0) {
@@ -309,10 +323,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int slot = 0;
     uint32_t phase = 0;
   };
-  if (warp == 0 && lane == 0) {
+  if (idle) {
+    // nothing to compute: straight to the cluster-wide teardown
+  } else if (warp == 0 && lane == 0) {
     // ============================================================ QK producer
     // per tile and 64-dim chunk: this CTA's Q chunk and its 128 keys' chunk
-    const uint32_t full0 = map_to_rank(bar(kBarKFull), 0);
+    const uint32_t full0 = map_to_rank(bar(kBarKFull), pbase);
     Ring rg;
     const int qrow = u.b * req_rows + row0;
     for (int t = 0; t < u.T; ++t) {
@@ -354,7 +370,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == 2 && lane == 0) {
     // ============================================================ V producer
     // per tile and 64-key group: this CTA's two 128-dim value blocks
-    const uint32_t full0 = map_to_rank(bar(kBarVFull), 0);
+    const uint32_t full0 = map_to_rank(bar(kBarVFull), pbase);
     Ring rg;
     const int x = 128 * (int)rank;
     for (int t = 0; t < u.T; ++t) {
@@ -401,10 +417,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 4; ++k)
             mma_pair_ss(d, smem_desc_sw128(a0 + 32 * k, 16, 1024), smem_desc_sw128(b0 + 32 * k, 16, 1024), kIdescQK,
                         (ch | k) != 0);
-          if (rg.slot & 1) mma_commit_pair_mc(bar(kBarKEmpty + (rg.slot >> 1)), 0x3);
+          if (rg.slot & 1) mma_commit_pair_mc(bar(kBarKEmpty + (rg.slot >> 1)), pmask);
           if (++rg.slot == kKStages) { rg.slot = 0; rg.phase ^= 1u; }
         }
-        if (ok) mma_commit_pair_mc(bar(kBarSFull + sb), 0x3);
+        if (ok) mma_commit_pair_mc(bar(kBarSFull + sb), pmask);
       }
     } else {
       // P.V into the two 128-column output blocks
@@ -425,10 +441,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                           smem_desc_sw128(b0 + 2 * j * kBoxBytes + 2048 * k, kBoxBytes, 1024), kIdescPV,
                           (t > 0 || g > 0 || k > 0) ? 1u : 0u);
           }
-          mma_commit_pair_mc(bar(kBarVEmpty + rg.slot), 0x3);
+          mma_commit_pair_mc(bar(kBarVEmpty + rg.slot), pmask);
           if (++rg.slot == kVStages) { rg.slot = 0; rg.phase ^= 1u; }
         }
-        if (ok) mma_commit_pair_mc(bar(kBarOFull), 0x3);
+        if (ok) mma_commit_pair_mc(bar(kBarOFull), pmask);
       }
     }
   } else if (warp >= 4) {
@@ -447,8 +463,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t* mw = s_mask + rho * kMaxW;
     float* red = reinterpret_cast<float*>(smem + kOffRed);
     float* lred = reinterpret_cast<float*>(smem + kOffLred);
-    const uint32_t sempty0 = map_to_rank(bar(kBarSEmpty), 0);
-    const uint32_t pfull0 = map_to_rank(bar(kBarPFull), 0);
+    const uint32_t sempty0 = map_to_rank(bar(kBarSEmpty), pbase);
+    const uint32_t pfull0 = map_to_rank(bar(kBarPFull), pbase);
     unsigned char* pchunk = smem + kOffP + grp * kBoxBytes + rho * 128;
     const float sl2 = p.scale_log2;
     float m_used = -INFINITY, lsum = 0.0f;
@@ -585,14 +601,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t sw = (uint32_t)(rho & 7);
     const bool f32_out = p.out_dtype == DDT_F32;
     int* s_flag = reinterpret_cast<int*>(smem + kOffTmem + 4);
-    unsigned* cnt = multi ? p.counter + (((size_t)u.b * p.rowtiles + u.rt) * 2 + rank) * 2 : nullptr;
-    if (multi && threadIdx.x == 128) {
+    // both splits of these rows in this cluster: merge through distributed
+    // shared memory; otherwise through the workspace (merger elected below)
+    const bool xmerge = multi && p.csize == 4;
+    const uint32_t xpeer = crank ^ 2u;  // same rows, the other key split
+    if (xmerge) {
+      // arm the barrier the other split's bulk copy completes on, then tell
+      // that CTA that this CTA's staging is free (its MMAs are done)
+      if (threadIdx.x == 128 + 128 * (int)(crank >> 1))
+        mbar_arrive_expect_tx(bar(kBarXData), 8u * kBoxBytes + 64u * 8u);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_rank(bar(kBarXReady), xpeer));
+    }
+    unsigned* cnt = (multi && !xmerge) ? p.counter + (((size_t)u.b * p.rowtiles + u.rt) * 2 + rank) * 2 : nullptr;
+    if (multi && !xmerge && threadIdx.x == 128) {
       const bool last = atomicAdd(cnt, 1u) == (unsigned)(u.active - 1);
       if (last) cnt[0] = 0u;
       *s_flag = last ? 1 : 0;
     }
     named_bar_sync(1, 32 * kSoftmaxWarps);
-    const bool merger = multi && *s_flag != 0;
+    const bool merger = multi && !xmerge && *s_flag != 0;
     const float ltot = (lred[rho] + lred[64 + rho]) + (lred[128 + rho] + lred[192 + rho]);
     const bool real_row = ok && in_range && (rr / p.H) < u.n;
     const float m_own = real_row ? m_used : -INFINITY;
@@ -654,7 +682,92 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
     };
-    if (!merger) {
+    if (xmerge) {
+      // ---- merge with the other split's CTA of these rows (cluster rank
+      // crank ^ 2). This pair keeps output dims [256 kp, 256 kp + 256) (the
+      // TMEM block of the softmax threads with sub == kp); the other threads
+      // write their O -- the peer's dims -- into the peer's staging boxes, and
+      // one thread per row sends the row's (m, l).
+      const int kp = (int)(crank >> 1);
+      float* xml = reinterpret_cast<float*>(smem + kOffRed);            // the peer's (m, l) per row
+      float* xml_out = reinterpret_cast<float*>(smem + kOffRed + 512);  // this CTA's, sent to the peer
+      if (sub != kp) {
+        // stage the peer's dims of O (and the rows' (m, l)) locally, then one
+        // bulk copy into the peer's staging once the peer is ready
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(lane_addr + o_col + 32 * c, r);
+          tmem_wait_ld();
+          const int d0 = 256 * sub + 128 * eta + 32 * c;
+          unsigned char* row = smem + kOffStage32 + (d0 >> 5) * kBoxBytes + rho * 128;
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            *reinterpret_cast<uint4*>(row + (((uint32_t)i ^ sw) << 4)) =
+                make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+        }
+        if (eta == 0) {
+          xml_out[2 * rho] = m_own;
+          xml_out[2 * rho + 1] = ltot;
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(3, 128);
+        if (threadIdx.x == 128 + 128 * (1 - kp)) {
+          if (!mbar_wait(bar(kBarXReady), 0u, abort)) ok = false;
+          const uint32_t half = sbase + kOffStage32 + (uint32_t)(8 * (1 - kp) * kBoxBytes);
+          const uint32_t xbar = map_to_rank(bar(kBarXData), xpeer);
+          bulk_copy_to_cluster(map_to_rank(half, xpeer), half, 8u * kBoxBytes, xbar);
+          bulk_copy_to_cluster(map_to_rank(sbase + kOffRed, xpeer), sbase + kOffRed + 512u, 64u * 8u, xbar);
+        }
+      } else {
+        const int first_keeper = 128 + 128 * kp;
+        if (!mbar_wait_own(bar(kBarXData), 0u, abort)) ok = false;
+        const float mp = xml[2 * rho], lpeer = xml[2 * rho + 1];
+        const float M = fmaxf(m_own, mp);
+        const float w_own = m_own == -INFINITY ? 0.0f : exp2f(m_own - M);
+        const float w_p = mp == -INFINITY ? 0.0f : exp2f(mp - M);
+        const float den = w_own * ltot + w_p * lpeer;
+        const float dinv = den > 0.0f ? 1.0f / den : 0.0f;
+        const bool keep = real_row && ok;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          const int d0 = 256 * sub + 128 * eta + 32 * c;
+          uint32_t r[32];
+          tmem_ld32(lane_addr + o_col + 32 * c, r);
+          tmem_wait_ld();
+          const unsigned char* row = smem + kOffStage32 + (d0 >> 5) * kBoxBytes + rho * 128;
+          float f[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 v = *reinterpret_cast<const float4*>(row + (((uint32_t)i ^ sw) << 4));
+            f[4 * i] = keep ? fmaf(w_p, v.x, __uint_as_float(r[4 * i]) * w_own) * dinv : 0.0f;
+            f[4 * i + 1] = keep ? fmaf(w_p, v.y, __uint_as_float(r[4 * i + 1]) * w_own) * dinv : 0.0f;
+            f[4 * i + 2] = keep ? fmaf(w_p, v.z, __uint_as_float(r[4 * i + 2]) * w_own) * dinv : 0.0f;
+            f[4 * i + 3] = keep ? fmaf(w_p, v.w, __uint_as_float(r[4 * i + 3]) * w_own) * dinv : 0.0f;
+          }
+          stage_chunk(d0, f, f32_out);  // fp32: in place of the values just read
+          if (!f32_out && !(c & 1)) continue;
+          fence_proxy_async_smem();
+          named_bar_sync(2, 128);
+          if (threadIdx.x == first_keeper) {
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+              if (f32_out) {
+                const int j = 8 * kp + 4 * e2 + c;
+                tma_store_3d(&tm_out, sbase + kOffStage32 + j * kBoxBytes, 32 * j, row0, u.b);
+              } else {
+                const int j = 4 * kp + 2 * e2 + (c >> 1);
+                tma_store_3d(&tm_out, sbase + kOffStage16 + j * kBoxBytes, 64 * j, row0, u.b);
+              }
+            }
+            bulk_commit();
+          }
+        }
+        if (eta == 0 && in_range && p.lse)
+          p.lse[grow] = (keep && den > 0.0f) ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
+        if (threadIdx.x == first_keeper) bulk_wait_read_all();
+      }
+    } else if (!merger) {
       // the final output (one split) or this split's partial
       const int kind = multi ? 0 : (f32_out ? 1 : 2);
       const float inv = !real_row ? 0.0f : ((!multi && ltot > 0.0f) ? 1.0f / ltot : 1.0f);
@@ -932,7 +1045,31 @@ int launch_attn_tc(const AttnParams& a, int64_t kv_rows, int max_cache_len, void
       !make_out_map(&tpart, p.part_o, true, 4, (uint64_t)a.N * a.H, (uint64_t)a.B, (uint64_t)p.splits))
     return DDT_ERR_CUDA;
   const long long units = (long long)a.B * p.rowtiles * p.splits;
-  return launch_pdl(attn_tc_kernel, (unsigned)(2 * units), kThreads, kSmemAlloc, stream, tq, tkv, tout, tpart, p);
+  // two key splits: both in one cluster of 4 (merged through distributed
+  // shared memory); otherwise clusters of 2 (one CTA pair each)
+  auto launch = [&](int csize) -> cudaError_t {
+    p.csize = csize;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * units));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)csize;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, attn_tc_kernel, tq, tkv, tout, tpart, p);
+  };
+  if (p.splits == 2) {
+    if (launch(4) == cudaSuccess) return DDT_OK;
+    (void)cudaGetLastError();  // clusters of 4 not schedulable here: pairs + workspace merge
+  }
+  return launch(2) == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
 }
 
 }  // namespace ddt

@@ -149,3 +149,32 @@ def test_attn_bf16_status_word_stays_zero():
                         t_from(t["n_nodes"], DEV), 512, 64, s.scale, 4096, workspace=ws)
     torch.cuda.synchronize()
     assert lib.verify_attn_status(ws) == lib.DDT_OK
+
+
+def test_attn_bf16_two_splits_in_one_cluster():
+    """Two key splits put both splits of a row tile in one 4-CTA cluster and
+    merge them through distributed shared memory. Request 0 has a single key
+    tile (its second split is idle) and pad row tiles (n_nodes cut to 20);
+    request 1 uses both splits."""
+    s = synth.custom(B=2, D=4, K=4, N=32, H=64, d_l=512, d_r=64, V=64, L=(0, 1500), dtype="bf16", kv_scale=0.1,
+                     scale=1.0 / np.sqrt(192.0), seed=11)
+    x = synth.make_step(s)
+    t = _tree(x, s)
+    t["n_nodes"][0] = 20
+    maxL = 2000
+    d = step_to_device(x, DEV)
+    mask = t_from(t["mask"].view(np.int32), DEV)
+    nn = t_from(t["n_nodes"], DEV)
+    ws = torch.zeros(lib.verify_attn_workspace_size(s.B, s.N, s.H, 512, 64, maxL, torch.bfloat16), dtype=torch.uint8,
+                     device=DEV)
+    assert ws.numel() > 256  # the launch splits the keys
+    for _ in range(2):
+        out, lse = lib.verify_attn(d["q"], d["kv"], d["cache_off"], d["cache_len"], mask, nn, 512, 64, s.scale, maxL,
+                                   workspace=ws)
+    torch.cuda.synchronize()
+    assert lib.verify_attn_status(ws) == 0
+    ref, rl = oracle.verify_attn(x.q, x.kv, x.cache_off, x.cache_len, t["mask"], t["n_nodes"], s.H, 512, 64, s.scale,
+                                 "bf16")
+    got = widen_out(out)
+    _check(got, lse.cpu().numpy().astype(np.float64), ref, rl, True)
+    assert np.all(got[0, 20:] == 0) and np.all(np.isneginf(lse.cpu().numpy()[0, 20:]))
