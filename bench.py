@@ -42,6 +42,23 @@ L2_BYTES = 126 * 1024 * 1024
 # ---------------------------------------------------------------------------
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest value of x over the ranks of the default process group (x
+    itself without one): a multi-GPU time is the slowest replica's."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(nodes_per_step: int, steps: int, world: int, elapsed_ms: float) -> float:
+    """Whole-job tree nodes/s of `world` replicas that each ran `steps` steps of
+    `nodes_per_step` nodes, timed by the slowest replica."""
+    return nodes_per_step * world * steps / (elapsed_ms / 1e3)
+
+
 def profiled_traffic(shape: synth.Shape):
     """DRAM bytes (read + write) of one verify-attention launch from the ncu
     capture summarised in profiles/attn_tc_<workload>.md, or None when there is
@@ -344,11 +361,8 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
     build_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     accept_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    el = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(el, op=dist.ReduceOp.MAX)
-    elapsed_ms = float(el.item())
-    value = n_nodes_total * world * args.steps / (elapsed_ms / 1e3)
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
+    value = replica_throughput(n_nodes_total, args.steps, world, elapsed_ms)
 
     # ---- end to end through the public API with host buffers -------------------------
     e2e = run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_acc, out, lse, off, cap, maxL,
@@ -472,15 +486,12 @@ def run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_a
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = max_over_ranks(e0.elapsed_time(e1), dev)
     nodes = int(tree["n_nodes"].sum().item())
-    return {"value": nodes * world * steps / (float(t.item()) / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+    return {"value": replica_throughput(nodes, steps, world, ms), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps,
             "copies": "on the compute stream" if args.e2e_serial else "next step's copies overlap this step's kernels",
-            "h2d_gbs": h2d * steps / (float(t.item()) / 1e3) / 1e9}
+            "h2d_gbs": h2d * steps / (ms / 1e3) / 1e9}
 
 
 def cpu_baseline(args, shape, x, logits_h, t_host):
