@@ -175,6 +175,15 @@ __device__ __forceinline__ UnitInfo unit_info(const TcParams& p, int unit) {
   return u;
 }
 
+// 2^x with the hardware approximation, subnormal results flushed to zero: the
+// probabilities are rounded to bf16 next, and a probability below 2^-126 of
+// the row maximum cannot change a bf16 P.V product or the row sum.
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // 64-key groups of the unit's tile t that hold at least one key of the unit
 // (the last tile of a request can be ragged: P.V skips its empty groups)
 __device__ __forceinline__ int live_groups(const UnitInfo& u, int t) {
@@ -540,8 +549,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       float ps0 = 0.0f, ps1 = 0.0f;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float p0 = exp2f(fmaf(s[2 * i], sl2, -mref));
-        const float p1 = exp2f(fmaf(s[2 * i + 1], sl2, -mref));
+        const float p0 = ex2_ftz(fmaf(s[2 * i], sl2, -mref));
+        const float p1 = ex2_ftz(fmaf(s[2 * i + 1], sl2, -mref));
         ps0 += p0;
         ps1 += p1;
         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
