@@ -95,8 +95,8 @@ constexpr int kBarPFull = kBarSEmpty + 2;             // leader: P written (soft
 constexpr int kBarOFull = kBarPFull + 1;              // each CTA: PV finished
 constexpr int kBarEpi = kBarOFull + 1;                // [4] each CTA: epilogue tile loads, one per 32-dim chunk
 constexpr int kBarXReady = kBarEpi + 4;               // each CTA: the other split's CTA of these rows is done with its MMAs
-constexpr int kBarXData = kBarXReady + 1;             // each CTA: the other split's partial has landed here (bulk copy)
-constexpr int kNumBars = kBarXData + 1;
+constexpr int kBarXData = kBarXReady + 1;             // [4] each CTA: the other split's partial, one per 32-dim chunk (bulk copies)
+constexpr int kNumBars = kBarXData + 4;
 constexpr int kOffRed = kOffMisc + 256;                 // float [2 parity][4 groups][64]
 constexpr int kOffLred = kOffRed + 2 * 4 * 64 * 4;      // float [4][64]
 constexpr int kOffMask = kOffLred + 4 * 64 * 4;         // uint32 [64][kMaxW]
@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(kBarOFull), 1);
     for (int c = 0; c < 4; ++c) mbar_init(bar(kBarEpi + c), 1);
     mbar_init(bar(kBarXReady), kSoftmaxWarps);
-    mbar_init(bar(kBarXData), 1);
+    for (int c = 0; c < 4; ++c) mbar_init(bar(kBarXData + c), 1);
     fence_mbar_init_cluster();
   }
   if (warp == 0 && lane == 0) {
@@ -618,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // arm the barrier the other split's bulk copy completes on, then tell
       // that CTA that this CTA's staging is free (its MMAs are done)
       if (threadIdx.x == 128 + 128 * (int)(crank >> 1))
-        mbar_arrive_expect_tx(bar(kBarXData), 8u * kBoxBytes + 64u * 8u);
+        for (int c = 0; c < 4; ++c) mbar_arrive_expect_tx(bar(kBarXData + c), 2u * kBoxBytes + (c == 0 ? 64u * 8u : 0u));
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_to_rank(bar(kBarXReady), xpeer));
     }
@@ -701,8 +701,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* xml = reinterpret_cast<float*>(smem + kOffRed);            // the peer's (m, l) per row
       float* xml_out = reinterpret_cast<float*>(smem + kOffRed + 512);  // this CTA's, sent to the peer
       if (sub != kp) {
-        // stage the peer's dims of O (and the rows' (m, l)) locally, then one
-        // bulk copy into the peer's staging once the peer is ready
+        // stage the peer's dims of O chunk by chunk (and the rows' (m, l))
+        // locally; one thread ships each chunk's two boxes by bulk copy into
+        // the peer's staging once the peer is ready
+        if (eta == 0) {
+          xml_out[2 * rho] = m_own;
+          xml_out[2 * rho + 1] = ltot;
+        }
+        const int sender0 = 128 + 128 * (1 - kp);
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
@@ -714,23 +720,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 8; ++i)
             *reinterpret_cast<uint4*>(row + (((uint32_t)i ^ sw) << 4)) =
                 make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
-        }
-        if (eta == 0) {
-          xml_out[2 * rho] = m_own;
-          xml_out[2 * rho + 1] = ltot;
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(3, 128);
-        if (threadIdx.x == 128 + 128 * (1 - kp)) {
-          if (!mbar_wait(bar(kBarXReady), 0u, abort)) ok = false;
-          const uint32_t half = sbase + kOffStage32 + (uint32_t)(8 * (1 - kp) * kBoxBytes);
-          const uint32_t xbar = map_to_rank(bar(kBarXData), xpeer);
-          bulk_copy_to_cluster(map_to_rank(half, xpeer), half, 8u * kBoxBytes, xbar);
-          bulk_copy_to_cluster(map_to_rank(sbase + kOffRed, xpeer), sbase + kOffRed + 512u, 64u * 8u, xbar);
+          fence_proxy_async_smem();
+          named_bar_sync(3, 128);
+          if (threadIdx.x == sender0) {
+            if (c == 0 && !mbar_wait(bar(kBarXReady), 0u, abort)) ok = false;
+            const uint32_t xbar = map_to_rank(bar(kBarXData + c), xpeer);
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+              const uint32_t box = sbase + kOffStage32 + (uint32_t)((8 * sub + 4 * e2 + c) * kBoxBytes);
+              bulk_copy_to_cluster(map_to_rank(box, xpeer), box, kBoxBytes, xbar);
+            }
+            if (c == 0)
+              bulk_copy_to_cluster(map_to_rank(sbase + kOffRed, xpeer), sbase + kOffRed + 512u, 64u * 8u, xbar);
+          }
         }
       } else {
         const int first_keeper = 128 + 128 * kp;
-        if (!mbar_wait_own(bar(kBarXData), 0u, abort)) ok = false;
+        if (!mbar_wait_own(bar(kBarXData), 0u, abort)) ok = false;  // chunk 0 and the rows' (m, l)
         const float mp = xml[2 * rho], lpeer = xml[2 * rho + 1];
         const float M = fmaxf(m_own, mp);
         const float w_own = m_own == -INFINITY ? 0.0f : exp2f(m_own - M);
@@ -743,6 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int d0 = 256 * sub + 128 * eta + 32 * c;
           uint32_t r[32];
           tmem_ld32(lane_addr + o_col + 32 * c, r);
+          if (c > 0 && !mbar_wait_own(bar(kBarXData + c), 0u, abort)) ok = false;
           tmem_wait_ld();
           const unsigned char* row = smem + kOffStage32 + (d0 >> 5) * kBoxBytes + rho * 128;
           float f[32];
