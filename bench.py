@@ -42,6 +42,13 @@ L2_BYTES = 126 * 1024 * 1024
 # ---------------------------------------------------------------------------
 
 
+# (B, N, L) points of the Kimi-shaped sweep: step time against context length
+# at one and at 16 requests, and the tree budget at one request
+SWEEP_POINTS = [(1, 64, 512), (1, 64, 4096), (1, 64, 16384), (1, 64, 65536),
+                (16, 64, 512), (16, 64, 4096), (16, 64, 16384), (4, 64, 65536),
+                (1, 16, 4096), (1, 256, 4096), (64, 16, 4096)]
+
+
 def max_over_ranks(x: float, device) -> float:
     """The largest value of x over the ranks of the default process group (x
     itself without one): a multi-GPU time is the slowest replica's."""
@@ -365,8 +372,8 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
     value = replica_throughput(n_nodes_total, args.steps, world, elapsed_ms)
 
     # ---- end to end through the public API with host buffers -------------------------
-    e2e = run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_acc, out, lse, off, cap, maxL,
-                  world)
+    e2e = None if args.sweep else run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_acc, out,
+                                          lse, off, cap, maxL, world)
 
     if rank != 0:
         return
@@ -394,7 +401,10 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
         "clocks": clocks,
         "timed_loop": "cuda-graph replays of the step" if graphs is not None else "plain library calls",
     }
-    if args.cpu_baseline and world == 1:
+    if args.sweep:
+        line["sweep_point"] = True
+        line["attn_split_keys"] = lib.verify_attn_workspace_size(B, N, H, shape.d_l, shape.d_r, maxL, tdt) > 256
+    elif args.cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(args, shape, x, logits_h, t_host)
     print(json.dumps(line), flush=True)
 
@@ -515,6 +525,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--e2e-serial", action="store_true",
                     help="end-to-end leg: copy each step's inputs on the compute stream (no overlap)")
+    ap.add_argument("--sweep", default=None,
+                    help="context/budget sweep on Kimi shapes: 'default' or a comma list of B:N:L points; one "
+                         "JSON line per point (no end-to-end leg, no CPU baseline)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time plain library calls instead of CUDA-graph replays of the step")
     args = ap.parse_args()
@@ -534,7 +547,14 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     try:
-        run_ours(args, shape, rank, world, local_rank)
+        if args.sweep:
+            pts = SWEEP_POINTS if args.sweep == "default" else [tuple(int(v) for v in p.split(":"))
+                                                                 for p in args.sweep.split(",")]
+            for (b, n, l) in pts:
+                run_ours(args, synth.kimi_sweep(b, n, l), rank, world, local_rank)
+                torch.cuda.empty_cache()
+        else:
+            run_ours(args, shape, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()
