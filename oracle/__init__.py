@@ -10,6 +10,7 @@ from .ddt_oracle import (  # noqa: F401
     accept_compact,
     accept_walk,
     build_tree,
+    drafter_topk,
     row_argmax,
     verify_attn,
     visible_keys,

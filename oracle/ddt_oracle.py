@@ -302,3 +302,43 @@ def accept_compact(logits, logits_dtype, node_tok, parent, n_nodes, kv, cache_of
         res["cache_len"][b] = L_b + a + 1
     res["am"] = am
     return res
+
+
+# ---------------------------------------------------------------------------
+# drafter proposals: per-depth log-softmax + top-k over the vocabulary
+# ---------------------------------------------------------------------------
+
+
+def drafter_topk(logits, K):
+    """Per-row drafter proposals, the input contract of the tree build.
+
+    Source: capstone page, "The Oracle Drafter" (the drafter hands the tree
+    builder, for every depth, log-probabilities and token ids of its best
+    candidates, sorted best first); AR page, "The Broader Context" (the
+    draft tree is built from the drafter's per-depth top-k).
+
+    logits: [R, V] float (bf16 already widened exactly); K <= V.
+    Returns (logp [R, K] float32, tok [R, K] int32, status [R] int32):
+      tok[r] = the K indices of the largest logits, largest first;
+               READING: equal values are ordered by lower index first.
+      logp[r][k] = logits[r][tok[r][k]] - logsumexp(logits[r]), computed in
+               float64 and rounded to float32 once.
+      status OK, or ERR_INPUT for a row with a non-finite logit (READING:
+      that row's outputs are tok -1, logp -inf).
+    """
+    x = np.asarray(logits, dtype=np.float64)
+    R, V = x.shape
+    logp = np.full((R, K), -np.inf, np.float32)
+    tok = np.full((R, K), -1, np.int32)
+    status = np.full(R, OK, np.int32)
+    for r in range(R):
+        z = x[r]
+        if not np.all(np.isfinite(z)):
+            status[r] = ERR_INPUT
+            continue
+        m = z.max()
+        lse = m + math.log(np.exp(z - m).sum())
+        order = np.lexsort((np.arange(V), -z))[:K]  # value descending, then index ascending
+        tok[r] = order.astype(np.int32)
+        logp[r] = (z[order] - lse).astype(np.float32)
+    return logp, tok, status
