@@ -365,6 +365,7 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
     for k in range(n_stage):
         step(sets[k % n_sets], evs[k])
     torch.cuda.synchronize()
+    dr = measure_drafter(args, shape, lib, dev, tdt)
     build_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     accept_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
@@ -394,6 +395,7 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
         "stages_ms": {"build_tree": build_ms, "verify_attn": attn_ms, "accept_compact": accept_ms},
         "accept_hbm": {"achieved_gbs": acc_bytes / (accept_ms / 1e3) / 1e9, "peak_gbs": pk["hbm_gbs"],
                        "frac": acc_bytes / (accept_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
+        "drafter_topk": dict(dr, frac=dr["gbs"] / pk["hbm_gbs"], peak_gbs=pk["hbm_gbs"]),
         "nodes_per_step": n_nodes_total,
         "attn_gflop_per_step": flops / 1e9,
         "gpu_launches": launches_per_step * args.steps,
@@ -417,6 +419,42 @@ def attn_launches(shape: synth.Shape) -> int:
 def _tdtype(shape):
     import torch
     return torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+
+
+def measure_drafter(args, shape, lib, dev, tdt):
+    """ddt_drafter_topk on the workload's B x D rows of V drafter logits (the
+    build's inputs), timed alone over rotating sets larger than 2 x L2 (random
+    device-side logits; its parity is covered by the tests)."""
+    import torch
+    R, V, K = shape.B * shape.D, shape.V, shape.K
+    row_bytes = R * V * (2 if tdt == torch.bfloat16 else 4)
+    n = max(2, math.ceil(2 * L2_BYTES / row_bytes))
+    g = torch.Generator(device=dev)
+    g.manual_seed(shape.seed)
+    z = (torch.randn(n, R, V, device=dev, generator=g) * shape.drafter_sigma).to(tdt)
+    views = [z[i] for i in range(n)]
+    out = lib.drafter_topk(views[0], K)
+    for i in range(3):
+        lib.drafter_topk(views[i % n], K, out=out)
+    torch.cuda.synchronize()
+    # one graph launches the kernel once per set, so Python's per-call cost
+    # stays out of the kernel time
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            lib.drafter_topk(views[i], K, out=out, stream=torch.cuda.current_stream(dev))
+    g.replay()
+    torch.cuda.synchronize()
+    reps = max(2, min(50, math.ceil(400 / n)))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) / (reps * n) * 1e3
+    del g, views, z
+    return {"us": us, "gbs": row_bytes / (us / 1e6) / 1e9, "rows": R, "V": V, "K": K}
 
 
 def run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_acc, out, lse, off, cap, maxL, world):

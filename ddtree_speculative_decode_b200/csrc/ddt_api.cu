@@ -34,6 +34,23 @@ const char* ddt_status_string(int status) {
 
 int ddt_version(void) { return 100; }
 
+int ddt_drafter_topk(const void* logits, int logits_dtype, int V, int R, int K, float* logp, int32_t* tok,
+                     int32_t* dev_status, cudaStream_t stream) {
+  if (!logits || !logp || !tok) return DDT_ERR_INVALID_ARG;
+  if (R < 1 || V < 1 || K < 1 || K > 32 || K > V) return DDT_ERR_INVALID_ARG;
+  if (logits_dtype != DDT_F32 && logits_dtype != DDT_BF16) return DDT_ERR_INVALID_ARG;
+  ddt::DrafterParams p{};
+  p.logits = logits;
+  p.logits_dtype = logits_dtype;
+  p.V = V;
+  p.R = R;
+  p.K = K;
+  p.logp = logp;
+  p.tok = tok;
+  p.dev_status = dev_status;
+  return ddt::launch_drafter_topk(p, stream);
+}
+
 int ddt_build_tree(const float* logp, const int32_t* tok, const int32_t* root_tok,
                    const int32_t* cache_len, int B, int D, int K, int N, int32_t* node_tok,
                    int32_t* parent, int32_t* depth, int32_t* pos, float* score, uint32_t* mask,

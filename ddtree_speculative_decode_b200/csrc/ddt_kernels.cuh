@@ -55,6 +55,18 @@ int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream);
 size_t accept_noalloc_scratch_bytes();
 int launch_accept_compact_noalloc(AcceptParams p, cudaStream_t stream);
 
+// ---- drafter proposals --------------------------------------------------------
+struct DrafterParams {
+  const void* logits;   // [R][V]
+  int logits_dtype;
+  int V, R, K;
+  float* logp;          // [R][K]
+  int32_t* tok;         // [R][K]
+  int32_t* dev_status;  // [R], nullable
+  int vec;              // rows are 16-byte aligned
+};
+int launch_drafter_topk(DrafterParams p, cudaStream_t stream);
+
 // ---- verify attention -------------------------------------------------------
 struct AttnParams {
   const void* q;

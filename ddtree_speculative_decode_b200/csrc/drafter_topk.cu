@@ -1,0 +1,222 @@
+// Drafter proposals: per row (one request's depth), the log-softmax of the
+// drafter's logits over the vocabulary and its K best tokens, best first --
+// the input the best-first tree build consumes.
+//
+// What it computes is fixed in ddt.h (ddt_drafter_topk)
+// ("ddtree_speculative_decode_test_capstone", section "The Oracle Drafter":
+// per-depth log-probabilities and token ids of the drafter's candidates,
+// sorted best first; "autoregressive_test_driver_kdtree_engine", section "The
+// Broader Context": the draft tree is built from the drafter's per-depth
+// top-k).
+//
+// One CTA per row streams the row once with 16-byte loads, eight in flight
+// per thread. Each thread keeps
+// a running (max, sum of exponentials) for the log-sum-exp and a sorted list
+// of its K best packed keys (order-preserving value bits << 32 | ~index, so a
+// larger key is a larger value or, on equal values, a lower index); a new
+// value costs one compare unless it beats the thread's K-th best. Warps then
+// merge their lists by K rounds of a warp-wide maximum, and one warp merges
+// the warps' lists the same way.
+#include "ddt_kernels.cuh"
+
+namespace ddt {
+
+constexpr int kDrThreads = 512;
+constexpr int kDrWarps = kDrThreads / 32;
+
+__device__ __forceinline__ unsigned long long drafter_key(float v, int idx) {
+  return (static_cast<unsigned long long>(float_order_key(v)) << 32) |
+         static_cast<unsigned long long>(~static_cast<uint32_t>(idx));
+}
+
+__device__ __forceinline__ float key_value(unsigned long long k) {
+  const uint32_t u = static_cast<uint32_t>(k >> 32);
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// 2^x by the hardware approximation (relative error about 2^-22; subnormal
+// results flushed to zero)
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// log-sum-exp state in base 2: m = running max of x log2(e), s = sum of
+// 2^(x log2(e) - m)
+__device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2) {
+  const float M = fmaxf(m, m2);
+  if (M == -INFINITY) return;
+  s = (m == -INFINITY ? 0.0f : s * ex2_ftz(m - M)) + (m2 == -INFINITY ? 0.0f : s2 * ex2_ftz(m2 - M));
+  m = M;
+}
+
+template <int KM>
+__device__ __forceinline__ void topk_insert(unsigned long long (&k)[KM], unsigned long long key) {
+  if (key <= k[KM - 1]) return;
+  k[KM - 1] = key;
+#pragma unroll
+  for (int j = KM - 1; j > 0; --j) {
+    const unsigned long long a = k[j - 1], b = k[j];
+    const bool sw = b > a;
+    k[j - 1] = sw ? b : a;
+    k[j] = sw ? a : b;
+  }
+}
+
+// The warp's K best keys over the lanes' sorted lists (each consumed from its
+// head); round j's key ends up in lane j. Lists are destroyed.
+template <int KM>
+__device__ __forceinline__ unsigned long long warp_topk(unsigned long long (&k)[KM], int K, int lane) {
+  unsigned long long mine = 0ull;
+  for (int j = 0; j < K; ++j) {
+    unsigned long long best = k[0];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(DDT_FULL_MASK, best, o);
+      best = other > best ? other : best;
+    }
+    if (lane == j) mine = best;
+    const bool pop = best != 0ull && k[0] == best;  // keys are unique: one lane pops
+#pragma unroll
+    for (int i = 0; i < KM - 1; ++i) k[i] = pop ? k[i + 1] : k[i];
+    if (pop) k[KM - 1] = 0ull;
+  }
+  return mine;
+}
+
+template <int KM, bool kBF16>
+__global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int r = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int V = p.V;
+  const size_t esz = kBF16 ? 2 : 4;
+  const unsigned char* row = static_cast<const unsigned char*>(p.logits) + (size_t)r * V * esz;
+
+  unsigned long long k[KM];
+#pragma unroll
+  for (int i = 0; i < KM; ++i) k[i] = 0ull;  // 0 = empty; every finite value's key is larger
+  float m = -INFINITY, s = 0.0f;
+  bool bad = false;
+  // a batch of values: one running-max update, a batch sum of exponentials,
+  // then the top-k candidates (one compare per value unless it beats the K-th)
+  auto batch = [&](const float* x, int n, int idx0) {
+    float y[8];
+    float bm = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (t < n) {
+        bad |= !(fabsf(x[t]) <= 3.402823466e38f);
+        y[t] = x[t] * kLog2e;
+        bm = fmaxf(bm, y[t]);
+      }
+    }
+    if (bm > m) {
+      s *= ex2_ftz(m - bm);
+      m = bm;
+    }
+    float bs = 0.0f;
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      if (t < n) bs += ex2_ftz(y[t] - m);
+    s += bs;
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      if (t < n) topk_insert<KM>(k, drafter_key(x[t], idx0 + t));
+  };
+  if (p.vec) {  // 16-byte aligned rows: 8 bf16 or 4 f32 per load
+    constexpr int kPer = kBF16 ? 8 : 4;
+    const int nvec = V / kPer;
+    const uint4* src = reinterpret_cast<const uint4*>(row);
+    // eight 16-byte loads in flight per thread (64 KB per CTA) before any is used
+    constexpr int kU = 8;
+    for (int e0 = tid; e0 < nvec; e0 += kU * kDrThreads) {
+      uint4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int e = e0 + u * kDrThreads;
+        v[u] = e < nvec ? __ldcs(src + e) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int e = e0 + u * kDrThreads;
+        if (e >= nvec) break;
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        float x[8];
+#pragma unroll
+        for (int t = 0; t < kPer; ++t)
+          x[t] = kBF16 ? __uint_as_float((t & 1) ? (w[t >> 1] & 0xffff0000u) : (w[t >> 1] << 16))
+                       : __uint_as_float(w[t]);
+        batch(x, kPer, e * kPer);
+      }
+    }
+  } else {
+    for (int i = tid; i < V; i += kDrThreads) {
+      float x[8];
+      x[0] = kBF16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(row)[i])
+                   : reinterpret_cast<const float*>(row)[i];
+      batch(x, 1, i);
+    }
+  }
+  // ---- combine: log-sum-exp and non-finite flag
+  __shared__ float s_m[kDrWarps], s_s[kDrWarps];
+  __shared__ int s_bad;
+  __shared__ unsigned long long s_keys[kDrWarps][KM];
+  if (tid == 0) s_bad = 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(DDT_FULL_MASK, m, o), s2 = __shfl_xor_sync(DDT_FULL_MASK, s, o);
+    lse_merge(m, s, m2, s2);
+  }
+  const bool wbad = __any_sync(DDT_FULL_MASK, bad);
+  // ---- combine: each warp's K best
+  const unsigned long long wk = warp_topk<KM>(k, p.K, lane);
+  __syncthreads();
+  if (lane == 0) {
+    s_m[warp] = m;
+    s_s[warp] = s;
+    if (wbad) s_bad = 1;
+  }
+  if (lane < p.K) s_keys[warp][lane] = wk;
+  __syncthreads();
+  if (warp != 0) return;
+  // warp 0: the row's K best over the warps' lists (lane w < 16 holds warp w's)
+  unsigned long long kk[KM];
+#pragma unroll
+  for (int i = 0; i < KM; ++i) kk[i] = (lane < kDrWarps && i < p.K) ? s_keys[lane][i] : 0ull;
+  const unsigned long long best = warp_topk<KM>(kk, p.K, lane);
+  float M = lane < kDrWarps ? s_m[lane] : -INFINITY, S = lane < kDrWarps ? s_s[lane] : 0.0f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(DDT_FULL_MASK, M, o), s2 = __shfl_xor_sync(DDT_FULL_MASK, S, o);
+    lse_merge(M, S, m2, s2);
+  }
+  const bool row_bad = s_bad != 0;
+  if (lane < p.K) {
+    const float lse = (M + log2f(S)) * 0.6931471805599453f;
+    p.logp[(size_t)r * p.K + lane] = row_bad ? -INFINITY : key_value(best) - lse;
+    p.tok[(size_t)r * p.K + lane] = row_bad ? -1 : static_cast<int32_t>(~static_cast<uint32_t>(best & 0xffffffffull));
+  }
+  if (lane == 0 && p.dev_status) p.dev_status[r] = row_bad ? DDT_ERR_INPUT : DDT_OK;
+}
+
+template <int KM>
+static int launch_dr(const DrafterParams& p, cudaStream_t stream) {
+  if (p.logits_dtype == DDT_BF16)
+    return launch_pdl(drafter_topk_kernel<KM, true>, (unsigned)p.R, kDrThreads, 0, stream, p);
+  return launch_pdl(drafter_topk_kernel<KM, false>, (unsigned)p.R, kDrThreads, 0, stream, p);
+}
+
+int launch_drafter_topk(DrafterParams p, cudaStream_t stream) {
+  const size_t esz = p.logits_dtype == DDT_BF16 ? 2 : 4;
+  p.vec = (reinterpret_cast<uintptr_t>(p.logits) % 16 == 0) && (((size_t)p.V * esz) % 16 == 0);
+  if (p.K <= 8) return launch_dr<8>(p, stream);
+  if (p.K <= 16) return launch_dr<16>(p, stream);
+  return launch_dr<32>(p, stream);
+}
+
+}  // namespace ddt

@@ -29,6 +29,7 @@ EXPORTS = (
     "ddt_accept_compact_workspace_size",
     "ddt_accept_compact",
     "ddt_accept_compact_noalloc",
+    "ddt_drafter_topk",
 )
 
 _lib = None
@@ -70,6 +71,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.ddt_accept_compact_noalloc.restype = i32
     lib.ddt_accept_compact_noalloc.argtypes = [vp, i32, i32, vp, vp, vp, i32, i32, vp, i32, i32, i32, i64, vp, vp,
                                                vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.ddt_drafter_topk.restype = i32
+    lib.ddt_drafter_topk.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
     if path is None:
         _lib = lib
     return lib
@@ -127,6 +130,25 @@ def _raise(fn: str, st: int):
 # ---------------------------------------------------------------------------
 # the three calls
 # ---------------------------------------------------------------------------
+
+
+def drafter_topk(logits: torch.Tensor, K: int, out: Optional[dict] = None, stream=None) -> dict:
+    """ddt_drafter_topk. logits [..., V] f32 / bf16 (e.g. [B, D, V]); returns
+    logp [..., K] f32, tok [..., K] i32 (build_tree's inputs) and status [...]."""
+    _check(logits, "logits", (torch.float32, torch.bfloat16))
+    lead, V = tuple(logits.shape[:-1]), logits.shape[-1]
+    R = 1
+    for d in lead:
+        R *= d
+    dev = logits.device
+    if out is None:
+        out = {"logp": torch.empty(*lead, K, dtype=torch.float32, device=dev),
+               "tok": torch.empty(*lead, K, dtype=torch.int32, device=dev),
+               "status": torch.empty(*lead, dtype=torch.int32, device=dev)}
+    st = load().ddt_drafter_topk(_ptr(logits), _dt(logits), V, R, K, _ptr(out["logp"]), _ptr(out["tok"]),
+                                 _ptr(out["status"]), _stream(stream))
+    _raise("ddt_drafter_topk", st)
+    return out
 
 
 def build_tree(logp: torch.Tensor, tok: torch.Tensor, root_tok: torch.Tensor, cache_len: torch.Tensor, N: int,

@@ -2,7 +2,9 @@
  * ddt.h -- C ABI of libddt.so: one DDTree speculative-decoding tree-verify
  * step on an NVIDIA B200 (sm_100a).
  *
- * The step has three calls, issued in this order on one CUDA stream:
+ * The step has three calls, issued in this order on one CUDA stream (a
+ * fourth, ddt_drafter_topk, can produce the build's inputs from the
+ * drafter's logits):
  *
  *   ddt_build_tree      best-first draft tree from the drafter's per-depth
  *                       top-k log-probs ("autoregressive_test_driver_kdtree_
@@ -79,6 +81,33 @@ DDT_API const char* ddt_status_string(int status);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 DDT_API int ddt_version(void);
+
+/*
+ * ddt_drafter_topk -- the drafter's per-depth proposals from its logits: for
+ * every row (one request's depth), the log-softmax over the vocabulary and
+ * the K best tokens, best first. Its outputs are ddt_build_tree's logp / tok
+ * inputs (rows = B * D, row-major [B][D]).
+ *
+ * Passage: capstone page, "The Oracle Drafter" (the drafter hands the tree
+ * builder per-depth log-probabilities and token ids of its candidates, sorted
+ * best first); first page, "The Broader Context" (the draft tree is built
+ * from the drafter's per-depth top-k). The pages fix no formula: the plainest
+ * reading is used.
+ *
+ * Definition: tok[r][k] = the index of the k-th largest logits[r][v] (equal
+ *   values: the lower index first; bf16 widened exactly to float32);
+ *   logp[r][k] = logits[r][tok[r][k]] - logsumexp_v(logits[r][v]), float32
+ *   arithmetic (the log-sum-exp is a float32 running sum of 2^(x log2 e - max)).
+ * Inputs (device): logits [R][V] logits_dtype (F32 or BF16), finite.
+ * Outputs (device): logp [R][K] float32, tok [R][K] int32; dev_status [R]
+ *   (nullable): DDT_OK, or DDT_ERR_INPUT for a row holding a non-finite
+ *   logit (that row's tok = -1, logp = -inf).
+ * Sizes: R >= 1, V >= 1, 1 <= K <= min(V, 32).
+ * One CTA per row; no workspace. Errors: DDT_ERR_INVALID_ARG (nulls, sizes,
+ *   dtype).
+ */
+DDT_API int ddt_drafter_topk(const void* logits, int logits_dtype, int V, int R, int K, float* logp,
+                             int32_t* tok, int32_t* dev_status, cudaStream_t stream);
 
 /*
  * ddt_build_tree -- best-first draft tree for every request.

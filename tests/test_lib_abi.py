@@ -90,3 +90,14 @@ def test_noalloc_accept_rejects_sizes_beyond_its_array(so):
     st = so.ddt_accept_compact_noalloc(None, 1, 163840, p, p, p, 1, 64, p, 1, 576, 1, 0, p, p, p, p, p, p, p, p, p,
                                        None)
     assert st == lib.DDT_ERR_INVALID_ARG
+
+
+def test_drafter_topk_host_validation(so):
+    p = ctypes.c_void_p(256)
+    # nulls, K outside [1, min(V, 32)], bad dtype: rejected before any CUDA call
+    assert so.ddt_drafter_topk(None, 1, 100, 4, 8, p, p, None, None) == lib.DDT_ERR_INVALID_ARG
+    assert so.ddt_drafter_topk(p, 1, 100, 4, 33, p, p, None, None) == lib.DDT_ERR_INVALID_ARG
+    assert so.ddt_drafter_topk(p, 1, 4, 4, 5, p, p, None, None) == lib.DDT_ERR_INVALID_ARG
+    assert so.ddt_drafter_topk(p, 1, 100, 4, 0, p, p, None, None) == lib.DDT_ERR_INVALID_ARG
+    assert so.ddt_drafter_topk(p, 7, 100, 4, 8, p, p, None, None) == lib.DDT_ERR_INVALID_ARG
+    assert so.ddt_drafter_topk(p, 1, 100, 0, 8, p, p, None, None) == lib.DDT_ERR_INVALID_ARG
