@@ -97,13 +97,22 @@ __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams 
   const size_t esz = kBF16 ? 2 : 4;
   const unsigned char* row = static_cast<const unsigned char*>(p.logits) + (size_t)r * V * esz;
 
-  unsigned long long k[KM];
-#pragma unroll
-  for (int i = 0; i < KM; ++i) k[i] = 0ull;  // 0 = empty; every finite value's key is larger
+  // The warp's K best so far, lane j holding entry j (0 = empty; every
+  // finite value's key is larger); wthr = its last entry. A value is only
+  // looked at further when it beats wthr, so after the first few batches a
+  // value costs one compare and its warp one ballot.
+  unsigned long long wl = 0ull, wthr = 0ull;
   float m = -INFINITY, s = 0.0f;
   bool bad = false;
-  // a batch of values: one running-max update, a batch sum of exponentials,
-  // then the top-k candidates (one compare per value unless it beats the K-th)
+  auto insert = [&](unsigned long long key) {
+    // lanes whose entry beats key keep their place; the rest move down one
+    const int pos = __popc(__ballot_sync(DDT_FULL_MASK, lane < p.K && wl > key));
+    const unsigned long long up = __shfl_up_sync(DDT_FULL_MASK, wl, 1);
+    if (lane > pos && lane < p.K) wl = up;
+    if (lane == pos && pos < p.K) wl = key;
+    wthr = __shfl_sync(DDT_FULL_MASK, wl, p.K - 1);
+  };
+  // a batch of n of this lane's values (all lanes of the warp call it together)
   auto batch = [&](const float* x, int n, int idx0) {
     float y[8];
     float bm = -INFINITY;
@@ -125,41 +134,52 @@ __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams 
       if (t < n) bs += ex2_ftz(y[t] - m);
     s += bs;
 #pragma unroll
-    for (int t = 0; t < 8; ++t)
-      if (t < n) topk_insert<KM>(k, drafter_key(x[t], idx0 + t));
+    for (int t = 0; t < 8; ++t) {
+      const unsigned long long key =
+          (t < n && fabsf(x[t]) <= 3.402823466e38f) ? drafter_key(x[t], idx0 + t) : 0ull;
+      unsigned hits = __ballot_sync(DDT_FULL_MASK, key > wthr);
+      while (hits) {  // warp-uniform
+        const int src = __ffs(hits) - 1;
+        hits &= hits - 1u;
+        const unsigned long long kk = __shfl_sync(DDT_FULL_MASK, key, src);
+        if (kk > wthr) insert(kk);
+      }
+    }
   };
   if (p.vec) {  // 16-byte aligned rows: 8 bf16 or 4 f32 per load
     constexpr int kPer = kBF16 ? 8 : 4;
     const int nvec = V / kPer;
     const uint4* src = reinterpret_cast<const uint4*>(row);
-    // eight 16-byte loads in flight per thread (64 KB per CTA) before any is used
+    // eight 16-byte loads in flight per thread (64 KB per CTA) before any is
+    // used; whole warps step together (lanes past the end take no values)
     constexpr int kU = 8;
-    for (int e0 = tid; e0 < nvec; e0 += kU * kDrThreads) {
+    for (int e0 = warp * 32; e0 < nvec; e0 += kU * kDrThreads) {
       uint4 v[kU];
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
-        const int e = e0 + u * kDrThreads;
+        const int e = e0 + lane + u * kDrThreads;
         v[u] = e < nvec ? __ldcs(src + e) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
-        const int e = e0 + u * kDrThreads;
-        if (e >= nvec) break;
+        const int e = e0 + lane + u * kDrThreads;
         const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
         float x[8];
 #pragma unroll
         for (int t = 0; t < kPer; ++t)
           x[t] = kBF16 ? __uint_as_float((t & 1) ? (w[t >> 1] & 0xffff0000u) : (w[t >> 1] << 16))
                        : __uint_as_float(w[t]);
-        batch(x, kPer, e * kPer);
+        batch(x, e < nvec ? kPer : 0, e * kPer);
       }
     }
   } else {
-    for (int i = tid; i < V; i += kDrThreads) {
+    for (int i0 = warp * 32; i0 < V; i0 += kDrThreads) {  // whole warps step together
+      const int i = i0 + lane;
       float x[8];
-      x[0] = kBF16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(row)[i])
-                   : reinterpret_cast<const float*>(row)[i];
-      batch(x, 1, i);
+      x[0] = i < V ? (kBF16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(row)[i])
+                            : reinterpret_cast<const float*>(row)[i])
+                   : 0.0f;
+      batch(x, i < V ? 1 : 0, i);
     }
   }
   // ---- combine: log-sum-exp and non-finite flag
@@ -173,8 +193,7 @@ __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams 
     lse_merge(m, s, m2, s2);
   }
   const bool wbad = __any_sync(DDT_FULL_MASK, bad);
-  // ---- combine: each warp's K best
-  const unsigned long long wk = warp_topk<KM>(k, p.K, lane);
+  const unsigned long long wk = wl;  // this warp's K best: lane j holds entry j
   __syncthreads();
   if (lane == 0) {
     s_m[warp] = m;
