@@ -64,6 +64,8 @@ struct DrafterParams {
   int32_t* tok;         // [R][K]
   int32_t* dev_status;  // [R], nullable
   int vec;              // rows are 16-byte aligned
+  int C;                // CTAs (one cluster) per row
+  int chunk;            // logits per CTA (a multiple of 8)
 };
 int launch_drafter_topk(DrafterParams p, cudaStream_t stream);
 

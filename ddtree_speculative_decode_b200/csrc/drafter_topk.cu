@@ -9,17 +9,43 @@
 // Broader Context": the draft tree is built from the drafter's per-depth
 // top-k).
 //
-// One CTA per row streams the row once with 16-byte loads, eight in flight
-// per thread. Each thread keeps
+// A row is split over the CTAs of one cluster (up to 8); each streams its
+// slice once with 16-byte loads, eight in flight per thread. Each thread keeps
 // a running (max, sum of exponentials) for the log-sum-exp and a sorted list
 // of its K best packed keys (order-preserving value bits << 32 | ~index, so a
 // larger key is a larger value or, on equal values, a lower index); a new
-// value costs one compare unless it beats the thread's K-th best. Warps then
-// merge their lists by K rounds of a warp-wide maximum, and one warp merges
-// the warps' lists the same way.
+// value costs one compare unless it beats the warp's K-th best. One warp per
+// CTA merges the warps' lists by K rounds of a warp-wide maximum, and the
+// cluster's first CTA merges the CTAs' lists, read through distributed shared
+// memory, the same way.
+#include <algorithm>
+
 #include "ddt_kernels.cuh"
+#include "sm100_ptx.cuh"
 
 namespace ddt {
+
+using sm100::cluster_ctarank;
+using sm100::cluster_sync;
+using sm100::map_to_rank;
+using sm100::smem_u32;
+
+// loads from shared memory of a CTA of the cluster (address from map_to_rank)
+__device__ __forceinline__ unsigned long long ld_cluster_u64(uint32_t addr) {
+  unsigned long long v;
+  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
 
 constexpr int kDrThreads = 512;
 constexpr int kDrWarps = kDrThreads / 32;
@@ -91,9 +117,11 @@ template <int KM, bool kBF16>
 __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams p) {
   pdl_wait();
   pdl_launch_dependents();
-  const int r = blockIdx.x;
+  const uint32_t crank = cluster_ctarank();  // this CTA's slice of the row
+  const int r = (int)(blockIdx.x / (unsigned)p.C);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int V = p.V;
+  const int v0 = min(V, (int)crank * p.chunk), v1 = min(V, v0 + p.chunk);
   const size_t esz = kBF16 ? 2 : 4;
   const unsigned char* row = static_cast<const unsigned char*>(p.logits) + (size_t)r * V * esz;
 
@@ -148,12 +176,12 @@ __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams 
   };
   if (p.vec) {  // 16-byte aligned rows: 8 bf16 or 4 f32 per load
     constexpr int kPer = kBF16 ? 8 : 4;
-    const int nvec = V / kPer;
+    const int nvec = v1 / kPer;  // the slice [v0, v1) starts on a vector
     const uint4* src = reinterpret_cast<const uint4*>(row);
     // eight 16-byte loads in flight per thread (64 KB per CTA) before any is
     // used; whole warps step together (lanes past the end take no values)
     constexpr int kU = 8;
-    for (int e0 = warp * 32; e0 < nvec; e0 += kU * kDrThreads) {
+    for (int e0 = v0 / kPer + warp * 32; e0 < nvec; e0 += kU * kDrThreads) {
       uint4 v[kU];
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
@@ -173,13 +201,13 @@ __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams 
       }
     }
   } else {
-    for (int i0 = warp * 32; i0 < V; i0 += kDrThreads) {  // whole warps step together
+    for (int i0 = v0 + warp * 32; i0 < v1; i0 += kDrThreads) {  // whole warps step together
       const int i = i0 + lane;
       float x[8];
-      x[0] = i < V ? (kBF16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(row)[i])
-                            : reinterpret_cast<const float*>(row)[i])
-                   : 0.0f;
-      batch(x, i < V ? 1 : 0, i);
+      x[0] = i < v1 ? (kBF16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(row)[i])
+                             : reinterpret_cast<const float*>(row)[i])
+                    : 0.0f;
+      batch(x, i < v1 ? 1 : 0, i);
     }
   }
   // ---- combine: log-sum-exp and non-finite flag
@@ -202,40 +230,101 @@ __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams 
   }
   if (lane < p.K) s_keys[warp][lane] = wk;
   __syncthreads();
-  if (warp != 0) return;
-  // warp 0: the row's K best over the warps' lists (lane w < 16 holds warp w's)
-  unsigned long long kk[KM];
+  // this CTA's K best and (max, sum) over its warps, for the cluster's first CTA
+  __shared__ unsigned long long s_cta[KM];
+  __shared__ float s_cta_m, s_cta_s;
+  __shared__ int s_cta_bad;
+  if (warp == 0) {
+    unsigned long long kk[KM];
 #pragma unroll
-  for (int i = 0; i < KM; ++i) kk[i] = (lane < kDrWarps && i < p.K) ? s_keys[lane][i] : 0ull;
-  const unsigned long long best = warp_topk<KM>(kk, p.K, lane);
-  float M = lane < kDrWarps ? s_m[lane] : -INFINITY, S = lane < kDrWarps ? s_s[lane] : 0.0f;
+    for (int i = 0; i < KM; ++i) kk[i] = (lane < kDrWarps && i < p.K) ? s_keys[lane][i] : 0ull;
+    const unsigned long long best = warp_topk<KM>(kk, p.K, lane);
+    float M = lane < kDrWarps ? s_m[lane] : -INFINITY, S = lane < kDrWarps ? s_s[lane] : 0.0f;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float m2 = __shfl_xor_sync(DDT_FULL_MASK, M, o), s2 = __shfl_xor_sync(DDT_FULL_MASK, S, o);
-    lse_merge(M, S, m2, s2);
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(DDT_FULL_MASK, M, o), s2 = __shfl_xor_sync(DDT_FULL_MASK, S, o);
+      lse_merge(M, S, m2, s2);
+    }
+    if (lane < p.K) s_cta[lane] = best;
+    if (lane == 0) {
+      s_cta_m = M;
+      s_cta_s = S;
+      s_cta_bad = s_bad;
+    }
   }
-  const bool row_bad = s_bad != 0;
-  if (lane < p.K) {
-    const float lse = (M + log2f(S)) * 0.6931471805599453f;
-    p.logp[(size_t)r * p.K + lane] = row_bad ? -INFINITY : key_value(best) - lse;
-    p.tok[(size_t)r * p.K + lane] = row_bad ? -1 : static_cast<int32_t>(~static_cast<uint32_t>(best & 0xffffffffull));
+  // every thread of every CTA of the cluster takes both cluster barriers
+  cluster_sync();
+  if (crank == 0 && warp == 0) {
+    // lane q < C reads CTA q's list and (max, sum)
+    const bool has = lane < p.C;
+    unsigned long long kk[KM];
+#pragma unroll
+    for (int i = 0; i < KM; ++i)
+      kk[i] = (has && i < p.K) ? ld_cluster_u64(map_to_rank(smem_u32(&s_cta[i]), (uint32_t)lane)) : 0ull;
+    float M = has ? ld_cluster_f32(map_to_rank(smem_u32(&s_cta_m), (uint32_t)lane)) : -INFINITY;
+    float S = has ? ld_cluster_f32(map_to_rank(smem_u32(&s_cta_s), (uint32_t)lane)) : 0.0f;
+    const int qbad = has ? ld_cluster_s32(map_to_rank(smem_u32(&s_cta_bad), (uint32_t)lane)) : 0;
+    const unsigned long long best = warp_topk<KM>(kk, p.K, lane);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(DDT_FULL_MASK, M, o), s2 = __shfl_xor_sync(DDT_FULL_MASK, S, o);
+      lse_merge(M, S, m2, s2);
+    }
+    const bool row_bad = __any_sync(DDT_FULL_MASK, qbad != 0);
+    if (lane < p.K) {
+      const float lse = (M + log2f(S)) * 0.6931471805599453f;
+      p.logp[(size_t)r * p.K + lane] = row_bad ? -INFINITY : key_value(best) - lse;
+      p.tok[(size_t)r * p.K + lane] =
+          row_bad ? -1 : static_cast<int32_t>(~static_cast<uint32_t>(best & 0xffffffffull));
+    }
+    if (lane == 0 && p.dev_status) p.dev_status[r] = row_bad ? DDT_ERR_INPUT : DDT_OK;
   }
-  if (lane == 0 && p.dev_status) p.dev_status[r] = row_bad ? DDT_ERR_INPUT : DDT_OK;
+  cluster_sync();  // the slices' shared memory stays until the first CTA has read it
+}
+
+template <int KM, bool kBF16>
+static int launch_dr_t(const DrafterParams& p, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(p.R * p.C));
+  cfg.blockDim = dim3(kDrThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)p.C;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, drafter_topk_kernel<KM, kBF16>, p) == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
 }
 
 template <int KM>
 static int launch_dr(const DrafterParams& p, cudaStream_t stream) {
-  if (p.logits_dtype == DDT_BF16)
-    return launch_pdl(drafter_topk_kernel<KM, true>, (unsigned)p.R, kDrThreads, 0, stream, p);
-  return launch_pdl(drafter_topk_kernel<KM, false>, (unsigned)p.R, kDrThreads, 0, stream, p);
+  if (p.logits_dtype == DDT_BF16) return launch_dr_t<KM, true>(p, stream);
+  return launch_dr_t<KM, false>(p, stream);
 }
 
 int launch_drafter_topk(DrafterParams p, cudaStream_t stream) {
   const size_t esz = p.logits_dtype == DDT_BF16 ? 2 : 4;
   p.vec = (reinterpret_cast<uintptr_t>(p.logits) % 16 == 0) && (((size_t)p.V * esz) % 16 == 0);
-  if (p.K <= 8) return launch_dr<8>(p, stream);
-  if (p.K <= 16) return launch_dr<16>(p, stream);
-  return launch_dr<32>(p, stream);
+  // slices of at least 16384 logits, at most 8 CTAs (one portable cluster) per
+  // row; slice starts stay on a 16-byte vector
+  auto launch = [&](int C) -> int {
+    p.C = C;
+    p.chunk = ((p.V + C - 1) / C + 7) / 8 * 8;
+    if (p.K <= 8) return launch_dr<8>(p, stream);
+    if (p.K <= 16) return launch_dr<16>(p, stream);
+    return launch_dr<32>(p, stream);
+  };
+  const int C = std::max(1, std::min(8, (p.V + 16383) / 16384));
+  if (C > 1) {
+    if (launch(C) == DDT_OK) return DDT_OK;
+    (void)cudaGetLastError();  // clusters of C not schedulable here: one CTA per row
+  }
+  return launch(1);
 }
 
 }  // namespace ddt

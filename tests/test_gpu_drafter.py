@@ -1,7 +1,8 @@
 """GPU parity of ddt_drafter_topk against oracle.drafter_topk: token ids bit
 exact (top-k order, ties to the lower index), log-probs within a float32
 tolerance, on Kimi-sized rows, odd vocabulary sizes (scalar path), every K
-range of the kernel and heavily tied rows."""
+range of the kernel, rows split over several CTAs (a cluster of up to 8 per
+row, slices of at least 16384 logits) and heavily tied rows."""
 import numpy as np
 import pytest
 import torch
@@ -50,7 +51,11 @@ def test_kimi_rows(dtype, K):
     _check(out, z, K)
 
 
-@pytest.mark.parametrize("V,K", [(1, 1), (5, 5), (7, 3), (256, 8), (1001, 16), (4099, 32), (65537, 9)])
+@pytest.mark.parametrize(
+    "V,K",
+    [(1, 1), (5, 5), (7, 3), (256, 8), (1001, 16), (4099, 32), (16384, 4), (16392, 5), (40000, 16),
+     (65537, 9), (114696, 32), (200000, 8)],
+)
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_sizes(V, K, dtype):
     t, z = _logits(5, V, dtype, seed=V + K)
@@ -65,6 +70,34 @@ def test_ties_go_to_the_lower_index(dtype):
     out = lib.drafter_topk(t, 32)
     torch.cuda.synchronize()
     _check(out, z, 32)
+
+
+@pytest.mark.parametrize("V", [40000, 163840, 50001])
+def test_ties_and_winners_across_slices(V):
+    """Equal maxima in different CTAs' slices go to the lower index; the K
+    best all in the last slice, or straddling a slice start."""
+    z = np.random.default_rng(V).standard_normal((4, V)).astype(np.float32)
+    z[0, [V - 1, V // 2, 3, V // 3 + 1]] = 9.0      # four-way tie across slices
+    z[1, V - 20:] = np.linspace(5.0, 8.0, 20, dtype=np.float32)  # all winners last
+    C = min(8, (V + 16383) // 16384)
+    chunk = ((V + C - 1) // C + 7) // 8 * 8
+    for c in range(1, C):                           # around each slice start
+        z[2, c * chunk - 2: c * chunk + 2] = 7.0 + c * 0.01
+    z[3, :] = 0.0                                   # all equal: ids 0..K-1
+    out = lib.drafter_topk(torch.from_numpy(z).to(DEV), 16)
+    torch.cuda.synchronize()
+    _check(out, z, 16)
+    assert list(out["tok"].cpu().numpy()[3]) == list(range(16))
+
+
+def test_non_finite_in_a_later_slice():
+    z = np.random.default_rng(5).standard_normal((3, 100000)).astype(np.float32)
+    z[0, 99999] = np.nan
+    z[2, 60000] = np.inf
+    out = lib.drafter_topk(torch.from_numpy(z).to(DEV), 8)
+    torch.cuda.synchronize()
+    _check(out, z, 8)
+    assert list(out["status"].cpu().numpy()) == [lib.DDT_ERR_INPUT, lib.DDT_OK, lib.DDT_ERR_INPUT]
 
 
 def test_non_finite_rows():
