@@ -11,13 +11,17 @@
 //
 // A row is split over the CTAs of one cluster (up to 8); each streams its
 // slice once with 16-byte loads, eight in flight per thread. Each thread keeps
-// a running (max, sum of exponentials) for the log-sum-exp and a sorted list
-// of its K best packed keys (order-preserving value bits << 32 | ~index, so a
-// larger key is a larger value or, on equal values, a lower index); a new
-// value costs one compare unless it beats the warp's K-th best. One warp per
-// CTA merges the warps' lists by K rounds of a warp-wide maximum, and the
-// cluster's first CTA merges the CTAs' lists, read through distributed shared
-// memory, the same way.
+// a running (max, sum of exponentials) for the log-sum-exp; each warp keeps a
+// sorted list of its K best packed keys (order-preserving value bits << 32 |
+// ~index, so a larger key is a larger value or, on equal values, a lower
+// index). A new value costs one compare unless it beats the larger of the
+// warp's K-th best and the best K-th entry any warp of the CTA has published
+// (no value below either can be among the row's K best); the few that do are
+// taken by one out-of-line routine, inserted one by one or, when many lanes
+// hit at once, by a bitonic sort of the hits and a bitonic merge with the
+// list. One warp per CTA merges the warps' lists by K rounds of a warp-wide
+// maximum, and the cluster's first CTA merges the CTAs' lists, read through
+// distributed shared memory, the same way.
 #include <algorithm>
 
 #include "ddt_kernels.cuh"
@@ -79,17 +83,62 @@ __device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2
   m = M;
 }
 
-template <int KM>
-__device__ __forceinline__ void topk_insert(unsigned long long (&k)[KM], unsigned long long key) {
-  if (key <= k[KM - 1]) return;
-  k[KM - 1] = key;
+// Bitonic network over the warp's 32 lanes, one key per lane: the full sort
+// leaves lane 0 with the largest key; the merge sorts a bitonic sequence.
+__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long x, int lane) {
 #pragma unroll
-  for (int j = KM - 1; j > 0; --j) {
-    const unsigned long long a = k[j - 1], b = k[j];
-    const bool sw = b > a;
-    k[j - 1] = sw ? b : a;
-    k[j] = sw ? a : b;
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const unsigned long long y = __shfl_xor_sync(DDT_FULL_MASK, x, j);
+      // blocks of k lanes alternate direction; the lower lane of a pair keeps
+      // the larger key in a descending block
+      const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+      x = keep_max ? (y > x ? y : x) : (y < x ? y : x);
+    }
   }
+  return x;
+}
+
+__device__ __forceinline__ unsigned long long warp_merge_desc(unsigned long long x, int lane) {
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const unsigned long long y = __shfl_xor_sync(DDT_FULL_MASK, x, j);
+    x = ((lane & j) == 0) ? (y > x ? y : x) : (y < x ? y : x);
+  }
+  return x;
+}
+
+constexpr int kMergeHits = 6;  // from this many hits one sort-merge beats serial inserts
+
+// Takes a warp's hits (cand on the lanes set in hits, 0 elsewhere) into its
+// sorted list wl (lane j = entry j, 0 = empty, lanes >= K hold 0); returns the
+// new list. Out of line: one copy of the code serves every call site.
+__device__ __noinline__ unsigned long long take_hits(unsigned long long wl, unsigned long long cand,
+                                                     unsigned hits, int K, int lane) {
+  if (__popc(hits) >= kMergeHits) {
+    // sorted hits reversed (ascending) against the descending list: the
+    // lane-wise maximum holds the 32 best of both as a bitonic sequence
+    const unsigned long long c = warp_sort_desc(cand, lane);
+    const unsigned long long crev = __shfl_sync(DDT_FULL_MASK, c, 31 - lane);
+    const unsigned long long m = warp_merge_desc(wl > crev ? wl : crev, lane);
+    return lane < K ? m : 0ull;
+  }
+  unsigned long long last = __shfl_sync(DDT_FULL_MASK, wl, K - 1);
+  while (hits) {  // warp-uniform
+    const int src = __ffs(hits) - 1;
+    hits &= hits - 1u;
+    const unsigned long long kk = __shfl_sync(DDT_FULL_MASK, cand, src);
+    if (kk > last) {
+      // lanes whose entry beats kk keep their place; the rest move down one
+      const int pos = __popc(__ballot_sync(DDT_FULL_MASK, lane < K && wl > kk));
+      const unsigned long long up = __shfl_up_sync(DDT_FULL_MASK, wl, 1);
+      if (lane > pos && lane < K) wl = up;
+      if (lane == pos && pos < K) wl = kk;
+      last = __shfl_sync(DDT_FULL_MASK, wl, K - 1);
+    }
+  }
+  return wl;
 }
 
 // The warp's K best keys over the lanes' sorted lists (each consumed from its
@@ -126,19 +175,26 @@ __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams 
   const unsigned char* row = static_cast<const unsigned char*>(p.logits) + (size_t)r * V * esz;
 
   // The warp's K best so far, lane j holding entry j (0 = empty; every
-  // finite value's key is larger); wthr = its last entry. A value is only
-  // looked at further when it beats wthr, so after the first few batches a
-  // value costs one compare and its warp one ballot.
-  unsigned long long wl = 0ull, wthr = 0ull;
+  // finite value's key is larger); wthr = its last entry, s_thr = the largest
+  // last entry any warp of this CTA has published. A key at or below either
+  // has K larger keys in the row, so it is dropped: after the first few
+  // batches a value costs one compare and its warp one ballot.
+  __shared__ unsigned long long s_thr;
+  if (tid == 0) s_thr = 0ull;
+  __syncthreads();
+  unsigned long long wl = 0ull, wthr = 0ull, thr = 0ull, pub = 0ull;
   float m = -INFINITY, s = 0.0f;
   bool bad = false;
-  auto insert = [&](unsigned long long key) {
-    // lanes whose entry beats key keep their place; the rest move down one
-    const int pos = __popc(__ballot_sync(DDT_FULL_MASK, lane < p.K && wl > key));
-    const unsigned long long up = __shfl_up_sync(DDT_FULL_MASK, wl, 1);
-    if (lane > pos && lane < p.K) wl = up;
-    if (lane == pos && pos < p.K) wl = key;
-    wthr = __shfl_sync(DDT_FULL_MASK, wl, p.K - 1);
+  // before each batch: the CTA's threshold; after it: publish this warp's
+  auto refresh = [&]() {
+    const unsigned long long c = *reinterpret_cast<volatile unsigned long long*>(&s_thr);
+    thr = c > wthr ? c : wthr;
+  };
+  auto publish = [&]() {
+    if (wthr > pub) {  // warp-uniform
+      if (lane == 0) atomicMax(&s_thr, wthr);
+      pub = wthr;
+    }
   };
   // a batch of n of this lane's values (all lanes of the warp call it together)
   auto batch = [&](const float* x, int n, int idx0) {
@@ -165,12 +221,12 @@ __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams 
     for (int t = 0; t < 8; ++t) {
       const unsigned long long key =
           (t < n && fabsf(x[t]) <= 3.402823466e38f) ? drafter_key(x[t], idx0 + t) : 0ull;
-      unsigned hits = __ballot_sync(DDT_FULL_MASK, key > wthr);
-      while (hits) {  // warp-uniform
-        const int src = __ffs(hits) - 1;
-        hits &= hits - 1u;
-        const unsigned long long kk = __shfl_sync(DDT_FULL_MASK, key, src);
-        if (kk > wthr) insert(kk);
+      const bool hit = key > thr;
+      const unsigned hits = __ballot_sync(DDT_FULL_MASK, hit);
+      if (hits) {  // warp-uniform
+        wl = take_hits(wl, hit ? key : 0ull, hits, p.K, lane);
+        wthr = __shfl_sync(DDT_FULL_MASK, wl, p.K - 1);
+        thr = wthr > thr ? wthr : thr;
       }
     }
   };
@@ -197,7 +253,9 @@ __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams 
         for (int t = 0; t < kPer; ++t)
           x[t] = kBF16 ? __uint_as_float((t & 1) ? (w[t >> 1] & 0xffff0000u) : (w[t >> 1] << 16))
                        : __uint_as_float(w[t]);
+        refresh();
         batch(x, e < nvec ? kPer : 0, e * kPer);
+        publish();
       }
     }
   } else {
@@ -207,7 +265,9 @@ __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams 
       x[0] = i < v1 ? (kBF16 ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(row)[i])
                              : reinterpret_cast<const float*>(row)[i])
                     : 0.0f;
+      refresh();
       batch(x, i < v1 ? 1 : 0, i);
+      publish();
     }
   }
   // ---- combine: log-sum-exp and non-finite flag
