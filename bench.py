@@ -366,6 +366,8 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
         step(sets[k % n_sets], evs[k])
     torch.cuda.synchronize()
     dr = measure_drafter(args, shape, lib, dev, tdt)
+    comp = None if args.sweep or args.layers < 2 else measure_compaction(
+        args, shape, lib, dev, tdt, sets[0], tree, cl0, off, cap, acc, ws_acc)
     build_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     accept_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
@@ -396,6 +398,8 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
         "accept_hbm": {"achieved_gbs": acc_bytes / (accept_ms / 1e3) / 1e9, "peak_gbs": pk["hbm_gbs"],
                        "frac": acc_bytes / (accept_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
         "drafter_topk": dict(dr, frac=dr["gbs"] / pk["hbm_gbs"], peak_gbs=pk["hbm_gbs"]),
+        "compaction_layers": None if comp is None else dict(
+            comp, frac=comp["marginal_gbs"] / pk["hbm_gbs"], peak_gbs=pk["hbm_gbs"]),
         "nodes_per_step": n_nodes_total,
         "attn_gflop_per_step": flops / 1e9,
         "gpu_launches": launches_per_step * args.steps,
@@ -419,6 +423,64 @@ def attn_launches(shape: synth.Shape) -> int:
 def _tdtype(shape):
     import torch
     return torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+
+
+def measure_compaction(args, shape, lib, dev, tdt, s, tree, cl0, off, cap, acc, ws_acc):
+    """ddt_accept_compact on a pool of args.layers copies of the workload's
+    latent cache at a layer stride (every layer compacted along the same
+    accepted path), against the same call on one layer. The target logits are
+    the step's with one change: along each tree's deepest path (to its
+    deepest node, the lowest index on ties) the next node's token is made the
+    argmax, so every request accepts that whole path (several tokens per step,
+    as the pages' runs do). Each call is timed
+    alone with events after writing a buffer larger than L2, so the moved rows
+    come from HBM. The marginal bandwidth counts the extra layers' bytes (each
+    accepted row read once and written once) over the extra time."""
+    import torch
+    layers = args.layers
+    par, tokn = tree["parent"].cpu().numpy(), tree["node_tok"].cpu().numpy()
+    dep, nn = tree["depth"].cpu().numpy(), tree["n_nodes"].cpu().numpy()
+    logits = s["logits"].clone()
+    for b in range(len(nn)):
+        node = int(np.argmax(dep[b, :int(nn[b])]))
+        while node > 0:
+            logits[b, int(par[b, node]), int(tokn[b, node])] = 30.0  # above every drawn logit
+            node = int(par[b, node])
+    kv1 = s["kv"]
+    stride = kv1.shape[0]
+    pool = kv1.unsqueeze(0).expand(layers, stride, kv1.shape[1]).contiguous().view(layers * stride, kv1.shape[1])
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    cl = cl0.clone()
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(n_layers, kv, reps):
+        ts = []
+        for _ in range(reps):
+            torch.add(cl0, 0, out=cl)
+            flush.zero_()  # also keeps the GPU busy while the host enqueues the call
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            lib.accept_compact(logits, tree["node_tok"], tree["parent"], tree["n_nodes"], kv, off, cl, cap,
+                               n_layers=n_layers, layer_stride_rows=stride, out=acc, workspace=ws_acc,
+                               stream=stream)
+            e1.record(stream)
+            ts.append((e0, e1))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ts) * 1e3
+
+    timed(1, kv1, 3)
+    timed(layers, pool, 3)
+    us1 = timed(1, kv1, 30)
+    usL = timed(layers, pool, 30)
+    a = acc["acc_len"].cpu().numpy().astype(np.int64)
+    row_bytes = kv1.shape[1] * kv1.element_size()
+    per_layer = float(2 * (a + 1).sum() * row_bytes)
+    del pool, flush, logits
+    return {"layers": layers, "accepted_rows": int((a + 1).sum()), "us_1_layer": us1, "us": usL,
+            "bytes_per_layer": per_layer,
+            "marginal_gbs": per_layer * (layers - 1) / max(usL - us1, 1e-3) * 1e-3,
+            "gbs": per_layer * layers / usL * 1e-3,
+            "timing": "one call per pair of events after a 252 MiB L2 flush; median of 30"}
 
 
 def measure_drafter(args, shape, lib, dev, tdt):
@@ -559,6 +621,8 @@ def main():
     ap.add_argument("--config", default="kimi-1req", choices=sorted(synth.NAMED))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--layers", type=int, default=61,
+                    help="layers of the multi-layer compaction measurement (< 2: skip it)")
     ap.add_argument("--ref-nodes", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--e2e-serial", action="store_true",

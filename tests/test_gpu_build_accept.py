@@ -184,6 +184,21 @@ def test_accept_ties_and_multilayer():
     _run_accept_and_compare(s, x, tree, logits, n_layers=2, stride=stride, kv_host=kv2)
 
 
+def test_accept_many_layers():
+    """61 layers (the Kimi model's depth) at a stride, each holding different
+    rows: every layer compacted along the same accepted path."""
+    s = synth.custom(B=3, D=4, K=3, N=16, H=1, d_l=64, d_r=16, V=500, L=(7, 0, 40), dtype="bf16", seed=61,
+                     accept_p=0.9)
+    x, tree, logits = _accept_case(s)
+    rows, n_layers = x.kv.shape[0], 61
+    stride = rows + 3
+    kvl = np.zeros((stride * n_layers, x.kv.shape[1]), x.kv.dtype)
+    for layer in range(n_layers):
+        kvl[layer * stride:layer * stride + rows] = np.roll(x.kv, layer, axis=0)
+    got, _ = _run_accept_and_compare(s, x, tree, logits, n_layers=n_layers, stride=stride, kv_host=kvl)
+    assert got["acc_len"].sum() > 0
+
+
 def test_accept_capacity_and_empty_tree():
     s = synth.custom(B=3, D=3, K=2, N=6, H=1, d_l=8, d_r=0, V=50, L=(3, 3, 3), seed=4)
     x, tree, logits = _accept_case(s)

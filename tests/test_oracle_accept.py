@@ -196,6 +196,36 @@ def test_multi_layer_and_capacity():
         np.testing.assert_array_equal(kv2[layer * stride + 3], before[layer * stride + 4])
 
 
+def test_many_layers_equal_one_layer_each():
+    """61 layers at a stride are 61 independent copies along the same path:
+    each layer's slice ends as a one-layer call on that slice alone leaves it,
+    and the gap rows between layers stay untouched."""
+    rng = np.random.default_rng(61)
+    parent = np.array([[-1, 0, 0, 1, 2, 4, 4]], np.int32)
+    node_tok = np.array([[9, 3, 4, 5, 6, 7, 8]], np.int32)
+    lg = rng.standard_normal((1, 7, 12)).astype(np.float32)
+    lg[0, 0, 4] = 9.0  # root -> node 2
+    lg[0, 2, 6] = 9.0  # node 2 -> node 4
+    lg[0, 4, 8] = 9.0  # node 4 -> node 6
+    L, n_layers, rows = 5, 61, 12
+    stride = rows + 2
+    kv = rng.standard_normal((n_layers * stride, 3))
+    before = kv.copy()
+    r = accept_compact(lg, "f32", node_tok, parent, np.array([7]), kv, np.array([0]), np.array([L]),
+                       np.array([L + 7]), n_layers=n_layers, layer_stride_rows=stride)
+    assert list(r["acc_nodes"][0, :4]) == [0, 2, 4, 6] and r["acc_len"][0] == 3
+    for layer in range(n_layers):
+        one = before[layer * stride:layer * stride + rows].copy()
+        r1 = accept_compact(lg, "f32", node_tok, parent, np.array([7]), one, np.array([0]), np.array([L]),
+                            np.array([L + 7]))
+        assert r1["acc_len"][0] == 3
+        np.testing.assert_array_equal(kv[layer * stride:layer * stride + rows], one)
+        np.testing.assert_array_equal(kv[layer * stride + rows:(layer + 1) * stride],
+                                      before[layer * stride + rows:(layer + 1) * stride])
+        for j, node in enumerate([0, 2, 4, 6]):
+            np.testing.assert_array_equal(kv[layer * stride + L + j], before[layer * stride + L + node])
+
+
 def test_walk_picks_lowest_index_on_duplicate_tokens():
     parent = [-1, 0, 0]
     node_tok = [1, 5, 5]
