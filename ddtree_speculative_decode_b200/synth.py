@@ -266,6 +266,43 @@ def target_logits(shape: Shape, parent: np.ndarray, node_tok: np.ndarray, n_node
     return out
 
 
+def lmhead_inputs(shape: Shape, parent: np.ndarray, node_tok: np.ndarray, n_nodes: np.ndarray, d_model: int,
+                  requests: Optional[list] = None):
+    """Inputs of the target's LM head for every verify row: the head's weights
+    w_vocab [V, d_model] (one row per token, N(0, 1 / d_model), so logits have
+    unit scale like target_logits') and final hidden states hidden
+    [B, N, d_model] (N(0, 1)). At the same fraction of nodes as target_logits,
+    a uniformly chosen child's token t gets the acceptance bias: hidden row i
+    moves by bias * w_t / |w_t|^2 (w_t as stored), which raises its logit for t
+    by the bias before rounding. Returns (hidden, w_vocab, planted [B, N] i32:
+    the planted token, or -1), hidden and w_vocab in the shape's dtype."""
+    s = shape
+    reqs = list(range(s.B)) if requests is None else list(requests)
+    w32 = (_rng(s.seed, 7).standard_normal((s.V, d_model), dtype=np.float32) /
+           np.float32(math.sqrt(d_model))).astype(np.float32)
+    w = _store(w32, s.dtype)
+    wv = w.astype(np.float64) if s.dtype == "f32" else bf16_bits_to_f32(w).astype(np.float64)
+    hidden = np.empty((len(reqs), s.N, d_model), w.dtype)
+    planted = np.full((len(reqs), s.N), -1, np.int32)
+    for j, b in enumerate(reqs):
+        h = _rng(s.seed, 8, b).standard_normal((s.N, d_model)).astype(np.float64)
+        rb = _rng(s.seed, 9, b)
+        n = int(n_nodes[j])
+        for i in range(s.N):
+            u = rb.random()
+            pick = rb.random()
+            if i >= n:
+                continue
+            kids = [c for c in range(n) if parent[j, c] == i]
+            if kids and u < s.accept_p:
+                c = kids[min(len(kids) - 1, int(pick * len(kids)))]
+                t = int(node_tok[j, c])
+                h[i] += s.accept_bias * wv[t] / float(wv[t] @ wv[t])
+                planted[j, i] = t
+        hidden[j] = _store(h.astype(np.float32), s.dtype)
+    return hidden, w, planted
+
+
 def oracle_drafter(golden: np.ndarray, D: int, K: int, sentinel_from: Optional[int] = None):
     """Drafter fixture that proposes a known continuation ("ddtree_speculative_
     decode_test_capstone", section "The Oracle Drafter" and "What the Test

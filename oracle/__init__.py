@@ -11,6 +11,10 @@ from .ddt_oracle import (  # noqa: F401
     accept_walk,
     build_tree,
     drafter_topk,
+    lmhead_argmax,
+    lmhead_f32_error_bound,
+    lmhead_logits,
+    lmhead_valid_argmax,
     row_argmax,
     verify_attn,
     visible_keys,

@@ -19,6 +19,10 @@ Conventions (arrays are numpy):
   the root (N - 1 drafted nodes), H heads, d_l latent dim, d_r rope dim,
   V vocab, W = ceil(N / 32) mask words.
 
+Two steps around the path are here as well: the drafter's per-depth
+proposals (log-softmax + top-k over the vocabulary) feeding the build, and the
+target's LM head folded into the accept argmax (logits never stored).
+
 Parity status: every function here is pinned by tests in tests/test_oracle_*.
 """
 from __future__ import annotations
@@ -342,3 +346,68 @@ def drafter_topk(logits, K):
         tok[r] = order.astype(np.int32)
         logp[r] = (z[order] - lse).astype(np.float32)
     return logp, tok, status
+
+
+# ---------------------------------------------------------------------------
+# target LM head folded into the accept argmax
+# ---------------------------------------------------------------------------
+
+
+def lmhead_logits(hidden, w_vocab):
+    """The target's logits from its final hidden states: z[r][v] = sum over c of
+    hidden[r][c] * w_vocab[v][c], in float64 from the stored values (bf16
+    already widened exactly).
+
+    Source: AR page, "What the Message Actually Says" (the greedy token of a
+    verify row is the argmax of the target's logits, checked exactly);
+    "the_validation_pivot", "Assumptions Embedded in This Message" (Kimi K2.6:
+    hidden size 7168; the tests' tiny model: hidden 64, vocabulary 400).
+    hidden: [R, d]; w_vocab: [V, d] (one row per token). Returns [R, V]."""
+    h = np.asarray(hidden, dtype=np.float64)
+    w = np.asarray(w_vocab, dtype=np.float64)
+    return h @ w.T
+
+
+def lmhead_argmax(hidden, w_vocab):
+    """Greedy target token of every verify row without materialised logits:
+    the lowest v attaining the float64 maximum of lmhead_logits (the tie rule
+    is row_argmax's). Returns am [R] int32."""
+    return np.argmax(lmhead_logits(hidden, w_vocab), axis=-1).astype(np.int32)
+
+
+# READING (the pages fix no precision for the head): a GPU evaluates the dot
+# products in float32 with every bf16 x bf16 product exact (16 significant bits
+# fit float32's 24) and every addition off by at most u relative, in an order
+# of its own. If no product passes through more than n roundings on its way
+# into the sum, the classical bound on floating-point summation (Higham,
+# "Accuracy and Stability of Numerical Algorithms", section 4.2) gives
+# |z32 - z| <= gamma(n) * sum over c of |h_c w_vc|, gamma(n) = n u / (1 - n u).
+# n = d - 1 covers every order; an evaluation that adds 16-product steps one
+# after another has n <= 15 + d / 16. u = 2^-22: twice float32's truncation
+# unit, a margin for tensor-core accumulators that align the products of one
+# step to the largest before adding them.
+LMHEAD_U = 2.0 ** -22
+
+
+def lmhead_f32_error_bound(hidden, w_vocab, depth=None):
+    """Per row, the largest over v of the float32 evaluation bound above, for
+    at most ``depth`` roundings per product (default d - 1: any order).
+    Returns [R] float64."""
+    h = np.abs(np.asarray(hidden, dtype=np.float64))
+    w = np.abs(np.asarray(w_vocab, dtype=np.float64))
+    n = max(h.shape[1] - 1, 0) if depth is None else int(depth)
+    gamma = n * LMHEAD_U / (1.0 - n * LMHEAD_U)
+    return gamma * (h @ w.T).max(axis=-1)
+
+
+def lmhead_valid_argmax(hidden, w_vocab, depth=None):
+    """The tokens a float32 evaluation within the bound may pick for each row:
+    every v with z[v] >= max(z) - 2 * bound (a pick g has z[g] >= z32[g] - bound
+    >= z32[am] - bound >= z[am] - 2 * bound). Returns (am [R] int32, valid: a
+    list of R sorted int32 arrays, each holding am)."""
+    z = lmhead_logits(hidden, w_vocab)
+    bound = lmhead_f32_error_bound(hidden, w_vocab, depth)
+    am = np.argmax(z, axis=-1).astype(np.int32)
+    top = z.max(axis=-1)
+    valid = [np.flatnonzero(z[r] >= top[r] - 2.0 * bound[r]).astype(np.int32) for r in range(z.shape[0])]
+    return am, valid
