@@ -175,7 +175,9 @@ def blas_threads() -> int:
 def oracle_step_time(shape: synth.Shape, x, logits, tree, attn_nodes: int, seed: int = 0):
     """Seconds the oracle needs for one full step of this workload, from a
     bounded sample: the whole tree build, attention for `attn_nodes` sampled
-    nodes (all heads) scaled by the node count, the whole accept + compaction."""
+    nodes (all heads) scaled by the node count, the whole accept + compaction.
+    Returns (scaled step seconds, sampled nodes, all nodes, wall seconds of the
+    parts that do not scale with the sample, wall seconds per sampled node)."""
     import oracle
 
     t0 = time.perf_counter()
@@ -194,7 +196,19 @@ def oracle_step_time(shape: synth.Shape, x, logits, tree, attn_nodes: int, seed:
     oracle.accept_compact(logits, shape.dtype, tree["node_tok"], tree["parent"], tree["n_nodes"], kv, x.cache_off,
                           x.cache_len, x.cache_cap)
     t_acc = time.perf_counter() - t0
-    return t_build + t_attn + t_acc, len(pick), len(all_rows)
+    per_node = t_attn / max(1, len(all_rows))
+    return t_build + t_attn + t_acc, len(pick), len(all_rows), t_build + t_acc, per_node
+
+
+def reference_steps(steps: int, budget_s: float, step_wall_s: float) -> int:
+    """How many of the requested steps the reference arm times: all of them if
+    they fit the wall-time budget, else as many as it holds (at least one).
+    The per-step sample stays fixed, so the value does not depend on K (a
+    smaller attention sample would scale the oracle's per-call setup up with
+    it)."""
+    if step_wall_s <= 0:
+        return steps
+    return int(max(1, min(steps, budget_s // step_wall_s)))
 
 
 def run_reference(args, shape: synth.Shape, rank: int):
@@ -208,18 +222,21 @@ def run_reference(args, shape: synth.Shape, rank: int):
     logits = synth.target_logits(shape, tree["parent"], tree["node_tok"], tree["n_nodes"])
     nodes = int(tree["n_nodes"].sum())
     sample = max(1, min(nodes, args.ref_nodes))
-    for _ in range(args.warmup if args.warmup < 2 else 1):
-        oracle_step_time(shape, x, logits, tree, sample)
+    # one untimed step (whatever W is) also measures a step's wall time
+    _, _, _, fixed_s, per_node_s = oracle_step_time(shape, x, logits, tree, sample)
+    run = reference_steps(args.steps, args.ref_budget, fixed_s + sample * per_node_s)
     times = []
-    for k in range(args.steps):
-        t, _, _ = oracle_step_time(shape, x, logits, tree, sample, seed=k)
+    for k in range(run):
+        t, _, _, _, _ = oracle_step_time(shape, x, logits, tree, sample, seed=k)
         times.append(t)
     sec = float(np.mean(times))
     value = nodes / sec
     desc = (f"per step: full tree build, attention on {sample} sampled nodes x {shape.H} heads scaled to "
-            f"{nodes} nodes, full accept + compaction")
+            f"{nodes} nodes, full accept + compaction; {run} of {args.steps} requested steps timed "
+            f"(wall-time budget {args.ref_budget:.0f} s)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "steps": run, "steps_requested": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_dict(shape),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
@@ -607,7 +624,7 @@ def run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_a
 def cpu_baseline(args, shape, x, logits_h, t_host):
     import oracle
     tree = oracle.build_tree(x.logp, x.tok, x.root_tok, x.cache_len, shape.N)
-    sec, picked, total = oracle_step_time(shape, x, logits_h, tree, args.ref_nodes)
+    sec, picked, total, _, _ = oracle_step_time(shape, x, logits_h, tree, args.ref_nodes)
     return {"value": total / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"one step: full build, attention on {picked} of {total} nodes (all heads) scaled by "
                       f"{total}/{picked}, full accept + compaction"}
@@ -624,6 +641,8 @@ def main():
     ap.add_argument("--layers", type=int, default=61,
                     help="layers of the multi-layer compaction measurement (< 2: skip it)")
     ap.add_argument("--ref-nodes", type=int, default=8)
+    ap.add_argument("--ref-budget", type=float, default=120.0,
+                    help="wall seconds the reference arm's timed steps may take")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--e2e-serial", action="store_true",
                     help="end-to-end leg: copy each step's inputs on the compute stream (no overlap)")

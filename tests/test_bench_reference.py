@@ -1,0 +1,39 @@
+"""The reference arm (the oracle timed on the host cores): any --steps K stays
+within the wall-time budget with a fixed per-step sample, and its JSON line
+carries the contract's keys."""
+import json
+import os
+import subprocess
+import sys
+import time
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_all_steps_when_they_fit():
+    assert bench.reference_steps(10, 120.0, 0.15) == 10
+
+
+def test_steps_capped_by_the_budget():
+    run = bench.reference_steps(10000, 120.0, 0.15)
+    assert run == 800 and run * 0.15 <= 120.0
+    assert bench.reference_steps(10000, 120.0, 500.0) == 1  # at least one step
+
+
+def test_reference_line_on_the_tiny_workload():
+    t0 = time.time()
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config",
+                          "tiny-f32", "--steps", "5", "--warmup", "3", "--ref-budget", "20"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert time.time() - t0 < 300
+    assert line["impl"] == "reference" and line["value"] > 0 and line["higher_is_better"] is True
+    assert line["steps"] == 5 and line["steps_requested"] == 5
+    for k in ("metric", "unit", "n_gpus", "warmup", "ms_per_step", "scaling", "dtype", "data", "config"):
+        assert k in line, k
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
