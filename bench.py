@@ -622,10 +622,21 @@ def run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_a
 
 
 def cpu_baseline(args, shape, x, logits_h, t_host):
+    """The oracle's time for one step of this workload (bounded sample) on the
+    host cores, with numpy's BLAS on all its threads and again on one."""
     import oracle
     tree = oracle.build_tree(x.logp, x.tok, x.root_tok, x.cache_len, shape.N)
     sec, picked, total, _, _ = oracle_step_time(shape, x, logits_h, tree, args.ref_nodes)
+    one = None
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1, user_api="blas"):
+            sec1, _, _, _, _ = oracle_step_time(shape, x, logits_h, tree, args.ref_nodes)
+        one = total / sec1
+    except Exception:  # no BLAS thread control here: report the all-threads figure only
+        one = None
     return {"value": total / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "value_1thread": one,
             "sample": f"one step: full build, attention on {picked} of {total} nodes (all heads) scaled by "
                       f"{total}/{picked}, full accept + compaction"}
 

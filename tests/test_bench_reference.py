@@ -37,3 +37,17 @@ def test_reference_line_on_the_tiny_workload():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_cpu_baseline_reports_all_threads_and_one():
+    import argparse
+
+    import oracle
+    from ddtree_speculative_decode_b200 import synth
+    shape = synth.tiny_f32()
+    x = synth.make_step(shape)
+    tree = oracle.build_tree(x.logp, x.tok, x.root_tok, x.cache_len, shape.N)
+    logits = synth.target_logits(shape, tree["parent"], tree["node_tok"], tree["n_nodes"])
+    cb = bench.cpu_baseline(argparse.Namespace(ref_nodes=8), shape, x, logits, None)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
+    assert cb["value_1thread"] is None or cb["value_1thread"] > 0
