@@ -194,6 +194,10 @@ DDT_API int ddt_build_tree(const float* logp, const int32_t* tok, const int32_t*
  *   (except after a timeout: zero the whole workspace then). The rest holds
  *   per-split partial results; its contents do not matter. Calls that share
  *   a workspace must not overlap in time.
+ * Preconditions: cache_off[b] + cache_len[b] + n_nodes[b] <= kv_rows,
+ *   cache_len[b] <= max_cache_len, n_nodes[b] <= N, none negative. The bf16
+ *   kernel reads the pool through TMA, which returns zeros for rows beyond
+ *   kv_rows. The f32 kernel does not check these bounds.
  * Errors: DDT_ERR_INVALID_ARG (nulls, sizes, workspace too small or
  *   misaligned, kv / q not 16-byte aligned for bf16), DDT_ERR_UNSUPPORTED.
  */
@@ -244,10 +248,14 @@ DDT_API int ddt_verify_attn(const void* q, const void* kv, int64_t kv_rows, cons
  *   2 s); if one expires the status word holds DDT_ERR_TIMEOUT and the
  *   outputs are not valid (zero the workspace before reusing it). Calls that
  *   share a workspace must not overlap on the GPU.
- * Runs as two kernels: the logits stream through shared memory by bulk
- *   copies on at most one CTA per SM (row maxima by 64-bit atomic max), then
- *   one CTA per request finds each node's accepted child, walks the path and
- *   compacts the rows.
+ * Preconditions the library cannot check (it is not told the pool's size):
+ *   every row the compaction touches, l*layer_stride_rows + cache_off[b] +
+ *   [cache_len[b], cache_len[b] + n_nodes[b]), lies inside the kv pool, and
+ *   the layers and requests own disjoint rows. The kernels do not check them.
+ * Runs as two kernels: the logits stream once with 16-byte loads, each warp
+ *   owning contiguous 2048-entry slices of the rows (two 512-thread CTAs per
+ *   SM; row maxima published by 64-bit atomic max), then one CTA per request
+ *   finds each node's accepted child, walks the path and compacts the rows.
  */
 DDT_API size_t ddt_accept_compact_workspace_size(int B, int N, int V);
 
