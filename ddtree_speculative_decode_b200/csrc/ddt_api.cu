@@ -39,6 +39,8 @@ int ddt_drafter_topk(const void* logits, int logits_dtype, int V, int R, int K, 
   if (!logits || !logp || !tok) return DDT_ERR_INVALID_ARG;
   if (R < 1 || V < 1 || K < 1 || K > 32 || K > V) return DDT_ERR_INVALID_ARG;
   if (logits_dtype != DDT_F32 && logits_dtype != DDT_BF16) return DDT_ERR_INVALID_ARG;
+  // up to 8 CTAs per row in a one-dimensional grid; slice bounds stay in int
+  if (R > (1 << 28) - 1 || V > (1 << 30)) return DDT_ERR_UNSUPPORTED;
   ddt::DrafterParams p{};
   p.logits = logits;
   p.logits_dtype = logits_dtype;

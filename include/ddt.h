@@ -102,10 +102,12 @@ DDT_API int ddt_version(void);
  * Outputs (device): logp [R][K] float32, tok [R][K] int32; dev_status [R]
  *   (nullable): DDT_OK, or DDT_ERR_INPUT for a row holding a non-finite
  *   logit (that row's tok = -1, logp = -inf).
- * Sizes: R >= 1, V >= 1, 1 <= K <= min(V, 32).
+ * Sizes: R >= 1, V >= 1, 1 <= K <= min(V, 32); R < 2^28 and V <= 2^30
+ *   (DDT_ERR_UNSUPPORTED beyond).
  * A row is split over a cluster of min(8, ceil(V / 16384)) CTAs (one CTA
  *   per row where such a cluster cannot be scheduled); no workspace. Errors:
- *   DDT_ERR_INVALID_ARG (nulls, sizes, dtype), DDT_ERR_CUDA (launch).
+ *   DDT_ERR_INVALID_ARG (nulls, sizes, dtype), DDT_ERR_UNSUPPORTED (sizes
+ *   above), DDT_ERR_CUDA (launch).
  */
 DDT_API int ddt_drafter_topk(const void* logits, int logits_dtype, int V, int R, int K, float* logp,
                              int32_t* tok, int32_t* dev_status, cudaStream_t stream);

@@ -101,3 +101,6 @@ def test_drafter_topk_host_validation(so):
     assert so.ddt_drafter_topk(p, 1, 100, 4, 0, p, p, None, None) == lib.DDT_ERR_INVALID_ARG
     assert so.ddt_drafter_topk(p, 7, 100, 4, 8, p, p, None, None) == lib.DDT_ERR_INVALID_ARG
     assert so.ddt_drafter_topk(p, 1, 100, 0, 8, p, p, None, None) == lib.DDT_ERR_INVALID_ARG
+    # grid and slice arithmetic bounds
+    assert so.ddt_drafter_topk(p, 1, 100, 1 << 28, 8, p, p, None, None) == lib.DDT_ERR_UNSUPPORTED
+    assert so.ddt_drafter_topk(p, 1, (1 << 30) + 1, 4, 8, p, p, None, None) == lib.DDT_ERR_UNSUPPORTED
