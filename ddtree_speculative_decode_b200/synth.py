@@ -303,6 +303,37 @@ def lmhead_inputs(shape: Shape, parent: np.ndarray, node_tok: np.ndarray, n_node
     return hidden, w, planted
 
 
+def tiny_mla_weights(seed: int = 1234, V: int = 400, d_model: int = 64, n_layers: int = 6, H: int = 4,
+                     d_nope: int = 8, d_rope: int = 16, d_latent: int = 64, d_v: int = 16, d_ff: int = 256) -> dict:
+    """Random weights of a tiny MLA decoder with the pages' tiny-model sizes
+    (hidden 64, 6 layers, vocabulary 400; "the_validation_pivot", section
+    "Assumptions Embedded in This Message") and the tiny attention shape (4
+    heads, latent 64 + rope 16, scale 1/sqrt(8 + 16)). Every matrix is
+    N(0, 1 / fan_in) in float32; the embedding is N(0, 1)."""
+    r = _rng(seed, 10)
+
+    def m(*shape):
+        return (r.standard_normal(shape) / math.sqrt(shape[-1])).astype(np.float32)
+
+    layers = []
+    for _ in range(n_layers):
+        layers.append({
+            "w_dkv": m(d_latent, d_model),       # latent c = w_dkv x
+            "w_kr": m(d_rope, d_model),          # shared rope key, before rotation
+            "w_q": m(H, d_nope, d_model),        # per-head no-rope query
+            "w_qr": m(H, d_rope, d_model),       # per-head rope query, before rotation
+            "w_uk": m(H, d_nope, d_latent),      # key up-projection (absorbed into the query)
+            "w_uv": m(H, d_v, d_latent),         # value up-projection (applied to the latent output)
+            "w_o": m(d_model, H * d_v),
+            "w_1": m(d_ff, d_model),
+            "w_2": m(d_model, d_ff),
+        })
+    return {"embed": r.standard_normal((V, d_model)).astype(np.float32), "layers": layers,
+            "w_vocab": m(V, d_model), "V": V, "d_model": d_model, "H": H, "d_nope": d_nope,
+            "d_rope": d_rope, "d_latent": d_latent, "d_v": d_v,
+            "scale": 1.0 / math.sqrt(d_nope + d_rope)}
+
+
 def oracle_drafter(golden: np.ndarray, D: int, K: int, sentinel_from: Optional[int] = None):
     """Drafter fixture that proposes a known continuation ("ddtree_speculative_
     decode_test_capstone", section "The Oracle Drafter" and "What the Test
