@@ -382,6 +382,11 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
     for k in range(n_stage):
         step(sets[k % n_sets], evs[k])
     torch.cuda.synchronize()
+    # accepted drafts per request (every step of the loop is the same step)
+    acc_len = acc["acc_len"].cpu().numpy().astype(np.int64)
+    accept_hist = np.bincount(acc_len, minlength=min(shape.D, shape.N - 1) + 1).tolist()
+    if args.dump and rank == 0:
+        dump_step(args.dump, shape, x, logits_h, tree, out, lse, acc, cl)
     dr = measure_drafter(args, shape, lib, dev, tdt)
     comp = None if args.sweep or args.layers < 2 else measure_compaction(
         args, shape, lib, dev, tdt, sets[0], tree, cl0, off, cap, acc, ws_acc)
@@ -418,6 +423,8 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
         "compaction_layers": None if comp is None else dict(
             comp, frac=comp["marginal_gbs"] / pk["hbm_gbs"], peak_gbs=pk["hbm_gbs"]),
         "nodes_per_step": n_nodes_total,
+        "accept_len_hist": accept_hist,
+        "tokens_per_step": int((acc_len + 1).sum()),
         "attn_gflop_per_step": flops / 1e9,
         "gpu_launches": launches_per_step * args.steps,
         "e2e": e2e,
@@ -440,6 +447,22 @@ def attn_launches(shape: synth.Shape) -> int:
 def _tdtype(shape):
     import torch
     return torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+
+
+def dump_step(path, shape, x, logits_h, tree, out, lse, acc, cl):
+    """Writes the step's host inputs and the library's outputs of the last
+    stage-pass step (stepio format) for replay elsewhere."""
+    from ddtree_speculative_decode_b200 import stepio
+    inputs = {"logp": x.logp, "tok": x.tok, "root_tok": x.root_tok, "cache_len": x.cache_len,
+              "cache_off": x.cache_off, "cache_cap": x.cache_cap, "q": x.q, "kv": x.kv, "logits": logits_h}
+    outputs = {k: v.cpu().numpy() for k, v in tree.items()}
+    outputs.update({f"acc_{k}": v.cpu().numpy() for k, v in acc.items()})
+    outputs["attn_out"] = out.float().cpu().numpy()
+    outputs["lse"] = lse.cpu().numpy()
+    outputs["cache_len_after"] = cl.cpu().numpy()
+    meta = {"workload": shape.name, "B": shape.B, "N": shape.N, "D": shape.D, "K": shape.K, "H": shape.H,
+            "d_latent": shape.d_l, "d_rope": shape.d_r, "V": shape.V, "dtype": shape.dtype, "scale": shape.scale}
+    stepio.save_step(path, inputs, outputs, meta)
 
 
 def measure_compaction(args, shape, lib, dev, tdt, s, tree, cl0, off, cap, acc, ws_acc):
@@ -655,6 +678,8 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=120.0,
                     help="wall seconds the reference arm's timed steps may take")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--dump", default=None,
+                    help="write one step's inputs and the library's outputs to this .npz (replayable)")
     ap.add_argument("--e2e-serial", action="store_true",
                     help="end-to-end leg: copy each step's inputs on the compute stream (no overlap)")
     ap.add_argument("--sweep", default=None,
