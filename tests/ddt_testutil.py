@@ -1,5 +1,6 @@
-"""Helpers shared by the GPU parity tests: host arrays -> device tensors,
-guard-banded output buffers, and the tolerance checks the parity bar uses."""
+"""Helpers shared by the tests: host arrays -> device tensors, guard-banded
+output buffers, the tolerance checks the parity bar uses, and the drafters of
+the speculative-loop tests."""
 import numpy as np
 import torch
 
@@ -59,3 +60,32 @@ def assert_attn_close(got: np.ndarray, ref: np.ndarray, out_bf16: bool, what="")
             assert err <= TOL_BF16_REL * max(scale, 1e-30), f"{what} request {b}: max err {err} vs scale {scale}"
         else:
             assert err <= TOL_F32_ABS, f"{what} request {b}: max abs err {err}"
+
+
+def golden_drafter(golden, V, p_hit=1.0, seed=0):
+    """Per-depth top-K proposals from a golden continuation (for the
+    speculative-loop tests): rank 0 is the golden token with probability
+    p_hit; otherwise the golden token sits at a lower rank or is missing.
+    Distractors are other in-vocabulary tokens; log-probs are strictly
+    decreasing and <= 0. Returns draft(committed, D, K) -> (logp, tok)."""
+    rng = np.random.default_rng(seed)
+
+    def draft(committed, D, K):
+        lp = np.zeros((D, K), np.float32)
+        tk = np.zeros((D, K), np.int32)
+        for d in range(D):
+            g = int(golden[len(committed) + d])
+            others = [t for t in rng.permutation(V)[:K + 1] if t != g][:K]
+            r = rng.random()
+            if r < p_hit:
+                row = [g] + others[:K - 1]
+            elif r < p_hit + (1 - p_hit) / 2 and K > 1:
+                pos = int(rng.integers(1, K))
+                row = others[:pos] + [g] + others[pos:K - 1]
+            else:
+                row = others[:K]
+            tk[d] = row
+            lp[d] = -np.arange(K, dtype=np.float32) * 0.75 - (0.0 if r < p_hit else 0.5)
+        return lp, tk
+
+    return draft

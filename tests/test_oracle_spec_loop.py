@@ -11,6 +11,7 @@ import pytest
 
 from oracle import spec_loop
 from ddtree_speculative_decode_b200 import synth
+from ddt_testutil import golden_drafter as _drafter
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "capstone_ddtree_stats.txt")
 PROMPT = [3, 14, 15, 92, 65]
@@ -29,34 +30,6 @@ def _golden():
 @pytest.fixture(scope="module")
 def model():
     return synth.tiny_mla_weights()
-
-
-def _drafter(golden, V, p_hit=1.0, seed=0):
-    """Per-depth top-K proposals from the golden continuation: rank 0 is the
-    golden token with probability p_hit; otherwise the golden token sits at a
-    lower rank or is missing. Distractors are other in-vocabulary tokens;
-    log-probs are strictly decreasing and <= 0."""
-    rng = np.random.default_rng(seed)
-
-    def draft(committed, D, K):
-        lp = np.zeros((D, K), np.float32)
-        tk = np.zeros((D, K), np.int32)
-        for d in range(D):
-            g = int(golden[len(committed) + d])
-            others = [t for t in rng.permutation(V)[:K + 1] if t != g][:K]
-            r = rng.random()
-            if r < p_hit:
-                row = [g] + others[:K - 1]
-            elif r < p_hit + (1 - p_hit) / 2 and K > 1:
-                pos = int(rng.integers(1, K))
-                row = others[:pos] + [g] + others[pos:K - 1]
-            else:
-                row = others[:K]
-            tk[d] = row
-            lp[d] = -np.arange(K, dtype=np.float32) * 0.75 - (0.0 if r < p_hit else 0.5)
-        return lp, tk
-
-    return draft
 
 
 def test_oracle_drafter_reproduces_the_pages_statistics(model):
@@ -113,3 +86,13 @@ def test_other_block_sizes(model, blk, K):
     ar, _ = spec_loop.ar_generate(model, PROMPT, T + blk)
     dd, steps, _ = spec_loop.ddtree_generate(model, PROMPT, T, _drafter(ar, model["V"], 0.8, blk), blk, K)
     assert dd[:T] == ar[:T]
+
+
+def test_the_gpu_engine_has_no_cpu_path(model):
+    import torch
+
+    from ddtree_speculative_decode_b200 import spec_engine
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(RuntimeError):
+        spec_engine.TinyMLAEngine(model, capacity=64)

@@ -5,7 +5,7 @@ ddt_accept_compact_noalloc serves callers that cannot allocate device memory
 where they verify a tree (they are handed fixed buffers, or must not risk the
 device-wide synchronisation cudaMalloc can cause); its scratch is a fixed
 array inside the library. This file runs last (pytest collects it after the
-other tests), so a failure here never hides the other results. Two calls in a
+other parity tests), so a failure here never hides their results. Two calls in a
 row check that the shared array's leftovers from the previous call do not
 leak into the next one."""
 import numpy as np
