@@ -8,6 +8,7 @@ call raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from typing import Optional
@@ -114,6 +115,30 @@ def _check(t: torch.Tensor, name: str, dtype, shape=None):
         raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
+def _device(*tensors, stream=None):
+    """A context that makes the one CUDA device every tensor of a call lives
+    on (and the explicit stream, if any, belongs to) current for the launch;
+    nothing is switched when it is current already (as inside a graph
+    capture on that device)."""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"tensors of one call must share a CUDA device, got {sorted(map(str, devs))}")
+    dev = devs.pop()
+    if stream is not None and stream.device != dev:
+        raise ValueError(f"stream on {stream.device}, tensors on {dev}")
+    if dev.index is None or dev.index == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(dev)
+
+
+def _check_out(out: dict, spec: dict):
+    """Caller-supplied output tensors: name -> (dtype, shape)."""
+    for name, (dtype, shape) in spec.items():
+        if name not in out:
+            raise ValueError(f"out: missing {name}")
+        _check(out[name], f"out[{name}]", dtype, shape)
+
+
 def _dt(t: torch.Tensor) -> int:
     if t.dtype == torch.float32:
         return DDT_F32
@@ -145,8 +170,11 @@ def drafter_topk(logits: torch.Tensor, K: int, out: Optional[dict] = None, strea
         out = {"logp": torch.empty(*lead, K, dtype=torch.float32, device=dev),
                "tok": torch.empty(*lead, K, dtype=torch.int32, device=dev),
                "status": torch.empty(*lead, dtype=torch.int32, device=dev)}
-    st = load().ddt_drafter_topk(_ptr(logits), _dt(logits), V, R, K, _ptr(out["logp"]), _ptr(out["tok"]),
-                                 _ptr(out["status"]), _stream(stream))
+    _check_out(out, {"logp": (torch.float32, lead + (K,)), "tok": (torch.int32, lead + (K,)),
+                     "status": (torch.int32, lead)})
+    with _device(logits, *out.values(), stream=stream):
+        st = load().ddt_drafter_topk(_ptr(logits), _dt(logits), V, R, K, _ptr(out["logp"]), _ptr(out["tok"]),
+                                     _ptr(out["status"]), _stream(stream))
     _raise("ddt_drafter_topk", st)
     return out
 
@@ -165,10 +193,15 @@ def build_tree(logp: torch.Tensor, tok: torch.Tensor, root_tok: torch.Tensor, ca
     W = (N + 31) // 32
     if out is None:
         out = alloc_tree(B, N, dev)
-    st = load().ddt_build_tree(_ptr(logp), _ptr(tok), _ptr(root_tok), _ptr(cache_len), B, D, K, N,
-                               _ptr(out["node_tok"]), _ptr(out["parent"]), _ptr(out["depth"]), _ptr(out["pos"]),
-                               _ptr(out["score"]), _ptr(out["mask"]), _ptr(out["n_nodes"]),
-                               _ptr(out["status"]), _stream(stream))
+    i32 = torch.int32
+    _check_out(out, {"node_tok": (i32, (B, N)), "parent": (i32, (B, N)), "depth": (i32, (B, N)),
+                     "pos": (i32, (B, N)), "score": (torch.float32, (B, N)), "mask": (i32, (B, N, W)),
+                     "n_nodes": (i32, (B,)), "status": (i32, (B,))})
+    with _device(logp, tok, root_tok, cache_len, *out.values(), stream=stream):
+        st = load().ddt_build_tree(_ptr(logp), _ptr(tok), _ptr(root_tok), _ptr(cache_len), B, D, K, N,
+                                   _ptr(out["node_tok"]), _ptr(out["parent"]), _ptr(out["depth"]),
+                                   _ptr(out["pos"]), _ptr(out["score"]), _ptr(out["mask"]), _ptr(out["n_nodes"]),
+                                   _ptr(out["status"]), _stream(stream))
     _raise("ddt_build_tree", st)
     return out
 
@@ -227,9 +260,10 @@ def verify_attn(q: torch.Tensor, kv: torch.Tensor, cache_off: torch.Tensor, cach
     if workspace is None and need > 0:
         workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)  # status word must start at 0
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = load().ddt_verify_attn(_ptr(q), _ptr(kv), kv.shape[0], _ptr(cache_off), _ptr(cache_len), _ptr(mask),
-                                _ptr(n_nodes), B, N, H, d_l, d_r, float(scale), int(max_cache_len), _dt(q),
-                                _dt(out), _ptr(out), _ptr(lse), _ptr(workspace), wbytes, _stream(stream))
+    with _device(q, kv, cache_off, cache_len, mask, n_nodes, out, lse, workspace, stream=stream):
+        st = load().ddt_verify_attn(_ptr(q), _ptr(kv), kv.shape[0], _ptr(cache_off), _ptr(cache_len), _ptr(mask),
+                                    _ptr(n_nodes), B, N, H, d_l, d_r, float(scale), int(max_cache_len), _dt(q),
+                                    _dt(out), _ptr(out), _ptr(lse), _ptr(workspace), wbytes, _stream(stream))
     _raise("ddt_verify_attn", st)
     return out, lse
 
@@ -257,18 +291,28 @@ def accept_compact(logits: torch.Tensor, node_tok: torch.Tensor, parent: torch.T
     dev = logits.device
     if out is None:
         out = alloc_accept(B, N, dev)
+    _check_out(out, _accept_out_spec(B, N))
     need = accept_compact_workspace_size(B, N, V)
     if workspace is None:
         workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)  # arrival counters start at 0
+    _check(workspace, "workspace", None)
     row_elems = kv.shape[-1]
-    st = load().ddt_accept_compact(_ptr(logits), _dt(logits), V, _ptr(node_tok), _ptr(parent), _ptr(n_nodes), B, N,
-                                   _ptr(kv), _dt(kv), row_elems, n_layers, layer_stride_rows, _ptr(cache_off),
-                                   _ptr(cache_len), _ptr(cache_cap), _ptr(out["am"]), _ptr(out["acc_len"]),
-                                   _ptr(out["acc_nodes"]), _ptr(out["out_tok"]), _ptr(out["bonus"]),
-                                   _ptr(out["status"]), _ptr(workspace),
-                                   workspace.numel() * workspace.element_size(), _stream(stream))
+    with _device(logits, node_tok, parent, n_nodes, kv, cache_off, cache_len, cache_cap,
+                 workspace, *out.values(), stream=stream):
+        st = load().ddt_accept_compact(_ptr(logits), _dt(logits), V, _ptr(node_tok), _ptr(parent), _ptr(n_nodes),
+                                       B, N, _ptr(kv), _dt(kv), row_elems, n_layers, layer_stride_rows,
+                                       _ptr(cache_off), _ptr(cache_len), _ptr(cache_cap), _ptr(out["am"]),
+                                       _ptr(out["acc_len"]), _ptr(out["acc_nodes"]), _ptr(out["out_tok"]),
+                                       _ptr(out["bonus"]), _ptr(out["status"]), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream))
     _raise("ddt_accept_compact", st)
     return out
+
+
+def _accept_out_spec(B: int, N: int) -> dict:
+    i32 = torch.int32
+    return {"am": (i32, (B, N)), "acc_len": (i32, (B,)), "acc_nodes": (i32, (B, N)), "out_tok": (i32, (B, N)),
+            "bonus": (i32, (B,)), "status": (i32, (B,))}
 
 
 def alloc_accept(B: int, N: int, device) -> dict:
@@ -296,10 +340,14 @@ def accept_compact_noalloc(logits: torch.Tensor, node_tok: torch.Tensor, parent:
     _check(cache_cap, "cache_cap", torch.int32, (B,))
     if out is None:
         out = alloc_accept(B, N, logits.device)
-    st = load().ddt_accept_compact_noalloc(_ptr(logits), _dt(logits), V, _ptr(node_tok), _ptr(parent), _ptr(n_nodes),
-                                           B, N, _ptr(kv), _dt(kv), kv.shape[-1], n_layers, layer_stride_rows,
-                                           _ptr(cache_off), _ptr(cache_len), _ptr(cache_cap), _ptr(out["am"]),
-                                           _ptr(out["acc_len"]), _ptr(out["acc_nodes"]), _ptr(out["out_tok"]),
-                                           _ptr(out["bonus"]), _ptr(out["status"]), _stream(stream))
+    _check_out(out, _accept_out_spec(B, N))
+    with _device(logits, node_tok, parent, n_nodes, kv, cache_off, cache_len, cache_cap,
+                 *out.values(), stream=stream):
+        st = load().ddt_accept_compact_noalloc(_ptr(logits), _dt(logits), V, _ptr(node_tok), _ptr(parent),
+                                               _ptr(n_nodes), B, N, _ptr(kv), _dt(kv), kv.shape[-1], n_layers,
+                                               layer_stride_rows, _ptr(cache_off), _ptr(cache_len),
+                                               _ptr(cache_cap), _ptr(out["am"]), _ptr(out["acc_len"]),
+                                               _ptr(out["acc_nodes"]), _ptr(out["out_tok"]), _ptr(out["bonus"]),
+                                               _ptr(out["status"]), _stream(stream))
     _raise("ddt_accept_compact_noalloc", st)
     return out

@@ -104,3 +104,21 @@ def test_drafter_topk_host_validation(so):
     # grid and slice arithmetic bounds
     assert so.ddt_drafter_topk(p, 1, 100, 1 << 28, 8, p, p, None, None) == lib.DDT_ERR_UNSUPPORTED
     assert so.ddt_drafter_topk(p, 1, (1 << 30) + 1, 4, 8, p, p, None, None) == lib.DDT_ERR_UNSUPPORTED
+
+
+def test_one_device_per_call():
+    import torch
+    a = torch.zeros(2)
+    b = torch.zeros(2, device="meta")
+    with lib._device(a, a, None):  # one device (and None skipped): nothing to switch
+        pass
+    with pytest.raises(ValueError):
+        lib._device(a, b)
+
+
+def test_supplied_outputs_are_checked():
+    import torch
+    with pytest.raises((TypeError, ValueError)):
+        lib._check_out({"status": torch.zeros(3, dtype=torch.int32)}, {"status": (torch.int32, (3,))})  # not CUDA
+    with pytest.raises(ValueError):
+        lib._check_out({}, {"status": (torch.int32, (3,))})  # missing
