@@ -16,6 +16,7 @@ the max-over-ranks of the elapsed time.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -246,7 +247,8 @@ def run_reference(args, shape: synth.Shape, rank: int):
 
 
 def config_dict(shape: synth.Shape, extra=None):
-    d = {"workload": shape.name, "B": shape.B, "N": shape.N, "D": shape.D, "K": shape.K, "H": shape.H,
+    d = {"workload": shape.name, "seed": shape.seed, "B": shape.B, "N": shape.N, "D": shape.D, "K": shape.K,
+         "H": shape.H,
          "d_latent": shape.d_l, "d_rope": shape.d_r, "V": shape.V, "cache_len": list(shape.L)[:4] +
          (["..."] if len(shape.L) > 4 else []), "in_dtype": shape.dtype}
     if extra:
@@ -670,6 +672,9 @@ def main():
     ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--config", default="kimi-1req", choices=sorted(synth.NAMED))
+    ap.add_argument("--seed", type=int, default=None,
+                    help="seed of the step's draws (drafter output, cache, queries, logits) instead of the "
+                         "workload's own; the workload's cache lengths stay as defined")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--layers", type=int, default=61,
@@ -690,7 +695,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    shape = synth.NAMED[args.config]()
+    def seeded(sh):
+        return sh if args.seed is None else dataclasses.replace(sh, seed=args.seed)
+
+    shape = seeded(synth.NAMED[args.config]())
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -708,7 +716,7 @@ def main():
             pts = SWEEP_POINTS if args.sweep == "default" else [tuple(int(v) for v in p.split(":"))
                                                                  for p in args.sweep.split(",")]
             for (b, n, l) in pts:
-                run_ours(args, synth.kimi_sweep(b, n, l), rank, world, local_rank)
+                run_ours(args, seeded(synth.kimi_sweep(b, n, l)), rank, world, local_rank)
                 torch.cuda.empty_cache()
         else:
             run_ours(args, shape, rank, world, local_rank)

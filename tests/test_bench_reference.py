@@ -51,3 +51,15 @@ def test_cpu_baseline_reports_all_threads_and_one():
     cb = bench.cpu_baseline(argparse.Namespace(ref_nodes=8), shape, x, logits, None)
     assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
     assert cb["value_1thread"] is None or cb["value_1thread"] > 0
+
+
+def test_seed_flag_changes_the_draws():
+    def run(*extra):
+        out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config",
+                              "tiny-f32", "--steps", "2", "--warmup", "3", "--ref-budget", "10", *extra],
+                             capture_output=True, text=True, timeout=600, cwd=ROOT)
+        assert out.returncode == 0, out.stderr
+        return json.loads(out.stdout.strip().splitlines()[-1])
+    default, seeded = run(), run("--seed", "77")
+    assert seeded["config"]["seed"] == 77 and default["config"]["seed"] != 77
+    assert seeded["config"]["cache_len"] == default["config"]["cache_len"]
