@@ -63,3 +63,21 @@ def test_seed_flag_changes_the_draws():
     default, seeded = run(), run("--seed", "77")
     assert seeded["config"]["seed"] == 77 and default["config"]["seed"] != 77
     assert seeded["config"]["cache_len"] == default["config"]["cache_len"]
+
+
+def test_two_ranks_under_torchrun_print_one_line():
+    """--impl reference under torchrun: rank 0 alone runs and prints; the other
+    rank exits 0 without work."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    out = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                          "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+                          "--impl", "reference", "--gpus", "2", "--config", "tiny-f32", "--steps", "2", "--warmup",
+                          "3", "--ref-budget", "10"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
