@@ -14,13 +14,18 @@ input here is synthetic:
 
 * drafter: per depth, logits ~ N(0, sigma) over the vocab, log_softmax in
   float64 rounded to float32, top-k by value (ties to the lower id), sorted
-  descending;
+  descending. This stands in for a drafter and produces the tree build's
+  inputs; it is the workload's recipe, not a side of any parity check (the
+  drafter-proposal kernel is checked on raw logits against the oracle's own
+  drafter_topk, which shares nothing with this function);
 * latent KV rows and queries ~ N(0, 1), KV optionally scaled (0.1 on the
   Kimi-shaped workloads), rounded to the storage dtype (bf16 round-to-nearest-
   even, or float32);
 * target logits ~ N(0, 1); for each tree node in index order a uniform draw u,
   and if u < p and the node has children, +bias on the token of one child
-  chosen uniformly (so accepted paths are non-contiguous in node index).
+  chosen uniformly (so accepted paths are non-contiguous in node index);
+* the target's LM-head inputs and a tiny decoder's random weights, for the
+  steps around the path (lmhead_inputs, tiny_mla_weights).
 
 ``N(0, s)`` is read as standard deviation ``s``.
 """
