@@ -151,3 +151,57 @@ def test_precondition_violation(bad):
     t = build_tree(lp, np.zeros((1, 2, 2), np.int32), np.array([1]), np.array([2]), 4)
     assert t["status"][0] == ERR_INPUT and t["n_nodes"][0] == 0
     assert np.all(t["node_tok"][0] == -1) and np.all(t["mask"][0] == 0)
+
+
+def _key(score, ranks):
+    # the build's total order: score descending, depth ascending, ranks lexicographic
+    return (-float(score), len(ranks), tuple(ranks))
+
+
+@pytest.mark.parametrize("D,K,N,quant", [(64, 32, 1024, None), (64, 32, 1024, 0.5), (8, 8, 64, 0.25),
+                                         (16, 8, 128, None), (6, 6, 32, 0.5), (3, 32, 700, 0.5),
+                                         (64, 1, 1024, None), (64, 2, 1024, 0.5), (12, 16, 256, 1.0)])
+def test_build_is_the_best_prefix_closed_set_at_full_sizes(D, K, N, quant):
+    """Where enumerating K^D paths is out of reach: the tree is prefix-closed,
+    its scores are the left-to-right float32 sums, its nodes come in the
+    order's sequence, and every unselected child of a selected path orders
+    after the last selected one. Since log-probs are <= 0, any unselected
+    path orders no earlier than its first unselected prefix, which is such a
+    child; so the tree holds exactly the N - 1 best paths."""
+    rng = np.random.default_rng(D * 1000 + K * 10 + N)
+    logp = _sorted_logp(rng, D, K, quant)
+    tok = np.stack([rng.permutation(50000)[:K] for _ in range(D)]).astype(np.int32)
+    t = build_tree(logp[None], tok[None], np.array([7]), np.array([100]), N)
+    n = int(t["n_nodes"][0])
+    total = sum(K ** d for d in range(1, D + 1))  # exact integers
+    assert n - 1 == min(N - 1, total)
+    rank_of = [{int(tok[d, r]): r for r in range(K)} for d in range(D)]
+    ranks = [()]
+    score = [np.float32(0.0)]
+    for i in range(1, n):
+        p = int(t["parent"][0, i])
+        d = int(t["depth"][0, i])
+        assert 0 <= p < i and d == len(ranks[p]) + 1 and d <= D
+        r = rank_of[d - 1][int(t["node_tok"][0, i])]
+        ranks.append(ranks[p] + (r,))
+        score.append(np.float32(score[p] + logp[d - 1, r]))
+        assert np.float32(t["score"][0, i]).view(np.uint32) == score[i].view(np.uint32)
+        assert int(t["pos"][0, i]) == 100 + d
+    keys = [_key(score[i], ranks[i]) for i in range(1, n)]
+    assert all(a < b for a, b in zip(keys, keys[1:]))
+    chosen = set(ranks)
+    last = keys[-1] if keys else None
+    for i in range(n):
+        if len(ranks[i]) == D:
+            continue
+        for r in range(K):
+            c = ranks[i] + (r,)
+            if c not in chosen:
+                s = np.float32(score[i] + logp[len(ranks[i]), r])
+                assert _key(s, c) > last, (c, last)
+    # masks: ancestors by the prefix relation
+    idx = {rk: i for i, rk in enumerate(ranks)}
+    for i in range(n):
+        want = {idx[ranks[i][:j]] for j in range(len(ranks[i]) + 1)}
+        got = {j for j in range(n) if (int(t["mask"][0, i, j >> 5]) >> (j & 31)) & 1}
+        assert got == want
