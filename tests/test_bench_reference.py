@@ -81,3 +81,33 @@ def test_two_ranks_under_torchrun_print_one_line():
     assert len(lines) == 1
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2
+
+
+def test_profiled_traffic_follows_the_captured_sources(tmp_path, monkeypatch):
+    """roofline.traffic comes from the ncu summary only while the captured
+    kernel sources are unchanged (the summary records their sha256), and only
+    for the captured workload."""
+    import hashlib
+
+    from ddtree_speculative_decode_b200 import synth
+    csrc = tmp_path / "ddtree_speculative_decode_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (csrc / "verify_attn_tc.cu").write_text("kernel A\n")
+    (csrc / "sm100_ptx.cuh").write_text("helpers B\n")
+
+    def sha(name):
+        return hashlib.sha256((csrc / name).read_bytes()).hexdigest()
+
+    (tmp_path / "profiles" / "attn_tc_kimi-1req.md").write_text(
+        "Source captured (sha256):\n\n"
+        f"    verify_attn_tc.cu {sha('verify_attn_tc.cu')}\n"
+        f"    sm100_ptx.cuh     {sha('sm100_ptx.cuh')}\n\n"
+        "| metric | value |\n|---|---|\n"
+        "| dram__bytes_read.sum | 9.5 MB |\n| dram__bytes_write.sum | 512 B |\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    shape = synth.kimi_1req()
+    assert bench.profiled_traffic(shape) == 9.5e6 + 512
+    assert bench.profiled_traffic(synth.NAMED["kimi-16req"]()) is None  # no capture of that workload
+    (csrc / "sm100_ptx.cuh").write_text("helpers B, changed\n")
+    assert bench.profiled_traffic(shape) is None
