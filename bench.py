@@ -646,24 +646,39 @@ def run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_a
             "h2d_gbs": h2d * steps / (ms / 1e3) / 1e9}
 
 
+def _oracle_steps(shape, x, logits_h, tree, nodes, seconds):
+    """Oracle step estimates (each with its own node sample) until `seconds`
+    of wall time have passed; returns (mean scaled step seconds, steps,
+    sampled nodes per step, all nodes)."""
+    t0 = time.perf_counter()
+    secs = []
+    picked = total = 0
+    while not secs or time.perf_counter() - t0 < seconds:
+        sec, picked, total, _, _ = oracle_step_time(shape, x, logits_h, tree, nodes, seed=len(secs))
+        secs.append(sec)
+    return float(np.mean(secs)), len(secs), picked, total
+
+
 def cpu_baseline(args, shape, x, logits_h, t_host):
-    """The oracle's time for one step of this workload (bounded sample) on the
-    host cores, with numpy's BLAS on all its threads and again on one."""
+    """The oracle's time for this workload's step on the host cores, from a
+    bounded sample (about args.cpu_seconds of wall time), with numpy's BLAS on
+    all its threads and again (for half as long) on one."""
     import oracle
     tree = oracle.build_tree(x.logp, x.tok, x.root_tok, x.cache_len, shape.N)
-    sec, picked, total, _, _ = oracle_step_time(shape, x, logits_h, tree, args.ref_nodes)
+    sec, steps, picked, total = _oracle_steps(shape, x, logits_h, tree, args.ref_nodes, args.cpu_seconds)
     one = None
     try:
         from threadpoolctl import threadpool_limits
         with threadpool_limits(limits=1, user_api="blas"):
-            sec1, _, _, _, _ = oracle_step_time(shape, x, logits_h, tree, args.ref_nodes)
+            sec1, _, _, _ = _oracle_steps(shape, x, logits_h, tree, args.ref_nodes, args.cpu_seconds / 2)
         one = total / sec1
     except Exception:  # no BLAS thread control here: report the all-threads figure only
         one = None
     return {"value": total / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "value_1thread": one,
-            "sample": f"one step: full build, attention on {picked} of {total} nodes (all heads) scaled by "
-                      f"{total}/{picked}, full accept + compaction"}
+            "sample": f"{steps} step estimates in about {args.cpu_seconds:.0f} s: each a full build, attention "
+                      f"on {picked} of {total} nodes (all heads, a new sample per step) scaled by {total}/{picked}, "
+                      f"full accept + compaction"}
 
 
 def main():
@@ -683,6 +698,8 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=120.0,
                     help="wall seconds the reference arm's timed steps may take")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="wall seconds of oracle work behind cpu_baseline (one-thread run: half)")
     ap.add_argument("--dump", default=None,
                     help="write one step's inputs and the library's outputs to this .npz (replayable)")
     ap.add_argument("--e2e-serial", action="store_true",

@@ -48,9 +48,10 @@ def test_cpu_baseline_reports_all_threads_and_one():
     x = synth.make_step(shape)
     tree = oracle.build_tree(x.logp, x.tok, x.root_tok, x.cache_len, shape.N)
     logits = synth.target_logits(shape, tree["parent"], tree["node_tok"], tree["n_nodes"])
-    cb = bench.cpu_baseline(argparse.Namespace(ref_nodes=8), shape, x, logits, None)
+    cb = bench.cpu_baseline(argparse.Namespace(ref_nodes=8, cpu_seconds=1.0), shape, x, logits, None)
     assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
     assert cb["value_1thread"] is None or cb["value_1thread"] > 0
+    assert int(cb["sample"].split()[0]) > 1  # many step estimates within the second
 
 
 def test_seed_flag_changes_the_draws():
