@@ -67,27 +67,28 @@ def replica_throughput(nodes_per_step: int, steps: int, world: int, elapsed_ms: 
     return nodes_per_step * world * steps / (elapsed_ms / 1e3)
 
 
-def profiled_traffic(shape: synth.Shape):
-    """DRAM bytes (read + write) of one verify-attention launch from the ncu
-    capture summarised in profiles/attn_tc_<workload>.md, or None when there is
-    no capture of this workload or the kernel sources changed since it was
-    taken (the summary records their sha256)."""
+# DRAM bytes (read + write) of one verify-attention launch, from one ncu
+# capture per workload (the capture command and figures are summarised under
+# profiles/), valid only while the kernel sources still have the sha256 they
+# had when captured.
+PROFILED_ATTN_DRAM = {}
+
+
+def profiled_traffic(shape: synth.Shape, table=None, root=None):
+    """roofline.traffic: the captured DRAM bytes of one verify-attention launch
+    of this workload, or None when there is no capture of it or the kernel
+    sources changed since (a stale count says nothing about the kernel as it
+    is)."""
     import hashlib
-    import re
-    tag = {"kimi-1req-L4096-N64": "kimi-1req"}.get(shape.name)
-    path = os.path.join(ROOT, "profiles", f"attn_tc_{tag}.md") if tag else None
-    if not path or not os.path.exists(path):
+    entry = (PROFILED_ATTN_DRAM if table is None else table).get(shape.name)
+    if entry is None:
         return None
-    text = open(path).read()
-    for fname, digest in re.findall(r"^\s+(\S+\.cuh?)\s+([0-9a-f]{64})\s*$", text, re.M):
-        src = os.path.join(ROOT, "ddtree_speculative_decode_b200", "csrc", fname)
-        if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != digest:
+    csrc = os.path.join(root or ROOT, "ddtree_speculative_decode_b200", "csrc")
+    for fname, digest in entry["sources"].items():
+        path = os.path.join(csrc, fname)
+        if not os.path.exists(path) or hashlib.sha256(open(path, "rb").read()).hexdigest() != digest:
             return None
-    rd = re.search(r"\| dram__bytes_read\.sum \| ([0-9.]+) MB \|", text)
-    wr = re.search(r"\| dram__bytes_write\.sum \| ([0-9.]+) (MB|B)", text)
-    if not rd or not wr:
-        return None
-    return float(rd.group(1)) * 1e6 + float(wr.group(1)) * (1e6 if wr.group(2) == "MB" else 1.0)
+    return float(entry["bytes"])
 
 
 def peaks():
@@ -173,70 +174,82 @@ def blas_threads() -> int:
 # ---------------------------------------------------------------------------
 
 
-def oracle_step_time(shape: synth.Shape, x, logits, tree, attn_nodes: int, seed: int = 0):
-    """Seconds the oracle needs for one full step of this workload, from a
-    bounded sample: the whole tree build, attention for `attn_nodes` sampled
-    nodes (all heads) scaled by the node count, the whole accept + compaction.
-    Returns (scaled step seconds, sampled nodes, all nodes, wall seconds of the
-    parts that do not scale with the sample, wall seconds per sampled node)."""
+def request_slice(x, logits, b):
+    """Request b of a step as a one-request step (its pool rows rebased to
+    row 0): the unit of work of the oracle timings."""
+    off, cap = int(x.cache_off[b]), int(x.cache_cap[b])
+    return {"logp": x.logp[b:b + 1], "tok": x.tok[b:b + 1], "root": x.root_tok[b:b + 1],
+            "L": x.cache_len[b:b + 1], "off": np.zeros(1, np.int64), "cap": x.cache_cap[b:b + 1],
+            "kv": x.kv[off:off + cap], "q": x.q[b:b + 1], "logits": logits[b:b + 1]}
+
+
+def oracle_request_step(shape: synth.Shape, r: dict, attn_nodes=None):
+    """Wall seconds of the oracle's whole step on one request: tree build,
+    attention (for the first `attn_nodes` nodes if given, else all of them,
+    every head), accept and compaction. Returns (seconds, attention seconds,
+    nodes attended, nodes of the request). The pool slice it compacts is a
+    copy made before the clock starts."""
     import oracle
 
+    kv = r["kv"].copy()
     t0 = time.perf_counter()
-    oracle.build_tree(x.logp, x.tok, x.root_tok, x.cache_len, shape.N)
-    t_build = time.perf_counter() - t0
-    rng = np.random.default_rng(seed)
-    all_rows = [(b, i) for b in range(shape.B) for i in range(int(tree["n_nodes"][b]))]
-    pick = [all_rows[j] for j in sorted(rng.choice(len(all_rows), size=min(attn_nodes, len(all_rows)),
-                                                   replace=False))]
-    t0 = time.perf_counter()
-    oracle.verify_attn(x.q, x.kv, x.cache_off, x.cache_len, tree["mask"], tree["n_nodes"], shape.H, shape.d_l,
-                       shape.d_r, shape.scale, shape.dtype, rows=pick)
-    t_attn = (time.perf_counter() - t0) * len(all_rows) / max(1, len(pick))
-    kv = x.kv.copy()
-    t0 = time.perf_counter()
-    oracle.accept_compact(logits, shape.dtype, tree["node_tok"], tree["parent"], tree["n_nodes"], kv, x.cache_off,
-                          x.cache_len, x.cache_cap)
-    t_acc = time.perf_counter() - t0
-    per_node = t_attn / max(1, len(all_rows))
-    return t_build + t_attn + t_acc, len(pick), len(all_rows), t_build + t_acc, per_node
+    tree = oracle.build_tree(r["logp"], r["tok"], r["root"], r["L"], shape.N)
+    n = int(tree["n_nodes"][0])
+    m = n if attn_nodes is None else max(1, min(n, int(attn_nodes)))
+    rows = None if m == n else [(0, i) for i in range(m)]
+    t1 = time.perf_counter()
+    oracle.verify_attn(r["q"], kv, r["off"], r["L"], tree["mask"], tree["n_nodes"], shape.H, shape.d_l, shape.d_r,
+                       shape.scale, shape.dtype, rows=rows)
+    t2 = time.perf_counter()
+    oracle.accept_compact(r["logits"], shape.dtype, tree["node_tok"], tree["parent"], tree["n_nodes"], kv, r["off"],
+                          r["L"], r["cap"])
+    t3 = time.perf_counter()
+    return t3 - t0, t2 - t1, m, n
 
 
 def reference_steps(steps: int, budget_s: float, step_wall_s: float) -> int:
     """How many of the requested steps the reference arm times: all of them if
-    they fit the wall-time budget, else as many as it holds (at least one).
-    The per-step sample stays fixed, so the value does not depend on K (a
-    smaller attention sample would scale the oracle's per-call setup up with
-    it)."""
+    they fit the wall-time budget, else as many as it holds (at least one)."""
     if step_wall_s <= 0:
         return steps
     return int(max(1, min(steps, budget_s // step_wall_s)))
 
 
-def run_reference(args, shape: synth.Shape, rank: int):
-    """--impl reference: the oracle as it stands, timed on the host cores."""
-    if rank != 0:
-        return
+def oracle_inputs(shape: synth.Shape):
+    """The workload's step drawn on the host and the oracle's tree and target
+    logits for it (inputs of the oracle timings; not timed)."""
     import oracle
 
     x = synth.make_step(shape)
     tree = oracle.build_tree(x.logp, x.tok, x.root_tok, x.cache_len, shape.N)
     logits = synth.target_logits(shape, tree["parent"], tree["node_tok"], tree["n_nodes"])
-    nodes = int(tree["n_nodes"].sum())
-    sample = max(1, min(nodes, args.ref_nodes))
+    return x, logits
+
+
+def run_reference(args, shape: synth.Shape, rank: int):
+    """--impl reference: the oracle as it stands, timed on the host cores.
+    A step is the oracle's whole step on one request of the workload
+    (requests in turn), nothing sampled or scaled: ms_per_step is what a step
+    took."""
+    if rank != 0:
+        return
+    x, logits = oracle_inputs(shape)
+    reqs = [request_slice(x, logits, b) for b in range(shape.B)]
     # one untimed step (whatever W is) also measures a step's wall time
-    _, _, _, fixed_s, per_node_s = oracle_step_time(shape, x, logits, tree, sample)
-    run = reference_steps(args.steps, args.ref_budget, fixed_s + sample * per_node_s)
-    times = []
+    t, _, _, _ = oracle_request_step(shape, reqs[0])
+    run = reference_steps(args.steps, args.ref_budget, t)
+    secs, nodes = [], 0
     for k in range(run):
-        t, _, _, _, _ = oracle_step_time(shape, x, logits, tree, sample, seed=k)
-        times.append(t)
-    sec = float(np.mean(times))
+        t, _, _, n = oracle_request_step(shape, reqs[k % shape.B])
+        secs.append(t)
+        nodes += n
+    sec = float(sum(secs))
     value = nodes / sec
-    desc = (f"per step: full tree build, attention on {sample} sampled nodes x {shape.H} heads scaled to "
-            f"{nodes} nodes, full accept + compaction; {run} of {args.steps} requested steps timed "
-            f"(wall-time budget {args.ref_budget:.0f} s)")
+    desc = (f"each step the oracle's whole step on one of the workload's {shape.B} requests in turn (tree build, "
+            f"attention on all its nodes and heads, accept + compaction), nothing sampled or scaled; {run} of "
+            f"{args.steps} requested steps timed (wall-time budget {args.ref_budget:.0f} s)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": run, "steps_requested": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+            "steps": run, "steps_requested": args.steps, "warmup": args.warmup, "ms_per_step": sec / run * 1e3,
             "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_dict(shape),
@@ -261,15 +274,16 @@ def config_dict(shape: synth.Shape, extra=None):
 # ---------------------------------------------------------------------------
 
 
-def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
+def measure_step(args, shape: synth.Shape, dev, world: int, full: bool):
+    """One workload on this GPU: the timed loop of K whole steps, the per-stage
+    kernel times and (when `full`) the drafter, compaction and end-to-end
+    legs. Returns a dict of results (and the host-side step for the CPU
+    baseline)."""
     import torch
     import torch.distributed as dist
 
     from ddtree_speculative_decode_b200 import lib
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    lib.load()
     bf = shape.dtype == "bf16"
     tdt = torch.bfloat16 if bf else torch.float32
 
@@ -304,8 +318,6 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
     cl = cl0.clone()
     stream = torch.cuda.current_stream(dev)
     n_nodes_total = int(t_host["n_nodes"].sum())
-    flops = attn_flops(shape, x.cache_len, t_host["depth"], t_host["n_nodes"])
-    acc_bytes = float(t_host["n_nodes"].sum()) * shape.V * (2 if bf else 4)
 
     def step(s, ev=None):
         st = torch.cuda.current_stream(dev)  # the capture stream while a graph is recorded
@@ -327,14 +339,6 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
             ev[3].record(st)
 
     # ---- warm-up ---------------------------------------------------------------
-    uuid = None
-    try:
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-        if not uuid.startswith("GPU-"):
-            uuid = "GPU-" + uuid
-    except Exception:
-        uuid = None
-    sampler = ClockSampler(uuid) if rank == 0 else ClockSampler(None)
     for w in range(args.warmup):
         step(sets[w % n_sets])
     torch.cuda.synchronize()
@@ -376,68 +380,257 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
     if world > 1:
         dist.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
-    clocks = sampler.stop()
-    # ---- per-stage breakdown (a separate pass: events between the kernels
-    # would cut their programmatic overlap inside the timed region) ----------------
-    n_stage = min(args.steps, 300)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_stage)]
-    for k in range(n_stage):
-        step(sets[k % n_sets], evs[k])
-    torch.cuda.synchronize()
-    # accepted drafts per request (every step of the loop is the same step)
-    acc_len = acc["acc_len"].cpu().numpy().astype(np.int64)
-    accept_hist = np.bincount(acc_len, minlength=min(shape.D, shape.N - 1) + 1).tolist()
-    if args.dump and rank == 0:
-        dump_step(args.dump, shape, x, logits_h, tree, out, lse, acc, cl)
-    dr = measure_drafter(args, shape, lib, dev, tdt)
-    comp = None if args.sweep or args.layers < 2 else measure_compaction(
-        args, shape, lib, dev, tdt, sets[0], tree, cl0, off, cap, acc, ws_acc)
+    # ---- per-stage kernel times: a separate pass (events between the kernels
+    # cut their programmatic overlap, so they stay out of the timed region),
+    # captured as one graph with event nodes between the stages so that the
+    # host's per-call cost never shows up as GPU time ------------------------------
+    n_stage = max(3, min(args.steps, 300))
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(n_stage)]
+    stage_pass = "one CUDA graph of the steps with timing-event nodes between the stages"
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for k in range(n_stage):
+                step(sets[k % n_sets], evs[k])
+        g.replay()
+        torch.cuda.synchronize()
+        del g
+    except Exception as e:  # no event nodes in graphs here: plain calls (host gaps included)
+        print(f"stage graph failed ({e}); timing stages with plain calls", file=sys.stderr)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_stage)]
+        for k in range(n_stage):
+            step(sets[k % n_sets], evs[k])
+        torch.cuda.synchronize()
+        stage_pass = "plain library calls with events between the stages"
     build_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     accept_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    elapsed_ms = max_over_ranks(elapsed_ms, dev)
-    value = replica_throughput(n_nodes_total, args.steps, world, elapsed_ms)
+    acc_len = acc["acc_len"].cpu().numpy().astype(np.int64)
+    res = {"shape": shape, "x": x, "logits_h": logits_h, "t_host": t_host, "n_sets": n_sets, "set_bytes": set_bytes,
+           "elapsed_ms": max_over_ranks(elapsed_ms, dev), "nodes": n_nodes_total,
+           "flops": attn_flops(shape, x.cache_len, t_host["depth"], t_host["n_nodes"]),
+           "acc_bytes": float(n_nodes_total) * shape.V * (2 if bf else 4),
+           "stages_ms": {"build_tree": build_ms, "verify_attn": attn_ms, "accept_compact": accept_ms},
+           "stage_pass": f"{stage_pass}, {n_stage} steps",
+           "acc_len": acc_len, "graphs": graphs is not None,
+           "split_keys": lib.verify_attn_workspace_size(B, N, H, shape.d_l, shape.d_r, maxL, tdt) > 256}
+    if full:
+        if args.dump:
+            dump_step(args.dump, shape, x, logits_h, tree, out, lse, acc, cl)
+        res["drafter"] = measure_drafter(args, shape, lib, dev, tdt)
+        res["compaction"] = None if args.layers < 2 else measure_compaction(
+            args, shape, lib, dev, tdt, sets[0], tree, cl0, off, cap, acc, ws_acc)
+        # ---- end to end through the public API with host buffers --------------------
+        res["e2e"] = run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_acc, out, lse, off,
+                             cap, maxL, world)
+        # ---- the same step with the target's LM head folded into the accept -------
+        if args.lmhead and shape.dtype == "bf16":
+            lm = measure_lmhead(args, shape, lib, dev, x, t_host,
+                                {"cl0": cl0, "cl": cl, "tree": tree, "off": off, "cap": cap, "ws_acc": ws_acc,
+                                 "acc": acc, "kv": sets[0]["kv"]})
+            w_head, hid = lm.pop("w"), lm.pop("hidden")
 
-    # ---- end to end through the public API with host buffers -------------------------
-    e2e = None if args.sweep else run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_acc, out,
-                                          lse, off, cap, maxL, world)
+            def step_lm(s):
+                st = torch.cuda.current_stream(dev)
+                torch.add(cl0, 0, out=cl)
+                lib.build_tree(logp, tok, root, cl, N, out=tree, stream=st)
+                lib.verify_attn(s["q"], s["kv"], off, cl, tree["mask"], tree["n_nodes"], shape.d_l, shape.d_r,
+                                shape.scale, maxL, out=out, lse=lse, workspace=ws_attn, stream=st)
+                lib.accept_compact_lmhead(hid, w_head, tree["node_tok"], tree["parent"], tree["n_nodes"], s["kv"],
+                                          off, cl, cap, out=acc, workspace=ws_acc, stream=st)
 
+            for k in range(3):
+                step_lm(sets[k % n_sets])
+            torch.cuda.synchronize()
+            n_lm = max(3, min(args.steps, 50))
+            gl = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gl):
+                for k in range(n_lm):
+                    step_lm(sets[k % n_sets])
+            gl.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            gl.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = max_over_ranks(e0.elapsed_time(e1), dev)
+            del gl
+            lm["step"] = {"value": replica_throughput(n_nodes_total, n_lm, world, ms), "unit": UNIT,
+                          "ms_per_step": ms / n_lm, "steps": n_lm,
+                          "what": "build -> verify attention -> accept with the LM head folded in (one graph)"}
+            lm["step"]["e2e"] = run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_acc, out,
+                                        lse, off, cap, maxL, world,
+                                        head={"w": w_head, "hidden_h": hid.cpu()})
+            res["lmhead"] = lm
+            del w_head, hid
+    del sets, graphs
+    return res
+
+
+def lmhead_width(shape: synth.Shape) -> int:
+    """Hidden size of the target whose head the fused accept folds in: Kimi
+    K2.6's 7168 for the Kimi-shaped workloads, the pages' tiny model's 64
+    otherwise."""
+    return 7168 if shape.V == 163840 else 64
+
+
+def measure_lmhead(args, shape, lib, dev, x, t_host, step_parts):
+    """The accept with the target's LM head folded in (ddt_accept_compact_lmhead)
+    on this workload's verify rows: a random-init bf16 head [V, d] and hidden
+    states drawn on the device (planted rows pushed toward a child's token as
+    the logits recipe biases them). Times the call alone (graph of calls after
+    a restore of cache_len), then the whole step with it in place of the
+    materialised-logits accept, then that step end to end with the hidden
+    states copied in each step."""
+    import torch
+    B, N, V = shape.B, shape.N, shape.V
+    d = lmhead_width(shape)
+    g = torch.Generator(device=dev)
+    g.manual_seed(shape.seed + 77)
+    w = (torch.randn(V, d, generator=g, device=dev) / math.sqrt(d)).to(torch.bfloat16)
+    hidden = torch.randn(B, N, d, generator=g, device=dev)
+    rng = np.random.default_rng(shape.seed + 78)
+    for b in range(B):
+        n = int(t_host["n_nodes"][b])
+        for i in range(n):
+            kids = np.flatnonzero(t_host["parent"][b, :n] == i)
+            if len(kids) and rng.random() < shape.accept_p:
+                t = int(t_host["node_tok"][b, int(kids[rng.integers(len(kids))])])
+                wt = w[t].float()
+                hidden[b, i] += shape.accept_bias * wt / (wt @ wt)
+    hidden = hidden.to(torch.bfloat16)
+    cl0, cl, tree, off, cap, ws_acc, acc, kv = (step_parts[k] for k in
+                                                 ("cl0", "cl", "tree", "off", "cap", "ws_acc", "acc", "kv"))
+    stream = torch.cuda.current_stream(dev)
+
+    def call(st):
+        torch.add(cl0, 0, out=cl)
+        lib.accept_compact_lmhead(hidden, w, tree["node_tok"], tree["parent"], tree["n_nodes"], kv, off, cl, cap,
+                                  out=acc, workspace=ws_acc, stream=st)
+
+    for _ in range(3):
+        call(stream)
+    torch.cuda.synchronize()
+    reps = max(3, min(50, int(0.2 / (2.0 * B * N * d * V / 1.0e15 + 1e-5))))
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for _ in range(reps):
+            call(torch.cuda.current_stream(dev))
+    gr.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    gr.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) / reps * 1e3
+    del gr
+    acc_len = acc["acc_len"].cpu().numpy().astype(np.int64)
+    return {"rows": B * N, "d_model": d, "V": V, "us": us, "flops": 2.0 * B * N * d * V,
+            "head_bytes": float(V * d * 2), "tokens_per_call": int((acc_len + 1).sum()),
+            "w": w, "hidden": hidden, "timing": f"graph of {reps} calls, each after a cache_len restore"}
+
+
+def stage_rooflines(res: dict, pk: dict) -> dict:
+    """Attention TFLOP/s and accept GB/s from the per-stage kernel times, as
+    fractions of the burst peaks (the stage pass is a short burst of work)."""
+    attn_ms = res["stages_ms"]["verify_attn"]
+    accept_ms = res["stages_ms"]["accept_compact"]
+    achieved = res["flops"] / (attn_ms / 1e3) / 1e12
+    gbs = res["acc_bytes"] / (accept_ms / 1e3) / 1e9
+    return {"attn_tflops": achieved, "attn_frac": achieved / pk["bf16_tflops"], "accept_gbs": gbs,
+            "accept_frac": gbs / pk["hbm_gbs"]}
+
+
+def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
+    import torch
+
+    from ddtree_speculative_decode_b200 import lib
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    lib.load()
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid) if rank == 0 else ClockSampler(None)
+    res = measure_step(args, shape, dev, world, full=not args.sweep)
+    clocks = sampler.stop()
+    extra = {}
+    if not args.sweep:
+        for name in [n for n in (args.extra or "").split(",") if n]:
+            sh = synth.NAMED[name]() if args.seed is None else dataclasses.replace(synth.NAMED[name](), seed=args.seed)
+            if sh.name == shape.name:
+                continue
+            r = measure_step(args, sh, dev, world, full=False)
+            extra[sh.name] = r
+            torch.cuda.empty_cache()
     if rank != 0:
         return
     pk = peaks()
-    achieved = flops / (attn_ms / 1e3) / 1e12
-    peak = pk["bf16_tflops_sustained"]
-    launches_per_step = 1 + attn_launches(shape) + 2  # build, attention, accept argmax + walk (cache_len memcpy excluded)
+    rf = stage_rooflines(res, pk)
+    value = replica_throughput(res["nodes"], args.steps, world, res["elapsed_ms"])
+    launches_per_step = 1 + attn_launches(shape) + 2  # build, attention, accept argmax + walk (cache_len restore excluded)
+    acc_len = res["acc_len"]
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": res["elapsed_ms"] / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic",
         "config": config_dict(shape, {"parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
-                                      "l2": f"{n_sets} rotating input sets of {set_bytes / 2**20:.1f} MiB "
-                                            f"(> 2x 126 MiB L2)"}),
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic(shape),
-                     "kernel": "ddt_verify_attn", "peak_kind": f"bf16 dense, sustained, {pk['source']}"},
-        "stages_ms": {"build_tree": build_ms, "verify_attn": attn_ms, "accept_compact": accept_ms},
-        "accept_hbm": {"achieved_gbs": acc_bytes / (accept_ms / 1e3) / 1e9, "peak_gbs": pk["hbm_gbs"],
-                       "frac": acc_bytes / (accept_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
-        "drafter_topk": dict(dr, frac=dr["gbs"] / pk["hbm_gbs"], peak_gbs=pk["hbm_gbs"]),
-        "compaction_layers": None if comp is None else dict(
-            comp, frac=comp["marginal_gbs"] / pk["hbm_gbs"], peak_gbs=pk["hbm_gbs"]),
-        "nodes_per_step": n_nodes_total,
-        "accept_len_hist": accept_hist,
+                                      "l2": f"{res['n_sets']} rotating input set(s) of {res['set_bytes'] / 2**20:.1f} "
+                                            f"MiB (each larger than the 126 MiB L2, or together > 2x L2)"}),
+        "roofline": {"bound": "tensor", "achieved": rf["attn_tflops"], "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": rf["attn_frac"], "traffic": profiled_traffic(shape),
+                     "kernel": "ddt_verify_attn",
+                     "achieved_from": f"algorithmic FLOPs {res['flops'] / 1e9:.1f} G per launch / mean launch time "
+                                      f"{res['stages_ms']['verify_attn'] * 1e3:.1f} us ({res['stage_pass']})",
+                     "peak_kind": f"bf16 dense, burst (kernel timed in a short pass), {pk['source']}"},
+        "stages_ms": res["stages_ms"],
+        "accept_hbm": {"achieved_gbs": rf["accept_gbs"], "peak_gbs": pk["hbm_gbs"], "frac": rf["accept_frac"],
+                       "bytes": res["acc_bytes"]},
+        "nodes_per_step": res["nodes"],
+        "accept_len_hist": np.bincount(acc_len, minlength=min(shape.D, shape.N - 1) + 1).tolist(),
         "tokens_per_step": int((acc_len + 1).sum()),
-        "attn_gflop_per_step": flops / 1e9,
+        "attn_gflop_per_step": res["flops"] / 1e9,
         "gpu_launches": launches_per_step * args.steps,
-        "e2e": e2e,
         "clocks": clocks,
-        "timed_loop": "cuda-graph replays of the step" if graphs is not None else "plain library calls",
+        "timed_loop": "cuda-graph replays of the step" if res["graphs"] else "plain library calls",
     }
     if args.sweep:
         line["sweep_point"] = True
-        line["attn_split_keys"] = lib.verify_attn_workspace_size(B, N, H, shape.d_l, shape.d_r, maxL, tdt) > 256
-    elif args.cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(args, shape, x, logits_h, t_host)
+        line["attn_split_keys"] = res["split_keys"]
+    else:
+        dr, comp = res["drafter"], res["compaction"]
+        line["drafter_topk"] = dict(dr, frac=dr["gbs"] / pk["hbm_gbs"], peak_gbs=pk["hbm_gbs"])
+        line["compaction_layers"] = None if comp is None else dict(
+            comp, frac=comp["marginal_gbs"] / pk["hbm_gbs"], peak_gbs=pk["hbm_gbs"])
+        line["e2e"] = res["e2e"]
+        lm = res.get("lmhead")
+        if lm is not None:
+            t_tc = lm["flops"] / (pk["bf16_tflops"] * 1e12)
+            t_hbm = lm["head_bytes"] / (pk["hbm_gbs"] * 1e9)
+            lm.update({"tflops": lm["flops"] / (lm["us"] * 1e-6) / 1e12,
+                       "head_gbs": lm["head_bytes"] / (lm["us"] * 1e-6) / 1e9,
+                       "bound": "tensor" if t_tc >= t_hbm else "hbm",
+                       "roofline_frac": max(t_tc, t_hbm) / (lm["us"] * 1e-6),
+                       "peaks": f"bf16 {pk['bf16_tflops']} TFLOP/s burst, HBM {pk['hbm_gbs']} GB/s ({pk['source']})"})
+            line["lmhead"] = lm
+        line["workloads"] = {}
+        for name, r in extra.items():
+            rr = stage_rooflines(r, pk)
+            line["workloads"][name] = {
+                "value": replica_throughput(r["nodes"], args.steps, world, r["elapsed_ms"]), "unit": UNIT,
+                "ms_per_step": r["elapsed_ms"] / args.steps, "stages_ms": r["stages_ms"],
+                "attn_tflops": rr["attn_tflops"], "attn_frac": rr["attn_frac"], "accept_gbs": rr["accept_gbs"],
+                "accept_frac": rr["accept_frac"], "nodes_per_step": r["nodes"],
+                "tokens_per_step": int((r["acc_len"] + 1).sum())}
+        if args.cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(args, shape, res["x"], res["logits_h"], res["t_host"])
     print(json.dumps(line), flush=True)
 
 
@@ -561,10 +754,13 @@ def measure_drafter(args, shape, lib, dev, tdt):
     return {"us": us, "gbs": row_bytes / (us / 1e6) / 1e9, "rows": R, "V": V, "K": K}
 
 
-def run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_acc, out, lse, off, cap, maxL, world):
+def run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_acc, out, lse, off, cap, maxL, world,
+            head=None):
     """Same step through the public API, inputs from pinned host memory each
     step (drafter output, queries, the tree rows' latent KV, target logits,
-    cache lengths) and the committed tokens read back."""
+    cache lengths) and the committed tokens read back. With `head` (device
+    head weights and host hidden states) the accept runs the fused LM head:
+    the verify rows' hidden states are copied in instead of logits."""
     import torch
     import torch.distributed as dist
 
@@ -577,7 +773,11 @@ def run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_a
 
     B, N = shape.B, shape.N
     h = {"logp": pin(x.logp), "tok": pin(x.tok), "root": pin(x.root_tok), "cl": pin(x.cache_len),
-         "q": pin(x.q, bf), "logits": pin(logits_h, bf)}
+         "q": pin(x.q, bf)}
+    if head is None:
+        h["logits"] = pin(logits_h, bf)
+    else:
+        h["hidden"] = head["hidden_h"].pin_memory()
     tree_rows = [pin(x.kv[int(x.cache_off[b]) + int(x.cache_len[b]):int(x.cache_off[b]) + int(x.cache_len[b]) + N],
                      bf) for b in range(B)]
     # two device copies of the per-step inputs: the next step's host-to-device
@@ -617,8 +817,12 @@ def run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_a
         lib.build_tree(d["logp"], d["tok"], d["root"], d["cl"], N, out=tree, stream=stream)
         lib.verify_attn(d["q"], kv, off, d["cl"], tree["mask"], tree["n_nodes"], shape.d_l, shape.d_r, shape.scale,
                         maxL, out=out, lse=lse, workspace=ws_attn, stream=stream)
-        lib.accept_compact(d["logits"], tree["node_tok"], tree["parent"], tree["n_nodes"], kv, off, d["cl"], cap,
-                           out=acc, workspace=ws_acc, stream=stream)
+        if head is None:
+            lib.accept_compact(d["logits"], tree["node_tok"], tree["parent"], tree["n_nodes"], kv, off, d["cl"], cap,
+                               out=acc, workspace=ws_acc, stream=stream)
+        else:
+            lib.accept_compact_lmhead(d["hidden"], head["w"], tree["node_tok"], tree["parent"], tree["n_nodes"], kv,
+                                      off, d["cl"], cap, out=acc, workspace=ws_acc, stream=stream)
         freed[i].record(stream)
         res_h["out_tok"].copy_(acc["out_tok"], non_blocking=True)
         res_h["acc_len"].copy_(acc["acc_len"], non_blocking=True)
@@ -646,47 +850,68 @@ def run_e2e(args, shape, x, logits_h, dev, stream, lib, tree, acc, ws_attn, ws_a
             "h2d_gbs": h2d * steps / (ms / 1e3) / 1e9}
 
 
-def _oracle_steps(shape, x, logits_h, tree, nodes, seconds):
-    """Oracle step estimates (each with its own node sample) until `seconds`
-    of wall time have passed; returns (mean scaled step seconds, steps,
-    sampled nodes per step, all nodes)."""
-    t0 = time.perf_counter()
-    secs = []
-    picked = total = 0
-    while not secs or time.perf_counter() - t0 < seconds:
-        sec, picked, total, _, _ = oracle_step_time(shape, x, logits_h, tree, nodes, seed=len(secs))
-        secs.append(sec)
-    return float(np.mean(secs)), len(secs), picked, total
-
-
-def cpu_baseline(args, shape, x, logits_h, t_host):
-    """The oracle's time for this workload's step on the host cores, from a
-    bounded sample (about args.cpu_seconds of wall time), with numpy's BLAS on
-    all its threads and again (for half as long) on one."""
-    import oracle
-    tree = oracle.build_tree(x.logp, x.tok, x.root_tok, x.cache_len, shape.N)
-    sec, steps, picked, total = _oracle_steps(shape, x, logits_h, tree, args.ref_nodes, args.cpu_seconds)
-    one = None
+def cpu_baseline(args, shape, x, logits_h, t_host=None):
+    """The oracle's throughput on this workload on the host cores: its whole
+    step on three of the workload's requests (requests in turn; each step
+    complete, nothing scaled), numpy's BLAS on all its threads; then one
+    request on one thread, with attention on as many of its nodes as fit
+    about args.cpu_seconds and scaled to all of them (labelled)."""
+    reqs = [request_slice(x, logits_h, b) for b in range(shape.B)]
+    secs, nodes, per_node = [], 0, []
+    for k in range(3):
+        t, ta, m, n = oracle_request_step(shape, reqs[k % shape.B])
+        secs.append(t)
+        nodes += n
+        per_node.append(ta / max(1, m))
+    value = nodes / float(sum(secs))
+    one, one_desc = None, None
     try:
         from threadpoolctl import threadpool_limits
+        r0 = reqs[0]
+        n0 = int(synth_nodes(shape))
+        # one thread runs the BLAS part several times slower: size the node
+        # sample from the all-threads rate, at least one node
+        m = max(1, min(n0, int(args.cpu_seconds / (4.0 * max(min(per_node), 1e-6)))))
         with threadpool_limits(limits=1, user_api="blas"):
-            sec1, _, _, _ = _oracle_steps(shape, x, logits_h, tree, args.ref_nodes, args.cpu_seconds / 2)
-        one = total / sec1
+            t, ta, m, n = oracle_request_step(shape, r0, attn_nodes=m)
+        full = (t - ta) + ta * n / m
+        one = n / full
+        one_desc = (f"one request, whole step on one BLAS thread" if m == n else
+                    f"one request on one BLAS thread: build, accept + compaction whole, attention on {m} of its "
+                    f"{n} nodes scaled by {n}/{m} (extrapolated)")
     except Exception:  # no BLAS thread control here: report the all-threads figure only
         one = None
-    return {"value": total / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "value_1thread": one,
-            "sample": f"{steps} step estimates in about {args.cpu_seconds:.0f} s: each a full build, attention "
-                      f"on {picked} of {total} nodes (all heads, a new sample per step) scaled by {total}/{picked}, "
-                      f"full accept + compaction"}
+    return {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "median_step_s": float(statistics.median(secs)),
+            "value_1thread": one, "sample_1thread": one_desc,
+            "sample": f"3 steps, each the oracle's whole step on one of the workload's {shape.B} requests in turn "
+                      f"(tree build, attention on all its nodes and heads, accept + compaction); "
+                      f"{nodes} nodes in {sum(secs):.1f} s, nothing scaled"}
+
+
+def synth_nodes(shape: synth.Shape) -> int:
+    """Tree nodes of one request (the budget, when the drafter's tree can fill
+    it, as every workload's can)."""
+    total, width = 1, 1
+    for _ in range(shape.D):
+        width *= shape.K
+        total += width
+        if total >= shape.N:
+            return shape.N
+    return total
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10000)
-    ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--config", default="kimi-1req", choices=sorted(synth.NAMED))
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="kimi-4req-32k", choices=sorted(synth.NAMED),
+                    help="the workload of the headline line (default: the long-context step, the largest that "
+                         "one GPU runs)")
+    ap.add_argument("--extra", default="kimi-1req,kimi-16req",
+                    help="comma list of further workloads measured after the headline one and reported under "
+                         "'workloads' ('' for none)")
     ap.add_argument("--seed", type=int, default=None,
                     help="seed of the step's draws (drafter output, cache, queries, logits) instead of the "
                          "workload's own; the workload's cache lengths stay as defined")
@@ -694,12 +919,11 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--layers", type=int, default=61,
                     help="layers of the multi-layer compaction measurement (< 2: skip it)")
-    ap.add_argument("--ref-nodes", type=int, default=8)
     ap.add_argument("--ref-budget", type=float, default=120.0,
                     help="wall seconds the reference arm's timed steps may take")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
-                    help="wall seconds of oracle work behind cpu_baseline (one-thread run: half)")
+                    help="about how long the one-thread oracle run of cpu_baseline may take")
     ap.add_argument("--dump", default=None,
                     help="write one step's inputs and the library's outputs to this .npz (replayable)")
     ap.add_argument("--e2e-serial", action="store_true",
@@ -707,6 +931,8 @@ def main():
     ap.add_argument("--sweep", default=None,
                     help="context/budget sweep on Kimi shapes: 'default' or a comma list of B:N:L points; one "
                          "JSON line per point (no end-to-end leg, no CPU baseline)")
+    ap.add_argument("--no-lmhead", dest="lmhead", action="store_false",
+                    help="skip the fused LM-head accept leg (head kernel, step and end to end)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time plain library calls instead of CUDA-graph replays of the step")
     args = ap.parse_args()

@@ -175,7 +175,10 @@ __global__ void __launch_bounds__(kWalkThreads) accept_walk_kernel(AcceptParams 
   // The tree and the cache bookkeeping are inputs the argmax kernel does not
   // write, and this grid starts only after that kernel has waited for all
   // earlier work: stage them before waiting for the argmax.
-  const int n = p.n_nodes[b];
+  // a node count outside [0, N] is bad input: the request is skipped, and
+  // only [0, N) is ever indexed
+  const int n_raw = p.n_nodes[b];
+  const int n = min(max(n_raw, 0), N);
   for (int i = tid; i < n; i += kWalkThreads) {
     s_par[i] = p.parent[(size_t)b * N + i];
     s_tok[i] = p.node_tok[(size_t)b * N + i];
@@ -184,12 +187,24 @@ __global__ void __launch_bounds__(kWalkThreads) accept_walk_kernel(AcceptParams 
   if (tid == 0) {
     int st = DDT_OK;
     const int L = p.cache_len[b];
-    if (n > 0 && (int64_t)L + n > (int64_t)p.cache_cap[b]) st = DDT_ERR_CAPACITY;
+    const int64_t off = p.cache_off[b];
+    // the rows the compaction may touch on every layer, l * stride + off +
+    // [L, L + n), must lie in the pool
+    const int64_t last = (int64_t)(p.n_layers - 1) * (p.layer_stride_bytes / p.row_bytes) + off + L + n;
+    if (n_raw > N) st = DDT_ERR_INPUT;
+    else if (n > 0 && (off < 0 || L < 0 || last > p.kv_rows)) st = DDT_ERR_BOUNDS;
+    else if (n > 0 && (int64_t)L + n > (int64_t)p.cache_cap[b]) st = DDT_ERR_CAPACITY;
     s_misc[0] = (n <= 0 || st != DDT_OK);
     if (p.dev_status) p.dev_status[b] = st;
   }
   pdl_wait();
   pdl_launch_dependents();
+  // the kernel that produced the row keys gave up a wait: they are not
+  // complete, so nothing is accepted (the keys are still cleared)
+  if (p.status_word != nullptr && tid == 0 && *reinterpret_cast<const volatile int*>(p.status_word) != 0) {
+    s_misc[0] = 1;
+    if (p.dev_status) p.dev_status[b] = DDT_ERR_TIMEOUT;
+  }
   for (int i = tid; i < N; i += kWalkThreads) {
     int a = -1;
     if (i < n) {
@@ -291,21 +306,10 @@ size_t accept_workspace_bytes(int B, int N, int V) {
   return zeroed_bytes(B, N);
 }
 
-static int sm_count() {
-  static int counts[128] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
-  if (counts[dev] == 0) {
-    int c = 0;
-    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
-    counts[dev] = c;
-  }
-  return counts[dev];
-}
 
 int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream) {
   unsigned char* ws = static_cast<unsigned char*>(workspace);
-  p.abort = reinterpret_cast<int*>(ws);
+  // the first 256 bytes are reserved (no kernel here waits on anything)
   p.rowkey = reinterpret_cast<unsigned long long*>(ws + header_bytes());
   const size_t esz = p.logits_dtype == DDT_BF16 ? 2 : 4;
   p.tma = (reinterpret_cast<uintptr_t>(p.logits) % 16 == 0) && (((size_t)p.V * esz) % 16 == 0);
@@ -318,6 +322,16 @@ int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream) 
                      ? launch_pdl(accept_argmax_kernel<true>, grid, kArgmaxThreads, 0, stream, p)
                      : launch_pdl(accept_argmax_kernel<false>, grid, kArgmaxThreads, 0, stream, p);
   if (st != DDT_OK) return st;
+  return launch_pdl(accept_walk_kernel, (unsigned)p.B, kWalkThreads, 0, stream, p);
+}
+
+// The walk and compaction alone, on row keys another kernel (the LM-head
+// argmax) left in the workspace; a non-zero status word there means that
+// kernel gave up.
+int launch_accept_walk(AcceptParams p, void* workspace, cudaStream_t stream) {
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  p.rowkey = reinterpret_cast<unsigned long long*>(ws + header_bytes());
+  p.status_word = reinterpret_cast<const int*>(ws);
   return launch_pdl(accept_walk_kernel, (unsigned)p.B, kWalkThreads, 0, stream, p);
 }
 
@@ -337,9 +351,9 @@ size_t accept_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 // the host it names a stand-in, not device memory.
 static void* noalloc_scratch_ptr(int* status) {
   static std::mutex mu;
-  static void* ptrs[128] = {nullptr};
+  static void* ptrs[kMaxDevices] = {nullptr};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     *status = DDT_ERR_CUDA;
     return nullptr;
   }

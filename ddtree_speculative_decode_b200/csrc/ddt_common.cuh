@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
 #include <utility>
 
 #include "../../include/ddt.h"
@@ -32,6 +34,29 @@ __device__ __forceinline__ uint32_t float_order_key(float x) {
 }
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Host state the library keeps per device ordinal (below this bound).
+constexpr int kMaxDevices = 128;
+
+// Streaming multiprocessors of the current device, looked up once per device
+// (148 on a B200; 148 also when the query fails).
+inline int sm_count() {
+  static std::mutex mu;
+  static int counts[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (counts[dev] == 0) {
+    int c = 0;
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
+    counts[dev] = c;
+  }
+  return counts[dev];
+}
+
+// Wall-clock limit of every bounded wait inside a kernel, in nanoseconds
+// (process-wide; read when a kernel is launched). ddt_set_wait_limit_ns sets it.
+uint64_t wait_limit_ns();
 
 // Programmatic dependent launch: a kernel launched with the PDL attribute may
 // start while its predecessor on the stream is still running; it must wait

@@ -33,6 +33,7 @@ struct AcceptParams {
   const int32_t* n_nodes;
   int B, N;
   unsigned char* kv;
+  int64_t kv_rows;              // rows in the pool (all layers)
   int row_bytes;
   int n_layers;
   int64_t layer_stride_bytes;
@@ -45,15 +46,21 @@ struct AcceptParams {
   int32_t* out_tok;
   int32_t* bonus;
   int32_t* dev_status;
-  int* abort;                   // workspace status word (DDT_ERR_TIMEOUT after an expired wait)
   unsigned long long* rowkey;   // [B*N] packed (value, ~index) row maxima (zero between calls)
-  int chunks;
+  const int* status_word;       // nullable: non-zero when the argmax producer gave up a wait
   int tma;                      // logits rows stream by bulk copies (16-byte aligned rows)
 };
 size_t accept_workspace_bytes(int B, int N, int V);
 int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream);
+int launch_accept_walk(AcceptParams p, void* workspace, cudaStream_t stream);
 size_t accept_noalloc_scratch_bytes();
 int launch_accept_compact_noalloc(AcceptParams p, cudaStream_t stream);
+
+// ---- target LM head folded into the accept argmax ------------------------------
+bool lmhead_supported(int d_model, int V, const void* hidden, const void* w_vocab);
+// row keys of the workspace (ddt_accept_compact layout) from hidden [B*N][d] x w [V][d]
+int launch_lmhead_argmax(const void* hidden, const void* w_vocab, int d_model, int V, int B, int N,
+                         const int32_t* n_nodes, void* workspace, cudaStream_t stream);
 
 // ---- drafter proposals --------------------------------------------------------
 struct DrafterParams {
@@ -82,12 +89,14 @@ struct AttnParams {
   int in_dtype, out_dtype;
   void* out;
   float* lse;
+  int32_t* dev_status;  // [B], nullable: DDT_OK or DDT_ERR_BOUNDS
+  int64_t kv_rows;
 };
 int launch_attn_simt(const AttnParams& p, cudaStream_t stream);
 
 bool tc_attn_supported(int d_l, int d_r, int in_dtype);
 size_t tc_attn_workspace_bytes(int B, int N, int H, int max_cache_len);
-int launch_attn_tc(const AttnParams& p, int64_t kv_rows, int max_cache_len, void* workspace,
+int launch_attn_tc(const AttnParams& p, int max_cache_len, void* workspace,
                    size_t workspace_bytes, cudaStream_t stream);
 
 }  // namespace ddt

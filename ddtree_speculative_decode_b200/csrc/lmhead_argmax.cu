@@ -1,0 +1,410 @@
+// Target LM head folded into the accept argmax, sm_100a: the greedy token of
+// every verify row, argmax_v sum_c hidden[r][c] * w_vocab[v][c], without ever
+// writing the logits to memory.
+//
+// What it computes is fixed in ddt.h (ddt_accept_compact_lmhead): the argmax
+// of the target's logits is the greedy token the walk compares against
+// ("autoregressive_test_driver_kdtree_engine", section "What the Message
+// Actually Says": the greedy token of a verify row is the argmax of the
+// target's logits, checked exactly); the head maps the final hidden state
+// (Kimi K2.6: 7168 wide; "the_validation_pivot", section "Assumptions
+// Embedded in This Message") to the vocabulary.
+//
+// Structure: a persistent grid of CTA pairs (clusters of 2) walks the tiles
+// (pass of up to 512 verify rows) x (256 vocabulary rows). The vocabulary is
+// the MMA's M side (tcgen05.mma.cta_group::2, M = 256: each CTA supplies 128
+// vocabulary rows of the head and holds their 128 x N fp32 accumulator in its
+// tensor memory) and the verify rows are its N side (each CTA supplies half
+// of them), so one head row is read from HBM once per pass however few rows
+// are verified. The head and hidden tiles stream through a ring of stages by
+// TMA (64 dims per stage, 128-byte swizzle); warp 0 loads, warp 1 of the
+// leader CTA issues the MMAs, warps 2..5 reduce each finished accumulator:
+// per verify row (column) a warp-wide maximum of order-preserving value keys
+// (redux.sync) and the lowest lane holding it (ballot), so every tile yields,
+// per row, (largest logit, lowest vocabulary index) packed in 64 bits. Rows
+// keep their running best in registers across the pass's tiles and publish it
+// once per CTA with a 64-bit atomic max into the same per-row keys the
+// materialised-logits argmax writes, so the accept walk that follows is the
+// same kernel. The accumulator is double-buffered when a pass has at most
+// 256 rows, so the reduction of one tile overlaps the MMAs of the next.
+//
+// Rounding: each MMA adds 16 exact bf16 x bf16 products to the float32
+// accumulator and the 64-dim stages follow one another, so a product passes
+// through at most 15 + ceil(d / 16) roundings (the depth ddt.h declares).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "ddt_kernels.cuh"
+#include "sm100_ptx.cuh"
+
+namespace ddt {
+namespace lmh {
+
+using namespace sm100;
+
+constexpr int kThreads = 192;           // warp 0 TMA, warp 1 MMA (+ TMEM), warps 2..5 reduction
+constexpr int kABytes = 128 * 128;      // 128 head rows x 64 dims bf16 per CTA and stage
+constexpr int kPassRows = 512;          // verify rows per pass over the head
+constexpr int kMaxStages = 12;
+constexpr int kStageBudget = 200 * 1024;
+constexpr int kMaxChunks = kPassRows / 32;
+
+// shared memory after the stages
+constexpr int kBarFull = 0;                      // [kMaxStages] leader: TMA bytes of a stage (both CTAs)
+constexpr int kBarEmpty = kBarFull + kMaxStages;  // [kMaxStages] each CTA: MMAs done with a stage
+constexpr int kBarAccFull = kBarEmpty + kMaxStages;  // [2] each CTA: accumulator buffer complete
+constexpr int kBarAccEmpty = kBarAccFull + 2;        // [2] leader: accumulator read (4 warps x 2 CTAs)
+constexpr int kNumBars = kBarAccEmpty + 2;
+constexpr int kMiscBytes = 256;                  // barriers
+constexpr int kSlotBytes = 16;                   // TMEM address + abort flag
+constexpr int kRedBytes = kPassRows * 8;         // per-column running key of the CTA
+static_assert(kNumBars * 8 <= kMiscBytes, "barrier area");
+
+struct Params {
+  int R, d, V, N;
+  int nkb;        // 64-dim stages per tile
+  int vtiles;     // 256-row vocabulary tiles
+  int passes;     // passes of up to 512 verify rows
+  int parts;      // N-parts per MMA step: 1 (pass <= 256 rows) or 2 (N = 256 each)
+  int npart;      // N of one part (multiple of 16)
+  int nh;         // verify rows one CTA supplies per part (npart / 2)
+  int stages, stage_bytes, nbuf;
+  const int32_t* n_nodes;
+  unsigned long long* rowkey;
+  int* abort;
+  uint64_t wait_ns;
+};
+
+__device__ __forceinline__ int ld_volatile_i32(const int* p) {
+  int v;
+  asm volatile("ld.volatile.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    lmhead_argmax_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_h,
+                         Params p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  pdl_wait();
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+  const int total = p.passes * p.vtiles;
+  const uint32_t misc = sbase + (uint32_t)(p.stages * p.stage_bytes);
+  auto bar = [&](int i) -> uint32_t { return misc + 8u * (uint32_t)i; };
+  unsigned char* slot_area = smem + p.stages * p.stage_bytes + kMiscBytes;
+  unsigned long long* s_red =
+      reinterpret_cast<unsigned long long*>(smem + p.stages * p.stage_bytes + kMiscBytes + kSlotBytes);
+  int* abort = p.abort;
+  const uint64_t wlim = p.wait_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(bar(kBarFull + s), 1);
+      mbar_init(bar(kBarEmpty + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(kBarAccFull + b), 1);
+      mbar_init(bar(kBarAccEmpty + b), 8);
+    }
+    fence_mbar_init_cluster();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_h);
+  }
+  for (int c = threadIdx.x; c < kPassRows; c += kThreads) s_red[c] = 0ull;
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(slot_area), 512);
+    tmem_relinquish_pair();
+  }
+  // a workspace whose status word already holds an error (an earlier call
+  // gave up a wait) makes the call do no work; the leader CTA reads the word
+  // and both CTAs of the pair take its value
+  if (leader && threadIdx.x == 0) *reinterpret_cast<volatile int*>(slot_area + 4) = ld_volatile_i32(abort);
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(slot_area);
+  const bool aborted = ld_cluster_u32(map_to_rank(smem_u32(slot_area + 4), 0)) != 0u;
+
+  if (aborted) {
+    // nothing to do: straight to the teardown
+  } else if (warp == 0 && lane == 0) {
+    // ============================================================ TMA producer
+    const uint32_t full0 = map_to_rank(bar(kBarFull), 0);
+    int slot = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = pair; t < total && ok; t += npairs) {
+      const int pass = t / p.vtiles, vt = t - pass * p.vtiles;
+      const int v0 = vt * 256 + 128 * (int)rank;
+      const int h0 = pass * kPassRows + p.nh * (int)rank;
+      for (int kb = 0; kb < p.nkb; ++kb) {
+        if (!mbar_wait(bar(kBarEmpty + slot), phase ^ 1u, abort, wlim)) {
+          ok = false;
+          break;
+        }
+        if (leader) mbar_arrive_expect_tx(bar(kBarFull + slot), 2u * (uint32_t)p.stage_bytes);
+        const uint32_t dst = sbase + (uint32_t)(slot * p.stage_bytes);
+        const uint32_t fb = full0 + 8u * (uint32_t)slot;
+        tma_load_2d_pair(dst, &tm_w, 64 * kb, v0, fb);
+        for (int j = 0; j < p.parts; ++j)
+          tma_load_2d_pair(dst + kABytes + (uint32_t)(j * p.nh * 128), &tm_h, 64 * kb, h0 + 256 * j, fb);
+        if (++slot == p.stages) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ============================================================ MMA issuer
+    const uint32_t idesc = idesc_bf16_f32(256, p.npart, false, false);
+    int slot = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    int lt = 0;
+    for (int t = pair; t < total && ok; t += npairs, ++lt) {
+      const int buf = lt % p.nbuf;
+      if (!mbar_wait(bar(kBarAccEmpty + buf), (uint32_t)((lt / p.nbuf) & 1) ^ 1u, abort, wlim)) break;
+      tc_fence_after();
+      for (int kb = 0; kb < p.nkb; ++kb) {
+        if (!mbar_wait(bar(kBarFull + slot), phase, abort, wlim)) {
+          ok = false;
+          break;
+        }
+        const uint32_t a0 = sbase + (uint32_t)(slot * p.stage_bytes);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          for (int j = 0; j < p.parts; ++j)
+            mma_pair_ss(tmem + (uint32_t)((buf * p.parts + j) * 256), smem_desc_sw128(a0 + 32 * k, 16, 1024),
+                        smem_desc_sw128(a0 + kABytes + (uint32_t)(j * p.nh * 128) + 32 * k, 16, 1024), idesc,
+                        (kb | k) != 0 ? 1u : 0u);
+        mma_commit_pair_mc(bar(kBarEmpty + slot), (uint16_t)0x3u);
+        if (++slot == p.stages) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok) mma_commit_pair_mc(bar(kBarAccFull + buf), (uint16_t)0x3u);
+    }
+  } else if (warp >= 2) {
+    // ============================================================ reduction
+    // thread = TMEM lane 32 q + lane = vocabulary row 128 rank + 32 q + lane
+    // of the tile; for every column (verify row) the warp's best over its 32
+    // rows, kept by lane (column % 32) in best[column / 32]
+    const int q = warp & 3;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
+    const uint32_t empty0 = map_to_rank(bar(kBarAccEmpty), 0);
+    const int ncols = p.parts == 2 ? kPassRows : p.npart;
+    const int nchunks = (ncols + 31) / 32;
+    unsigned long long best[kMaxChunks];
+#pragma unroll
+    for (int m = 0; m < kMaxChunks; ++m) best[m] = 0ull;
+    int cur_pass = -1;
+    bool ok = true;
+    // the CTA's best per column into shared memory, then one global atomic
+    // max per real verify row of the pass
+    auto flush = [&](int pass) {
+#pragma unroll
+      for (int m = 0; m < kMaxChunks; ++m) {
+        if (m < nchunks && best[m] != 0ull) atomicMax(s_red + 32 * m + lane, best[m]);
+        best[m] = 0ull;
+      }
+      named_bar_sync(1, 128);
+      for (int c = (int)threadIdx.x - 64; c < ncols; c += 128) {
+        const unsigned long long k = s_red[c];
+        s_red[c] = 0ull;
+        const int r = pass * kPassRows + c;
+        if (k == 0ull || r >= p.R) continue;
+        const int b = r / p.N, i = r - b * p.N;
+        if (i < __ldg(p.n_nodes + b)) atomicMax(p.rowkey + r, k);
+      }
+      named_bar_sync(1, 128);
+    };
+    named_bar_sync(1, 128);  // s_red zeroed by the whole CTA before the barrier above; keep the 4 warps in step
+    int lt = 0;
+    for (int t = pair; t < total; t += npairs, ++lt) {
+      const int pass = t / p.vtiles, vt = t - pass * p.vtiles;
+      if (pass != cur_pass) {
+        if (cur_pass >= 0) flush(cur_pass);
+        cur_pass = pass;
+      }
+      const int buf = lt % p.nbuf;
+      if (ok && !mbar_wait(bar(kBarAccFull + buf), (uint32_t)((lt / p.nbuf) & 1), abort, wlim)) ok = false;
+      tc_fence_after();
+      const int vrow = vt * 256 + 128 * (int)rank + 32 * q;  // vocabulary row of lane 0
+      const bool valid = ok && vrow + lane < p.V;
+      const uint32_t col0 = (uint32_t)(buf * p.parts * 256);
+#pragma unroll
+      for (int m = 0; m < kMaxChunks; ++m) {
+        if (m < nchunks) {
+          uint32_t r[32];
+          tmem_ld32(lane_addr + col0 + 32u * (uint32_t)m, r);
+          tmem_wait_ld();
+          if (m == nchunks - 1) {
+            // the accumulator buffer is free for the next tile's MMAs
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              if (leader) mbar_arrive_local(bar(kBarAccEmpty + buf));
+              else mbar_arrive_cluster(empty0 + 8u * (uint32_t)buf);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const uint32_t key = valid ? float_order_key(__uint_as_float(r[i])) : 0u;
+            const uint32_t mx = __reduce_max_sync(DDT_FULL_MASK, key);
+            const uint32_t hit = __ballot_sync(DDT_FULL_MASK, key == mx);
+            const unsigned long long packed =
+                ((unsigned long long)mx << 32) | (unsigned long long)(~(uint32_t)(vrow + __ffs(hit) - 1));
+            if (lane == i && mx != 0u && packed > best[m]) best[m] = packed;
+          }
+        }
+      }
+    }
+    if (cur_pass >= 0) flush(cur_pass);
+  }
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    return nullptr;
+  }();
+  return fn;
+}
+
+// [rows][d] bf16, row-major: boxes of 64 dims x box_rows rows, 128-byte swizzle
+static bool make_map(CUtensorMap* m, const void* base, uint64_t d, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int smem_bytes(const Params& p) {
+  return p.stages * p.stage_bytes + kMiscBytes + kSlotBytes + kRedBytes + 1024;
+}
+
+// CTA pairs of this kernel that can be resident at once on the current
+// device, looked up once per device (with the shared-memory opt-in set).
+static int device_pairs(int smem) {
+  static std::mutex mu;
+  static int pairs[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cudaFuncSetAttribute(lmhead_argmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kStageBudget + kMiscBytes + kSlotBytes + kRedBytes + 1024) != cudaSuccess)
+    return -1;
+  if (pairs[dev] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 64);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, lmhead_argmax_kernel, &cfg) != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = sm_count() / 2;
+    }
+    pairs[dev] = n;
+  }
+  return pairs[dev];
+}
+
+}  // namespace lmh
+
+bool lmhead_supported(int d_model, int V, const void* hidden, const void* w_vocab) {
+  return d_model >= 8 && d_model % 8 == 0 && V >= 1 && (reinterpret_cast<uintptr_t>(hidden) % 16) == 0 &&
+         (reinterpret_cast<uintptr_t>(w_vocab) % 16) == 0;
+}
+
+int launch_lmhead_argmax(const void* hidden, const void* w_vocab, int d_model, int V, int B, int N,
+                         const int32_t* n_nodes, void* workspace, cudaStream_t stream) {
+  using namespace lmh;
+  Params p{};
+  p.R = B * N;
+  p.d = d_model;
+  p.V = V;
+  p.N = N;
+  p.nkb = (d_model + 63) / 64;
+  p.vtiles = (V + 255) / 256;
+  if (p.R <= 256) {
+    p.parts = 1;
+    p.npart = std::max(16, (p.R + 15) / 16 * 16);
+    p.passes = 1;
+    p.nbuf = 2;
+  } else {
+    p.parts = 2;
+    p.npart = 256;
+    p.passes = (p.R + kPassRows - 1) / kPassRows;
+    p.nbuf = 1;
+  }
+  p.nh = p.npart / 2;
+  p.stage_bytes = kABytes + p.parts * p.nh * 128;
+  p.stages = std::min(kMaxStages, kStageBudget / p.stage_bytes);
+  p.n_nodes = n_nodes;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  p.abort = reinterpret_cast<int*>(ws);
+  p.rowkey = reinterpret_cast<unsigned long long*>(ws + 256);
+  p.wait_ns = wait_limit_ns();
+  CUtensorMap tw, th;
+  if (!make_map(&tw, w_vocab, (uint64_t)d_model, (uint64_t)V, 128) ||
+      !make_map(&th, hidden, (uint64_t)d_model, (uint64_t)p.R, (uint32_t)p.nh))
+    return DDT_ERR_CUDA;
+  const int smem = smem_bytes(p);
+  const int slots = device_pairs(smem);
+  if (slots <= 0) return DDT_ERR_CUDA;
+  const long long tiles = (long long)p.passes * p.vtiles;
+  const int pairs = (int)std::max<long long>(1, std::min<long long>(slots, tiles));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, lmhead_argmax_kernel, tw, th, p) == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
+}
+
+}  // namespace ddt

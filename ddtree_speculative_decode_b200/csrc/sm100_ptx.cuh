@@ -7,6 +7,8 @@
 
 #include <stdint.h>
 
+#include "../../include/ddt.h"
+
 namespace ddt {
 namespace sm100 {
 
@@ -76,6 +78,12 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_
   asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
+// Load from shared memory of a CTA of the cluster (address from map_to_rank).
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
 __device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float a, float b) {
   asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
 }
@@ -109,19 +117,22 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Default wall-clock limit of one wait (the launch passes the limit in force,
+// see ddt_set_wait_limit_ns).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
-// Wait until the phase with the given parity completed. Returns false (and
-// raises *abort) when the wall-clock limit passes or another thread aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* abort) {
+// Wait until the phase with the given parity completed. Returns false when
+// the wall-clock limit passes (the waiter then stores DDT_ERR_TIMEOUT in the
+// status word *abort) or when another thread already gave up (*abort != 0).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* abort, uint64_t limit_ns) {
   if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*reinterpret_cast<volatile int*>(abort) != 0) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        atomicExch(abort, 1);
+      if (global_timer_ns() - t0 > limit_ns) {
+        atomicExch(abort, DDT_ERR_TIMEOUT);
         return false;
       }
     }
@@ -131,13 +142,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* ab
 // Wait for a phase that this CTA's own copies complete: bounded by the same
 // wall-clock limit, but not cut short by another thread's abort (the copies
 // must land before their shared memory is reused or the CTA exits).
-__device__ __forceinline__ bool mbar_wait_own(uint32_t bar, uint32_t parity, int* abort) {
+__device__ __forceinline__ bool mbar_wait_own(uint32_t bar, uint32_t parity, int* abort, uint64_t limit_ns) {
   if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
-      atomicExch(abort, 1);
+    if ((it & 255u) == 0 && global_timer_ns() - t0 > limit_ns) {
+      atomicExch(abort, DDT_ERR_TIMEOUT);
       return false;
     }
   }

@@ -37,7 +37,13 @@ __global__ void __launch_bounds__(32 * kSimtWarps) attn_simt_kernel(AttnParams p
   const int i = (int)((row / p.H) % p.N);
   const int b = (int)(row / ((long long)p.H * p.N));
   const int d_qk = p.d_l + p.d_r;
-  const int n = p.n_nodes[b];
+  const int n_raw = p.n_nodes[b];
+  // a request whose rows do not lie in the pool (or whose node count is
+  // outside [0, N]) reads nothing: all its rows are written as pad rows
+  const bool oob = n_raw < 0 || n_raw > p.N || p.cache_off[b] < 0 || p.cache_len[b] < 0 ||
+                   p.cache_off[b] + p.cache_len[b] + n_raw > p.kv_rows;
+  const int n = oob ? 0 : n_raw;
+  if (p.dev_status && i == 0 && (row % p.H) == 0 && lane == 0) p.dev_status[b] = oob ? DDT_ERR_BOUNDS : DDT_OK;
 
   float* lse_out = p.lse ? p.lse + row : nullptr;
   if (i >= n) {

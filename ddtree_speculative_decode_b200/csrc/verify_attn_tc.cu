@@ -52,6 +52,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "ddt_kernels.cuh"
 #include "sm100_ptx.cuh"
@@ -78,16 +79,18 @@ constexpr float kRescaleThreshold = 8.0f;     // log2 units
 // V ring: one stage = 64 keys x both 128-dim output blocks (4 boxes, 32 KB).
 constexpr int kKStages = 4;
 constexpr int kKStageBytes = 3 * kBoxBytes;    // 24 KB
-constexpr int kVStages = 2;
-constexpr int kVStageBytes = 4 * kBoxBytes;    // 32 KB
+constexpr int kKGroup = 1;                     // QK stages released together (one barrier each way)
+constexpr int kKBars = kKStages / kKGroup;
+constexpr int kVStages = 4;
+constexpr int kVStageBytes = 2 * kBoxBytes;    // 16 KB: 64 keys x one 128-dim block of each output half
 constexpr int kOffKRing = 0;
 constexpr int kOffVRing = kOffKRing + kKStages * kKStageBytes;
 constexpr int kOffP = kOffVRing + kVStages * kVStageBytes;
 constexpr int kOffMisc = kOffP + kPBytes;
 // misc: barriers (8 B each)
-constexpr int kBarKFull = 0;                          // [kKStages / 2] leader: TMA bytes of a stage pair, both CTAs
-constexpr int kBarKEmpty = kBarKFull + kKStages / 2;  // [kKStages / 2] each CTA: QK MMAs done with a stage pair
-constexpr int kBarVFull = kBarKEmpty + kKStages / 2;  // [kVStages]
+constexpr int kBarKFull = 0;                          // [kKBars] leader: TMA bytes of a stage group, both CTAs
+constexpr int kBarKEmpty = kBarKFull + kKBars;        // [kKBars] each CTA: QK MMAs done with a stage group
+constexpr int kBarVFull = kBarKEmpty + kKBars;        // [kVStages]
 constexpr int kBarVEmpty = kBarVFull + kVStages;      // [kVStages]
 constexpr int kBarSFull = kBarVEmpty + kVStages;      // [2] each CTA: S buffer written
 constexpr int kBarSEmpty = kBarSFull + 2;             // [2] leader: S buffer read (softmax warps of both CTAs)
@@ -104,7 +107,7 @@ constexpr int kOffTmem = kOffMask + 64 * kMaxW * 4;     // uint32
 constexpr int kSmemBytes = kOffTmem + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;           // slack for 1024 alignment
 static_assert(kNumBars * 8 <= 256, "barrier area");
-static_assert(kKStages % 2 == 0, "QK stages are released in pairs");
+static_assert(kKStages % kKGroup == 0, "QK stages are released in whole groups");
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
 // epilogue staging (reuses the rings once the last MMA has completed): the
@@ -137,7 +140,10 @@ struct TcParams {
   float* part_o;     // [splits][B*N*H][512]
   float* part_ml;    // [splits][B*N*H][2]
   unsigned* counter; // [B * rowtiles * 2][2] per (row tile, CTA half): splits done, partials published; zero between calls
-  int* abort;
+  int32_t* dev_status;  // [B], nullable: DDT_OK or DDT_ERR_BOUNDS
+  int64_t kv_rows;
+  int* abort;        // workspace status word: DDT_ERR_TIMEOUT after a wait gave up
+  uint64_t wait_ns;  // wall-clock limit of every wait
 };
 
 struct UnitInfo {
@@ -147,6 +153,7 @@ struct UnitInfo {
   int kb, ke, T;     // key range [kb, ke) of this unit, T tiles
   int active;        // splits of this request that get keys (splits [0, active))
   bool pad_tile;     // every row of the row tile is a pad row
+  bool oob;          // the request's rows do not lie in the pool: all its rows are pad rows
 };
 
 __device__ __forceinline__ UnitInfo unit_info(const TcParams& p, int unit) {
@@ -155,9 +162,12 @@ __device__ __forceinline__ UnitInfo unit_info(const TcParams& p, int unit) {
   const int t = unit / p.splits;
   u.rt = t % p.rowtiles;
   u.b = t / p.rowtiles;
-  u.off_row = (int)p.cache_off[u.b];
-  u.L = p.cache_len[u.b];
-  u.n = p.n_nodes[u.b];
+  const int64_t off = p.cache_off[u.b];
+  const int L = p.cache_len[u.b], n = p.n_nodes[u.b];
+  u.oob = n < 0 || n > p.N || off < 0 || L < 0 || off + L + n > p.kv_rows;
+  u.off_row = u.oob ? 0 : (int)off;  // fits int: kv_rows does (checked on the host)
+  u.L = u.oob ? 0 : L;
+  u.n = u.oob ? 0 : n;
   u.nkeys = u.L + u.n;
   const int tiles = (u.nkeys + kTileKeys - 1) / kTileKeys;
   // splits get floor or ceil(tiles / splits) tiles, the larger shares last
@@ -221,6 +231,12 @@ __device__ __forceinline__ uint64_t group_visibility(int kw, int g0, int kend, i
   return range & (cache | mask_bits64(mw, W, kw - L));
 }
 
+__device__ __forceinline__ int ld_volatile_gpu(const int* p) {
+  int v;
+  asm volatile("ld.volatile.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -249,6 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int rows_total = p.B * p.N * p.H;
   const int req_rows = p.N * p.H;
   const int row0 = u.rt * 128 + 64 * (int)rank;  // first request-relative row of this CTA
+  if (p.dev_status && u.rt == 0 && u.split == 0 && rank == 0 && threadIdx.x == 0)
+    p.dev_status[u.b] = u.oob ? DDT_ERR_BOUNDS : DDT_OK;
 
   auto bar = [&](int i) -> uint32_t { return sbase + kOffMisc + 8u * (uint32_t)i; };
 
@@ -256,33 +274,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   // a split past the last one that gets keys has nothing to do; a row tile of
   // pad rows only is written (zeros, lse -inf) by split 0. In a 4-CTA cluster
   // an idle pair still takes part in the cluster-wide barriers below.
-  const bool idle = u.T == 0;
-  if (idle) {
-    if (u.pad_tile && u.split == 0) {
-      for (int r = threadIdx.x; r < 64; r += kThreads) {
-        const int rr = row0 + r;
-        if (rr >= req_rows) continue;
-        const size_t grow = (size_t)u.b * req_rows + rr;
-        if (p.lse) p.lse[grow] = -INFINITY;
-      }
-      for (int e = threadIdx.x; e < 64 * (kDL / 4); e += kThreads) {
-        const int r = e / (kDL / 4), c4 = e % (kDL / 4);
-        const int rr = row0 + r;
-        if (rr >= req_rows) continue;
-        const size_t grow = (size_t)u.b * req_rows + rr;
-        if (p.out_dtype == DDT_F32) {
-          reinterpret_cast<float4*>(static_cast<float*>(p.out) + grow * kDL)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
-        } else {
-          reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out) + grow * kDL)[c4] = make_uint2(0u, 0u);
-        }
+  // this CTA's 64 rows as pad rows (zeros, lse -inf), all threads
+  auto write_pad_rows = [&]() {
+    for (int r = threadIdx.x; r < 64; r += kThreads) {
+      const int rr = row0 + r;
+      if (rr >= req_rows) continue;
+      const size_t grow = (size_t)u.b * req_rows + rr;
+      if (p.lse) p.lse[grow] = -INFINITY;
+    }
+    for (int e = threadIdx.x; e < 64 * (kDL / 4); e += kThreads) {
+      const int r = e / (kDL / 4), c4 = e % (kDL / 4);
+      const int rr = row0 + r;
+      if (rr >= req_rows) continue;
+      const size_t grow = (size_t)u.b * req_rows + rr;
+      if (p.out_dtype == DDT_F32) {
+        reinterpret_cast<float4*>(static_cast<float*>(p.out) + grow * kDL)[c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out) + grow * kDL)[c4] = make_uint2(0u, 0u);
       }
     }
+  };
+  const bool idle = u.T == 0;
+  if (idle) {
+    if (u.pad_tile && u.split == 0) write_pad_rows();
     if (p.csize == 2) return;
   }
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kKStages / 2; ++s) {
+    for (int s = 0; s < kKBars; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
       mbar_init(bar(kBarKEmpty + s), 1);
     }
@@ -319,11 +339,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc_pair(sbase + kOffTmem, 512);
     tmem_relinquish_pair();
   }
+  // a workspace whose status word already holds an error (an earlier call
+  // gave up a wait) makes the call do no work: one thread of the cluster's
+  // first CTA reads the word and every CTA of the cluster takes its value, so
+  // the CTAs that share barriers agree
+  if (crank == 0 && threadIdx.x == 0) *reinterpret_cast<volatile int*>(smem + kOffTmem + 8) = ld_volatile_gpu(p.abort);
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmem);
+  const bool aborted = ld_cluster_u32(map_to_rank(sbase + kOffTmem + 8, 0)) != 0u;
   int* abort = p.abort;
+  const uint64_t wlim = p.wait_ns;
 
   // one ring of 16 KB stages per operand stream, each with its own producer
   // thread and its own MMA-issuing thread: while one issuer waits on a
@@ -332,8 +359,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int slot = 0;
     uint32_t phase = 0;
   };
-  if (idle) {
-    // nothing to compute: straight to the cluster-wide teardown
+  if (idle || aborted) {
+    // nothing to compute: straight to the cluster-wide teardown (after an
+    // earlier timeout split 0 writes its rows as pad rows)
+    if (aborted && !idle && u.split == 0) write_pad_rows();
   } else if (warp == 0 && lane == 0) {
     // ============================================================ QK producer
     // per tile and 64-dim chunk: this CTA's Q chunk and its 128 keys' chunk
@@ -346,17 +375,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int y1 = u.off_row + group_window(tile0 + 128 * (int)rank + 64, u.nkeys);
       bool ok = true;
       for (int ch = 0; ch < kChunks; ++ch) {
-        if ((rg.slot & 1) == 0) {
-          if (!mbar_wait(bar(kBarKEmpty + (rg.slot >> 1)), rg.phase ^ 1u, abort)) {
+        if (rg.slot % kKGroup == 0) {
+          if (!mbar_wait(bar(kBarKEmpty + rg.slot / kKGroup), rg.phase ^ 1u, abort, wlim)) {
             ok = false;
             break;
           }
-          // one barrier per stage pair; the pair is always filled completely
-          // (the last pair of the unit may get a duplicate stage, see below)
-          if (leader) mbar_arrive_expect_tx(bar(kBarKFull + (rg.slot >> 1)), 4u * kKStageBytes);
+          // one barrier per stage group; a group is always filled completely
+          // (the last group of the unit may get repeated stages, see below)
+          if (leader) mbar_arrive_expect_tx(bar(kBarKFull + rg.slot / kKGroup), 2u * kKGroup * kKStageBytes);
         }
         const uint32_t dst = sbase + kOffKRing + rg.slot * kKStageBytes;
-        const uint32_t fb = full0 + 8u * (uint32_t)(rg.slot >> 1);
+        const uint32_t fb = full0 + 8u * (uint32_t)(rg.slot / kKGroup);
         tma_load_2d_pair(dst, &tm_q, ch * 64, qrow, fb);
         tma_load_2d_pair(dst + kBoxBytes, &tm_kv, ch * 64, y0, fb);
         tma_load_2d_pair(dst + 2 * kBoxBytes, &tm_kv, ch * 64, y1, fb);
@@ -364,17 +393,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
     }
-    if (rg.slot & 1) {
-      // odd number of stages: complete the last pair's byte count with a
-      // repeat of the last Q box + key boxes (never consumed)
+    while (rg.slot % kKGroup != 0) {
+      // a partly filled last group: complete its byte count with repeats of
+      // the last Q box + key boxes (never consumed)
       const int tile0 = u.kb + (u.T - 1) * kTileKeys;
       const int y0 = u.off_row + group_window(tile0 + 128 * (int)rank, u.nkeys);
       const int y1 = u.off_row + group_window(tile0 + 128 * (int)rank + 64, u.nkeys);
       const uint32_t dst = sbase + kOffKRing + rg.slot * kKStageBytes;
-      const uint32_t fb = full0 + 8u * (uint32_t)(rg.slot >> 1);
+      const uint32_t fb = full0 + 8u * (uint32_t)(rg.slot / kKGroup);
       tma_load_2d_pair(dst, &tm_q, (kChunks - 1) * 64, qrow, fb);
       tma_load_2d_pair(dst + kBoxBytes, &tm_kv, (kChunks - 1) * 64, y0, fb);
       tma_load_2d_pair(dst + 2 * kBoxBytes, &tm_kv, (kChunks - 1) * 64, y1, fb);
+      if (++rg.slot == kKStages) { rg.slot = 0; rg.phase ^= 1u; }
     }
   } else if (warp == 2 && lane == 0) {
     // ============================================================ V producer
@@ -386,20 +416,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tile0 = u.kb + t * kTileKeys;
       bool ok = true;
       const int ng = live_groups(u, t);
-      for (int g = 0; g < ng; ++g) {
-        if (!mbar_wait(bar(kBarVEmpty + rg.slot), rg.phase ^ 1u, abort)) {
-          ok = false;
-          break;
-        }
-        if (leader) mbar_arrive_expect_tx(bar(kBarVFull + rg.slot), 2u * kVStageBytes);
+      for (int g = 0; g < ng && ok; ++g) {
         const int y = u.off_row + group_window(tile0 + 64 * g, u.nkeys);
-        const uint32_t dst = sbase + kOffVRing + rg.slot * kVStageBytes;
-        const uint32_t fb = full0 + 8u * (uint32_t)rg.slot;
-        tma_load_2d_pair(dst, &tm_kv, x, y, fb);
-        tma_load_2d_pair(dst + kBoxBytes, &tm_kv, x + 64, y, fb);
-        tma_load_2d_pair(dst + 2 * kBoxBytes, &tm_kv, x + 256, y, fb);
-        tma_load_2d_pair(dst + 3 * kBoxBytes, &tm_kv, x + 320, y, fb);
-        if (++rg.slot == kVStages) { rg.slot = 0; rg.phase ^= 1u; }
+        // one stage per output half j: this CTA's 128 dims of it
+        for (int j = 0; j < 2; ++j) {
+          if (!mbar_wait(bar(kBarVEmpty + rg.slot), rg.phase ^ 1u, abort, wlim)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(bar(kBarVFull + rg.slot), 2u * kVStageBytes);
+          const uint32_t dst = sbase + kOffVRing + rg.slot * kVStageBytes;
+          const uint32_t fb = full0 + 8u * (uint32_t)rg.slot;
+          tma_load_2d_pair(dst, &tm_kv, x + 256 * j, y, fb);
+          tma_load_2d_pair(dst + kBoxBytes, &tm_kv, x + 256 * j + 64, y, fb);
+          if (++rg.slot == kVStages) { rg.slot = 0; rg.phase ^= 1u; }
+        }
       }
       if (!ok) break;
     }
@@ -414,19 +445,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < u.T && ok; ++t) {
         const int sb = t & 1;
         if (t >= 2) {
-          if (!mbar_wait(bar(kBarSEmpty + sb), (uint32_t)(((t >> 1) + 1) & 1), abort)) { ok = false; break; }
+          if (!mbar_wait(bar(kBarSEmpty + sb), (uint32_t)(((t >> 1) + 1) & 1), abort, wlim)) { ok = false; break; }
           tc_fence_after();
         }
         const uint32_t d = tmem + (sb ? kColS1 : kColS0);
         for (int ch = 0; ch < kChunks; ++ch) {
-          if ((rg.slot & 1) == 0 && !mbar_wait(bar(kBarKFull + (rg.slot >> 1)), rg.phase, abort)) { ok = false; break; }
+          if (rg.slot % kKGroup == 0 && !mbar_wait(bar(kBarKFull + rg.slot / kKGroup), rg.phase, abort, wlim)) {
+            ok = false;
+            break;
+          }
           const uint32_t a0 = sbase + kOffKRing + rg.slot * kKStageBytes;
           const uint32_t b0 = a0 + kBoxBytes;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_pair_ss(d, smem_desc_sw128(a0 + 32 * k, 16, 1024), smem_desc_sw128(b0 + 32 * k, 16, 1024), kIdescQK,
                         (ch | k) != 0);
-          if (rg.slot & 1) mma_commit_pair_mc(bar(kBarKEmpty + (rg.slot >> 1)), pmask);
+          if (rg.slot % kKGroup == kKGroup - 1) mma_commit_pair_mc(bar(kBarKEmpty + rg.slot / kKGroup), pmask);
           if (++rg.slot == kKStages) { rg.slot = 0; rg.phase ^= 1u; }
         }
         if (ok) mma_commit_pair_mc(bar(kBarSFull + sb), pmask);
@@ -434,24 +468,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       // P.V into the two 128-column output blocks
       for (int t = 0; t < u.T && ok; ++t) {
-        if (!mbar_wait(bar(kBarPFull), (uint32_t)(t & 1), abort)) { ok = false; break; }
+        if (!mbar_wait(bar(kBarPFull), (uint32_t)(t & 1), abort, wlim)) { ok = false; break; }
         tc_fence_after();
         const int ng = live_groups(u, t);
-        for (int g = 0; g < ng; ++g) {
-          if (!mbar_wait(bar(kBarVFull + rg.slot), rg.phase, abort)) { ok = false; break; }
+        for (int g = 0; g < ng && ok; ++g) {
           const uint32_t a0 = sbase + kOffP + g * kBoxBytes;
-          const uint32_t b0 = sbase + kOffVRing + rg.slot * kVStageBytes;
-#pragma unroll
           for (int j = 0; j < 2; ++j) {
+            if (!mbar_wait(bar(kBarVFull + rg.slot), rg.phase, abort, wlim)) { ok = false; break; }
+            const uint32_t b0 = sbase + kOffVRing + rg.slot * kVStageBytes;
             const uint32_t d = tmem + (j ? kColO1 : kColO0);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               mma_pair_ss(d, smem_desc_sw128(a0 + 32 * k, 16, 1024),
-                          smem_desc_sw128(b0 + 2 * j * kBoxBytes + 2048 * k, kBoxBytes, 1024), kIdescPV,
+                          smem_desc_sw128(b0 + 2048 * k, kBoxBytes, 1024), kIdescPV,
                           (t > 0 || g > 0 || k > 0) ? 1u : 0u);
+            mma_commit_pair_mc(bar(kBarVEmpty + rg.slot), pmask);
+            if (++rg.slot == kVStages) { rg.slot = 0; rg.phase ^= 1u; }
           }
-          mma_commit_pair_mc(bar(kBarVEmpty + rg.slot), pmask);
-          if (++rg.slot == kVStages) { rg.slot = 0; rg.phase ^= 1u; }
         }
         if (ok) mma_commit_pair_mc(bar(kBarOFull), pmask);
       }
@@ -482,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // after an aborted wait; later waits then return at once
     for (int t = 0; t < u.T; ++t) {
       const int sb = t & 1;
-      if (ok && !mbar_wait(bar(kBarSFull + sb), (uint32_t)((t >> 1) & 1), abort)) ok = false;
+      if (ok && !mbar_wait(bar(kBarSFull + sb), (uint32_t)((t >> 1) & 1), abort, wlim)) ok = false;
       tc_fence_after();
       float s[64];
       {
@@ -559,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       lsum = lsum * alpha + (ps0 + ps1);
       // the P buffer and the output accumulator are free once PV(t-1) is done
       if (t > 0) {
-        if (ok && !mbar_wait(bar(kBarOFull), (uint32_t)((t - 1) & 1), abort)) ok = false;
+        if (ok && !mbar_wait(bar(kBarOFull), (uint32_t)((t - 1) & 1), abort, wlim)) ok = false;
         tc_fence_after();
       }
       if (rescale) {
@@ -600,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the other splits -- all already past their keys -- have published
     // theirs, loads them by TMA and merges them into its own O in TMEM:
     //   O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
-    if (ok) ok = mbar_wait(bar(kBarOFull), (uint32_t)((u.T - 1) & 1), abort);
+    if (ok) ok = mbar_wait(bar(kBarOFull), (uint32_t)((u.T - 1) & 1), abort, wlim);
     tc_fence_after();
     lred[grp * 64 + rho] = lsum;
     const int rr = row0 + rho;
@@ -723,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           named_bar_sync(3, 128);
           if (threadIdx.x == sender0) {
-            if (c == 0 && !mbar_wait(bar(kBarXReady), 0u, abort)) ok = false;
+            if (c == 0 && !mbar_wait(bar(kBarXReady), 0u, abort, wlim)) ok = false;
             const uint32_t xbar = map_to_rank(bar(kBarXData + c), xpeer);
 #pragma unroll
             for (int e2 = 0; e2 < 2; ++e2) {
@@ -736,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         const int first_keeper = 128 + 128 * kp;
-        if (!mbar_wait_own(bar(kBarXData), 0u, abort)) ok = false;  // chunk 0 and the rows' (m, l)
+        if (!mbar_wait_own(bar(kBarXData), 0u, abort, wlim)) ok = false;  // chunk 0 and the rows' (m, l)
         const float mp = xml[2 * rho], lpeer = xml[2 * rho + 1];
         const float M = fmaxf(m_own, mp);
         const float w_own = m_own == -INFINITY ? 0.0f : exp2f(m_own - M);
@@ -749,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int d0 = 256 * sub + 128 * eta + 32 * c;
           uint32_t r[32];
           tmem_ld32(lane_addr + o_col + 32 * c, r);
-          if (c > 0 && !mbar_wait_own(bar(kBarXData + c), 0u, abort)) ok = false;
+          if (c > 0 && !mbar_wait_own(bar(kBarXData + c), 0u, abort, wlim)) ok = false;
           tmem_wait_ld();
           const unsigned char* row = smem + kOffStage32 + (d0 >> 5) * kBoxBytes + rho * 128;
           float f[32];
@@ -825,8 +858,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ld_acquire_gpu(cnt + 1) != (unsigned)(u.active - 1)) {
           const uint64_t t0 = global_timer_ns();
           while (ld_acquire_gpu(cnt + 1) != (unsigned)(u.active - 1)) {
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
-              atomicExch(abort, 1);
+            if (global_timer_ns() - t0 > wlim) {
+              atomicExch(abort, DDT_ERR_TIMEOUT);
               pub = false;
               break;
             }
@@ -862,7 +895,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float wo = step == 0 ? w_own : 1.0f;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-          if (!mbar_wait_own(bar(kBarEpi + c), (uint32_t)(step & 1), abort)) ok = false;
+          if (!mbar_wait_own(bar(kBarEpi + c), (uint32_t)(step & 1), abort, wlim)) ok = false;
           const int d0 = 256 * sub + 128 * eta + 32 * c;
           uint32_t r[32];
           tmem_ld32(lane_addr + o_col + 32 * c, r);
@@ -931,14 +964,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  // looked up once per process (a function-local static initialises once,
+  // whichever host thread gets here first)
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void* f = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -973,20 +1008,47 @@ static bool make_out_map(CUtensorMap* m, void* base, bool f32, int rank, uint64_
   return r == CUDA_SUCCESS;
 }
 
-// number of key splits: minimise an estimate of the makespan over 74 CTA pairs
-static int choose_splits(int B, int N, int H, int max_cache_len) {
+// Launch shape: how many key splits per request and whether the two splits
+// of a row tile share one cluster of 4 (merged through distributed shared
+// memory) or every CTA pair runs alone (merged through the workspace).
+struct LaunchPlan {
+  int splits;
+  int csize;
+};
+
+// Pair slots: how many CTA pairs can be resident at once when the kernel runs
+// in clusters of 2 (pairs4: in clusters of 4). Clusters must fit inside one
+// GPC, so clusters of 4 can leave SMs of a GPC idle that pairs would use.
+struct PairSlots {
+  int pairs2;
+  int pairs4;
+};
+
+// Makespan estimate in key tiles per pair (a tile of 256 keys is the unit):
+// waves of units over the resident pairs, each unit its tiles plus a fixed
+// start-up cost, plus the split merge (cheaper through distributed shared
+// memory than through the workspace).
+static LaunchPlan plan_launch(int B, int N, int H, int max_cache_len, PairSlots slots) {
   const int rowtiles = (N * H + 127) / 128;
-  const int units1 = B * rowtiles;
+  const long units1 = (long)B * rowtiles;
   const int tiles = (max_cache_len + N + kTileKeys - 1) / kTileKeys;
-  const int slots = 74;
-  int best = 1;
+  const double kStart = 0.6, kMergeDsmem = 0.4, kMergeWs = 1.2;
+  LaunchPlan best{1, 2};
   double best_t = 1e30;
-  for (int s = 1; s <= std::min(kMaxSplits, std::max(1, tiles)); ++s) {
+  auto consider = [&](int s, int csize, int slots, double merge) {
+    if (slots <= 0) return;
     const int per = (tiles + s - 1) / s;
-    const long units = (long)units1 * s;
+    const long units = units1 * s;
     const long waves = (units + slots - 1) / slots;
-    const double t = (double)waves * (per + 0.6) + (s > 1 ? 0.4 : 0.0);
-    if (t < best_t - 1e-9) { best_t = t; best = s; }
+    const double t = (double)waves * (per + kStart) + merge;
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best = LaunchPlan{s, csize};
+    }
+  };
+  for (int s = 1; s <= std::min(kMaxSplits, std::max(1, tiles)); ++s) {
+    if (s == 2) consider(s, 4, slots.pairs4, kMergeDsmem);
+    consider(s, 2, slots.pairs2, s > 1 ? kMergeWs : 0.0);
   }
   return best;
 }
@@ -1004,8 +1066,56 @@ static size_t counter_bytes(int B, int N, int H) {
   return ((size_t)B * rowtiles * 2 * 2 * 4 + 255) / 256 * 256;
 }
 
+// Resident pairs of this kernel on the current device, looked up once per
+// device (the kernel's shared-memory opt-in is set there first).
+static int device_pair_slots(tc::PairSlots* out) {
+  using namespace tc;
+  static std::mutex mu;
+  static bool done[kMaxDevices] = {};
+  static PairSlots slots[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DDT_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc) != cudaSuccess)
+      return DDT_ERR_CUDA;
+    int sms = sm_count();
+    PairSlots ps{sms / 2, 0};
+    for (int csize : {2, 4}) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)(csize * 64));
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = kSmemAlloc;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = (unsigned)csize;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel, &cfg) == cudaSuccess && n > 0) {
+        if (csize == 2) ps.pairs2 = n;
+        else ps.pairs4 = 2 * n;
+      } else {
+        (void)cudaGetLastError();
+      }
+    }
+    slots[dev] = ps;
+    done[dev] = true;
+  }
+  *out = slots[dev];
+  return DDT_OK;
+}
+
+static tc::LaunchPlan current_plan(int B, int N, int H, int max_cache_len) {
+  tc::PairSlots slots{74, 64};
+  (void)device_pair_slots(&slots);  // without a device: the B200's figures
+  return tc::plan_launch(B, N, H, max_cache_len, slots);
+}
+
 size_t tc_attn_workspace_bytes(int B, int N, int H, int max_cache_len) {
-  const int s = tc::choose_splits(B, N, H, max_cache_len);
+  const int s = current_plan(B, N, H, max_cache_len).splits;
   size_t bytes = tc::ws_header();
   if (s > 1) {
     const size_t rows = (size_t)B * N * H;
@@ -1014,9 +1124,10 @@ size_t tc_attn_workspace_bytes(int B, int N, int H, int max_cache_len) {
   return bytes;
 }
 
-int launch_attn_tc(const AttnParams& a, int64_t kv_rows, int max_cache_len, void* workspace, size_t workspace_bytes,
+int launch_attn_tc(const AttnParams& a, int max_cache_len, void* workspace, size_t workspace_bytes,
                    cudaStream_t stream) {
   using namespace tc;
+  const int64_t kv_rows = a.kv_rows;
   if (a.N > 32 * kMaxW) return DDT_ERR_UNSUPPORTED;
   if (kv_rows > 0x7fffffffLL) return DDT_ERR_UNSUPPORTED;
   const long long q_rows = (long long)a.B * a.N * a.H;
@@ -1033,11 +1144,14 @@ int launch_attn_tc(const AttnParams& a, int64_t kv_rows, int max_cache_len, void
   p.H = a.H;
   p.W = a.W;
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  p.splits = choose_splits(a.B, a.N, a.H, max_cache_len);
+  const LaunchPlan plan = current_plan(a.B, a.N, a.H, max_cache_len);
+  p.splits = plan.splits;
   p.rowtiles = (a.N * a.H + 127) / 128;
   p.out_dtype = a.out_dtype;
   p.out = a.out;
   p.lse = a.lse;
+  p.dev_status = a.dev_status;
+  p.kv_rows = kv_rows;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   p.abort = reinterpret_cast<int*>(ws);
   if (p.splits > 1) {
@@ -1048,11 +1162,12 @@ int launch_attn_tc(const AttnParams& a, int64_t kv_rows, int max_cache_len, void
     p.part_ml = reinterpret_cast<float*>(ws + ws_header() + cb + (size_t)p.splits * rows * kDL * 4);
   }
   if (workspace_bytes < tc_attn_workspace_bytes(a.B, a.N, a.H, max_cache_len)) return DDT_ERR_INVALID_ARG;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc) != cudaSuccess)
-      return DDT_ERR_CUDA;
-    attr_set = true;
+  p.wait_ns = wait_limit_ns();
+  // the shared-memory opt-in is a per-device function attribute: set (with
+  // the pair slots) once on every device the library launches on
+  {
+    PairSlots slots;
+    if (device_pair_slots(&slots) != DDT_OK) return DDT_ERR_CUDA;
   }
   CUtensorMap tout, tpart;
   memset(&tpart, 0, sizeof(tpart));
@@ -1081,7 +1196,7 @@ int launch_attn_tc(const AttnParams& a, int64_t kv_rows, int max_cache_len, void
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, attn_tc_kernel, tq, tkv, tout, tpart, p);
   };
-  if (p.splits == 2) {
+  if (p.splits == 2 && plan.csize == 4) {
     if (launch(4) == cudaSuccess) return DDT_OK;
     (void)cudaGetLastError();  // clusters of 4 not schedulable here: pairs + workspace merge
   }

@@ -18,18 +18,21 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libddt.so")
 
-DDT_OK, DDT_ERR_INVALID_ARG, DDT_ERR_UNSUPPORTED, DDT_ERR_CAPACITY, DDT_ERR_INPUT, DDT_ERR_CUDA, DDT_ERR_TIMEOUT = range(7)
+(DDT_OK, DDT_ERR_INVALID_ARG, DDT_ERR_UNSUPPORTED, DDT_ERR_CAPACITY, DDT_ERR_INPUT, DDT_ERR_CUDA, DDT_ERR_TIMEOUT,
+ DDT_ERR_BOUNDS) = range(8)
 DDT_F32, DDT_BF16 = 0, 1
 
 EXPORTS = (
     "ddt_status_string",
     "ddt_version",
+    "ddt_set_wait_limit_ns",
     "ddt_build_tree",
     "ddt_verify_attn_workspace_size",
     "ddt_verify_attn",
     "ddt_accept_compact_workspace_size",
     "ddt_accept_compact",
     "ddt_accept_compact_noalloc",
+    "ddt_accept_compact_lmhead",
     "ddt_drafter_topk",
 )
 
@@ -57,21 +60,26 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.ddt_status_string.argtypes = [i32]
     lib.ddt_version.restype = i32
     lib.ddt_version.argtypes = []
+    lib.ddt_set_wait_limit_ns.restype = ctypes.c_uint64
+    lib.ddt_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.ddt_build_tree.restype = i32
     lib.ddt_build_tree.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.ddt_verify_attn_workspace_size.restype = sz
     lib.ddt_verify_attn_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i32]
     lib.ddt_verify_attn.restype = i32
     lib.ddt_verify_attn.argtypes = [vp, vp, i64, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32, i32, i32,
-                                    vp, vp, vp, sz, vp]
+                                    vp, vp, vp, vp, sz, vp]
     lib.ddt_accept_compact_workspace_size.restype = sz
     lib.ddt_accept_compact_workspace_size.argtypes = [i32, i32, i32]
     lib.ddt_accept_compact.restype = i32
-    lib.ddt_accept_compact.argtypes = [vp, i32, i32, vp, vp, vp, i32, i32, vp, i32, i32, i32, i64, vp, vp, vp,
-                                       vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.ddt_accept_compact.argtypes = [vp, i32, i32, vp, vp, vp, i32, i32, vp, i64, i32, i32, i32, i64, vp, vp,
+                                       vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.ddt_accept_compact_noalloc.restype = i32
-    lib.ddt_accept_compact_noalloc.argtypes = [vp, i32, i32, vp, vp, vp, i32, i32, vp, i32, i32, i32, i64, vp, vp,
-                                               vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.ddt_accept_compact_noalloc.argtypes = [vp, i32, i32, vp, vp, vp, i32, i32, vp, i64, i32, i32, i32, i64, vp,
+                                               vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.ddt_accept_compact_lmhead.restype = i32
+    lib.ddt_accept_compact_lmhead.argtypes = [vp, vp, i32, i32, vp, vp, vp, i32, i32, vp, i64, i32, i32, i32, i64,
+                                              vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.ddt_drafter_topk.restype = i32
     lib.ddt_drafter_topk.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
     if path is None:
@@ -85,6 +93,13 @@ def status_string(status: int) -> str:
 
 def version() -> int:
     return int(load().ddt_version())
+
+
+def set_wait_limit_ns(ns: int) -> int:
+    """ddt_set_wait_limit_ns: wall-clock limit of the kernels' bounded waits
+    for calls issued from now on (0: the 2 s default). Returns the previous
+    limit."""
+    return int(load().ddt_set_wait_limit_ns(int(ns)))
 
 
 # ---------------------------------------------------------------------------
@@ -234,9 +249,11 @@ def verify_attn(q: torch.Tensor, kv: torch.Tensor, cache_off: torch.Tensor, cach
                 mask: torch.Tensor, n_nodes: torch.Tensor, d_l: int, d_r: int, scale: float, max_cache_len: int,
                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, want_lse: bool = True,
                 out_dtype: Optional[torch.dtype] = None, workspace: Optional[torch.Tensor] = None,
-                stream=None):
+                status: Optional[torch.Tensor] = None, stream=None):
     """ddt_verify_attn. q [B, N, H, d_qk], kv [rows, d_qk] (same dtype, f32 or
     bf16), cache_off [B] i64, cache_len / n_nodes [B] i32, mask [B, N, W] i32.
+    status (optional, [B] i32) receives each request's device status (DDT_OK,
+    or DDT_ERR_BOUNDS for rows outside the pool).
     Returns (out [B, N, H, d_l], lse [B, N, H] f32 or None)."""
     B, N, H, d_qk = q.shape
     assert d_qk == d_l + d_r
@@ -256,14 +273,17 @@ def verify_attn(q: torch.Tensor, kv: torch.Tensor, cache_off: torch.Tensor, cach
         lse = torch.empty(B, N, H, dtype=torch.float32, device=q.device)
     if lse is not None:
         _check(lse, "lse", torch.float32, (B, N, H))
+    if status is not None:
+        _check(status, "status", torch.int32, (B,))
     need = verify_attn_workspace_size(B, N, H, d_l, d_r, max_cache_len, q.dtype)
     if workspace is None and need > 0:
         workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)  # status word must start at 0
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    with _device(q, kv, cache_off, cache_len, mask, n_nodes, out, lse, workspace, stream=stream):
+    with _device(q, kv, cache_off, cache_len, mask, n_nodes, out, lse, status, workspace, stream=stream):
         st = load().ddt_verify_attn(_ptr(q), _ptr(kv), kv.shape[0], _ptr(cache_off), _ptr(cache_len), _ptr(mask),
                                     _ptr(n_nodes), B, N, H, d_l, d_r, float(scale), int(max_cache_len), _dt(q),
-                                    _dt(out), _ptr(out), _ptr(lse), _ptr(workspace), wbytes, _stream(stream))
+                                    _dt(out), _ptr(out), _ptr(lse), _ptr(status), _ptr(workspace), wbytes,
+                                    _stream(stream))
     _raise("ddt_verify_attn", st)
     return out, lse
 
@@ -300,7 +320,8 @@ def accept_compact(logits: torch.Tensor, node_tok: torch.Tensor, parent: torch.T
     with _device(logits, node_tok, parent, n_nodes, kv, cache_off, cache_len, cache_cap,
                  workspace, *out.values(), stream=stream):
         st = load().ddt_accept_compact(_ptr(logits), _dt(logits), V, _ptr(node_tok), _ptr(parent), _ptr(n_nodes),
-                                       B, N, _ptr(kv), _dt(kv), row_elems, n_layers, layer_stride_rows,
+                                       B, N, _ptr(kv), kv.numel() // row_elems, _dt(kv), row_elems, n_layers,
+                                       layer_stride_rows,
                                        _ptr(cache_off), _ptr(cache_len), _ptr(cache_cap), _ptr(out["am"]),
                                        _ptr(out["acc_len"]), _ptr(out["acc_nodes"]), _ptr(out["out_tok"]),
                                        _ptr(out["bonus"]), _ptr(out["status"]), _ptr(workspace),
@@ -344,10 +365,51 @@ def accept_compact_noalloc(logits: torch.Tensor, node_tok: torch.Tensor, parent:
     with _device(logits, node_tok, parent, n_nodes, kv, cache_off, cache_len, cache_cap,
                  *out.values(), stream=stream):
         st = load().ddt_accept_compact_noalloc(_ptr(logits), _dt(logits), V, _ptr(node_tok), _ptr(parent),
-                                               _ptr(n_nodes), B, N, _ptr(kv), _dt(kv), kv.shape[-1], n_layers,
+                                               _ptr(n_nodes), B, N, _ptr(kv), kv.numel() // kv.shape[-1], _dt(kv),
+                                               kv.shape[-1], n_layers,
                                                layer_stride_rows, _ptr(cache_off), _ptr(cache_len),
                                                _ptr(cache_cap), _ptr(out["am"]), _ptr(out["acc_len"]),
                                                _ptr(out["acc_nodes"]), _ptr(out["out_tok"]), _ptr(out["bonus"]),
                                                _ptr(out["status"]), _stream(stream))
     _raise("ddt_accept_compact_noalloc", st)
+    return out
+
+
+def accept_compact_lmhead(hidden: torch.Tensor, w_vocab: torch.Tensor, node_tok: torch.Tensor, parent: torch.Tensor,
+                          n_nodes: torch.Tensor, kv: torch.Tensor, cache_off: torch.Tensor, cache_len: torch.Tensor,
+                          cache_cap: torch.Tensor, n_layers: int = 1, layer_stride_rows: int = 0,
+                          out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """ddt_accept_compact_lmhead: accept_compact with the target's LM head
+    folded into the argmax. hidden [B, N, d] bf16 (the verify rows' final
+    hidden states), w_vocab [V, d] bf16; the logits are never materialised.
+    Returns the same tensors as accept_compact."""
+    B, N, d = hidden.shape
+    V = w_vocab.shape[0]
+    _check(hidden, "hidden", torch.bfloat16)
+    _check(w_vocab, "w_vocab", torch.bfloat16, (V, d))
+    _check(node_tok, "node_tok", torch.int32, (B, N))
+    _check(parent, "parent", torch.int32, (B, N))
+    _check(n_nodes, "n_nodes", torch.int32, (B,))
+    _check(kv, "kv", (torch.float32, torch.bfloat16))
+    _check(cache_off, "cache_off", torch.int64, (B,))
+    _check(cache_len, "cache_len", torch.int32, (B,))
+    _check(cache_cap, "cache_cap", torch.int32, (B,))
+    dev = hidden.device
+    if out is None:
+        out = alloc_accept(B, N, dev)
+    _check_out(out, _accept_out_spec(B, N))
+    need = accept_compact_workspace_size(B, N, V)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)  # row keys start at 0
+    _check(workspace, "workspace", None)
+    row_elems = kv.shape[-1]
+    with _device(hidden, w_vocab, node_tok, parent, n_nodes, kv, cache_off, cache_len, cache_cap, workspace,
+                 *out.values(), stream=stream):
+        st = load().ddt_accept_compact_lmhead(
+            _ptr(hidden), _ptr(w_vocab), d, V, _ptr(node_tok), _ptr(parent), _ptr(n_nodes), B, N, _ptr(kv),
+            kv.numel() // row_elems, _dt(kv), row_elems, n_layers, layer_stride_rows, _ptr(cache_off),
+            _ptr(cache_len), _ptr(cache_cap), _ptr(out["am"]), _ptr(out["acc_len"]), _ptr(out["acc_nodes"]),
+            _ptr(out["out_tok"]), _ptr(out["bonus"]), _ptr(out["status"]), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream))
+    _raise("ddt_accept_compact_lmhead", st)
     return out

@@ -272,7 +272,7 @@ def target_logits(shape: Shape, parent: np.ndarray, node_tok: np.ndarray, n_node
 
 
 def lmhead_inputs(shape: Shape, parent: np.ndarray, node_tok: np.ndarray, n_nodes: np.ndarray, d_model: int,
-                  requests: Optional[list] = None):
+                  requests: Optional[list] = None, w_vocab: Optional[np.ndarray] = None):
     """Inputs of the target's LM head for every verify row: the head's weights
     w_vocab [V, d_model] (one row per token, N(0, 1 / d_model), so logits have
     unit scale like target_logits') and final hidden states hidden
@@ -280,13 +280,28 @@ def lmhead_inputs(shape: Shape, parent: np.ndarray, node_tok: np.ndarray, n_node
     a uniformly chosen child's token t gets the acceptance bias: hidden row i
     moves by bias * w_t / |w_t|^2 (w_t as stored), which raises its logit for t
     by the bias before rounding. Returns (hidden, w_vocab, planted [B, N] i32:
-    the planted token, or -1), hidden and w_vocab in the shape's dtype."""
+    the planted token, or -1), hidden and w_vocab in the shape's dtype.
+    ``w_vocab`` (optional, [V, d_model] as stored): use this head instead of
+    drawing one (several workloads against one large head)."""
     s = shape
     reqs = list(range(s.B)) if requests is None else list(requests)
-    w32 = (_rng(s.seed, 7).standard_normal((s.V, d_model), dtype=np.float32) /
-           np.float32(math.sqrt(d_model))).astype(np.float32)
-    w = _store(w32, s.dtype)
-    wv = w.astype(np.float64) if s.dtype == "f32" else bf16_bits_to_f32(w).astype(np.float64)
+    # drawn in row blocks (the same stream as one draw) so a Kimi-sized head
+    # (163840 x 7168) never needs more than a block of float32 temporaries
+    if w_vocab is not None:
+        w = w_vocab
+        assert w.shape == (s.V, d_model)
+    else:
+        rw = _rng(s.seed, 7)
+        w = np.empty((s.V, d_model), np.float32 if s.dtype == "f32" else np.uint16)
+        scale = np.float32(math.sqrt(d_model))
+        for v0 in range(0, s.V, 8192):
+            blk = rw.standard_normal((min(8192, s.V - v0), d_model), dtype=np.float32) / scale
+            w[v0:v0 + len(blk)] = _store(blk.astype(np.float32), s.dtype)
+
+    def wv(t):  # row t of the head as stored, in float64
+        row = w[t:t + 1]
+        return (row.astype(np.float64) if s.dtype == "f32" else bf16_bits_to_f32(row).astype(np.float64))[0]
+
     hidden = np.empty((len(reqs), s.N, d_model), w.dtype)
     planted = np.full((len(reqs), s.N), -1, np.int32)
     for j, b in enumerate(reqs):
@@ -302,7 +317,8 @@ def lmhead_inputs(shape: Shape, parent: np.ndarray, node_tok: np.ndarray, n_node
             if kids and u < s.accept_p:
                 c = kids[min(len(kids) - 1, int(pick * len(kids)))]
                 t = int(node_tok[j, c])
-                h[i] += s.accept_bias * wv[t] / float(wv[t] @ wv[t])
+                wt = wv(t)
+                h[i] += s.accept_bias * wt / float(wt @ wt)
                 planted[j, i] = t
         hidden[j] = _store(h.astype(np.float32), s.dtype)
     return hidden, w, planted

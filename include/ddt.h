@@ -34,8 +34,8 @@
  *   - The return value is a ddt_status. Host-side argument checks (null
  *     pointers, sizes, unsupported shapes or dtypes) are synchronous and
  *     launch nothing. A failed launch returns DDT_ERR_CUDA.
- *   - Device-side preconditions (bad drafter log-probs, cache capacity) never
- *     trap: the kernel writes a ddt_status value to dev_status[b] (when
+ *   - Device-side preconditions (bad drafter log-probs, cache capacity, a
+ *     request's rows inside the pool) never trap: the kernel writes a ddt_status value to dev_status[b] (when
  *     dev_status is non-null, else the problem is only visible through the
  *     padded outputs) and skips that request as documented per call.
  *   - Shapes: B requests, D drafter depth, K top-k, N verify rows per request
@@ -71,7 +71,8 @@ typedef enum {
   DDT_ERR_CAPACITY = 3,    /* device: cache_len + n_nodes > cache_cap         */
   DDT_ERR_INPUT = 4,       /* device: drafter log-probs violate preconditions */
   DDT_ERR_CUDA = 5,        /* a CUDA launch or driver call failed             */
-  DDT_ERR_TIMEOUT = 6      /* device: a bounded intra-kernel wait gave up     */
+  DDT_ERR_TIMEOUT = 6,     /* device: a bounded intra-kernel wait gave up     */
+  DDT_ERR_BOUNDS = 7       /* device: a request's rows fall outside the pool  */
 } ddt_status;
 
 typedef enum { DDT_F32 = 0, DDT_BF16 = 1 } ddt_dtype;
@@ -81,6 +82,17 @@ DDT_API const char* ddt_status_string(int status);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 DDT_API int ddt_version(void);
+
+/*
+ * ddt_set_wait_limit_ns -- wall-clock limit of every bounded wait inside the
+ * library's kernels (a barrier a pipeline stage waits on, a counter another
+ * CTA must advance). A wait that runs past it gives up: the kernel stores
+ * DDT_ERR_TIMEOUT in the call's workspace status word and returns instead of
+ * spinning. Process-wide; read when a kernel is launched, so it applies to
+ * calls issued after this one. 0 restores the default (2 s); values below
+ * 1 ms are raised to 1 ms. Returns the previous limit. Host only, thread-safe.
+ */
+DDT_API uint64_t ddt_set_wait_limit_ns(uint64_t ns);
 
 /*
  * ddt_drafter_topk -- the drafter's per-depth proposals from its logits: for
@@ -179,7 +191,10 @@ DDT_API int ddt_build_tree(const float* logp, const int32_t* tok, const int32_t*
  *   max_cache_len (host): an upper bound on every cache_len[b]; it sizes the
  *             launch and the workspace. kv_rows (host): rows in the pool.
  * Outputs (device): out [B][N][H][d_l] out_dtype; lse [B][N][H] float32
- *   (nullable).
+ *   (nullable); dev_status [B] int32 (nullable): DDT_OK, or DDT_ERR_BOUNDS
+ *   when cache_off[b] + cache_len[b] + n_nodes[b] > kv_rows, a value is
+ *   negative, or n_nodes[b] > N -- that request then reads nothing and all
+ *   its rows are written as pad rows.
  * Supported: in_dtype F32 (CUDA-core kernel, any d_l, d_r with d_qk <= 1024)
  *   and BF16 with (d_l, d_r) = (512, 64) (tensor-core kernel); out_dtype F32
  *   or BF16. Accumulation is float32 throughout. The bf16 kernel rounds the
@@ -188,18 +203,18 @@ DDT_API int ddt_build_tree(const float* logp, const int32_t* tok, const int32_t*
  *   memory, 256-byte aligned (may be null when that size is 0). Its first 256
  *   bytes are a device status word that must be zero before the first call
  *   (zero the buffer once after allocating it). Every wait inside the bf16
- *   kernel is bounded (about 2 s); if one expires the kernel stores
- *   DDT_ERR_TIMEOUT there and returns, and later calls with that workspace
- *   return at once until the caller zeroes it again. When the launch splits
+ *   kernel is bounded (ddt_set_wait_limit_ns, default 2 s); if one expires the
+ *   kernel stores DDT_ERR_TIMEOUT there, writes zeros for the rows it could
+ *   not finish and returns, and later calls with that workspace give up their
+ *   waits at once until the caller zeroes it again. When the launch splits
  *   the keys (the size above 256), the next bytes are per-row-tile arrival
  *   counters that must also start at zero; each call leaves them at zero
  *   (except after a timeout: zero the whole workspace then). The rest holds
  *   per-split partial results; its contents do not matter. Calls that share
  *   a workspace must not overlap in time.
- * Preconditions: cache_off[b] + cache_len[b] + n_nodes[b] <= kv_rows,
- *   cache_len[b] <= max_cache_len, n_nodes[b] <= N, none negative. The bf16
- *   kernel reads the pool through TMA, which returns zeros for rows beyond
- *   kv_rows. The f32 kernel does not check these bounds.
+ * Pool bounds: both kernels check, per request, that its rows lie in the
+ *   pool (see dev_status) before reading any. cache_len[b] <= max_cache_len
+ *   is a precondition of speed only: the launch is sized for max_cache_len.
  * Errors: DDT_ERR_INVALID_ARG (nulls, sizes, workspace too small or
  *   misaligned, kv / q not 16-byte aligned for bf16), DDT_ERR_UNSUPPORTED.
  */
@@ -210,7 +225,7 @@ DDT_API int ddt_verify_attn(const void* q, const void* kv, int64_t kv_rows, cons
                     const int32_t* cache_len, const uint32_t* mask, const int32_t* n_nodes,
                     int B, int N, int H, int d_latent, int d_rope, float scale,
                     int max_cache_len, int in_dtype, int out_dtype, void* out, float* lse,
-                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
+                    int32_t* dev_status, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * ddt_accept_compact -- greedy accept walk, then latent-KV compaction.
@@ -232,28 +247,29 @@ DDT_API int ddt_verify_attn(const void* q, const void* kv, int64_t kv_rows, cons
  *   cache_len[b] += a + 1.
  *
  * Inputs (device): logits [B][N][V] logits_dtype, finite; node_tok, parent
- *   [B][N] int32 and n_nodes [B] (from ddt_build_tree); kv pool with rows of
- *   row_elems elements of kv_dtype (row_elems * element size a multiple of
- *   4 bytes); cache_off [B] int64; cache_cap [B] int32 (rows owned by b).
+ *   [B][N] int32 and n_nodes [B] (from ddt_build_tree); kv pool of kv_rows
+ *   (host value: every layer's rows) rows of row_elems elements of kv_dtype
+ *   (row_elems * element size a multiple of 4 bytes); cache_off [B] int64;
+ *   cache_cap [B] int32 (rows owned by b).
  * In/out: cache_len [B] int32 (advanced by a + 1).
  * Outputs (device): am [B][N] int32 (nullable; -1 on pad rows), acc_len [B],
  *   acc_nodes [B][N] (path, -1 padded), out_tok [B][N] (-1 padded), bonus [B].
- *   dev_status [B] (nullable): DDT_OK; DDT_ERR_CAPACITY when cache_len[b] +
- *   n_nodes[b] > cache_cap[b] (request skipped: acc_len 0, bonus -1, nothing
- *   copied, cache_len unchanged). Requests with n_nodes[b] == 0 are skipped
- *   the same way with DDT_OK.
+ *   dev_status [B] (nullable): DDT_OK; DDT_ERR_INPUT when n_nodes[b] > N;
+ *   DDT_ERR_BOUNDS when a row the compaction may touch,
+ *   l*layer_stride_rows + cache_off[b] + [cache_len[b], cache_len[b] +
+ *   n_nodes[b]) for some layer l, lies outside [0, kv_rows);
+ *   DDT_ERR_CAPACITY when cache_len[b] + n_nodes[b] > cache_cap[b]. Each of
+ *   these skips the request: acc_len 0, bonus -1, nothing copied, cache_len
+ *   unchanged. Requests with n_nodes[b] == 0 are skipped the same way with
+ *   DDT_OK.
  * workspace: ddt_accept_compact_workspace_size(B, N, V) bytes, 256-byte
- *   aligned: a 256-byte status word, then one 8-byte running argmax key per
- *   row (B * N, rounded up to 256 bytes). All of it must be zero before the
+ *   aligned: 256 reserved bytes, then one 8-byte running argmax key per row
+ *   (B * N, rounded up to 256 bytes). All of it must be zero before the
  *   first call -- zero the buffer once after allocating it; every call
- *   leaves it at zero again. Every wait inside the kernels is bounded (about
- *   2 s); if one expires the status word holds DDT_ERR_TIMEOUT and the
- *   outputs are not valid (zero the workspace before reusing it). Calls that
- *   share a workspace must not overlap on the GPU.
- * Preconditions the library cannot check (it is not told the pool's size):
- *   every row the compaction touches, l*layer_stride_rows + cache_off[b] +
- *   [cache_len[b], cache_len[b] + n_nodes[b]), lies inside the kv pool, and
- *   the layers and requests own disjoint rows. The kernels do not check them.
+ *   leaves it at zero again. Nothing in these kernels waits on another CTA.
+ *   Calls that share a workspace must not overlap on the GPU.
+ * Precondition the library cannot check: the layers and requests own
+ *   disjoint rows.
  * Runs as two kernels: the logits stream once with 16-byte loads, each warp
  *   owning contiguous 2048-entry slices of the rows (two 512-thread CTAs per
  *   SM; row maxima published by 64-bit atomic max), then one CTA per request
@@ -263,11 +279,54 @@ DDT_API size_t ddt_accept_compact_workspace_size(int B, int N, int V);
 
 DDT_API int ddt_accept_compact(const void* logits, int logits_dtype, int V, const int32_t* node_tok,
                        const int32_t* parent, const int32_t* n_nodes, int B, int N, void* kv,
-                       int kv_dtype, int row_elems, int n_layers, int64_t layer_stride_rows,
+                       int64_t kv_rows, int kv_dtype, int row_elems, int n_layers, int64_t layer_stride_rows,
                        const int64_t* cache_off, int32_t* cache_len, const int32_t* cache_cap,
                        int32_t* am, int32_t* acc_len, int32_t* acc_nodes, int32_t* out_tok,
                        int32_t* bonus, int32_t* dev_status, void* workspace,
                        size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * ddt_accept_compact_lmhead -- ddt_accept_compact with the target's LM head
+ * folded into the argmax: the verify rows' greedy tokens come straight from
+ * their final hidden states and the head's weights, and the logits are never
+ * written to memory.
+ *
+ * Passage: first page, "What the Message Actually Says" (the greedy token of
+ * a verify row is the argmax of the target's logits, checked exactly);
+ * "the_validation_pivot", "Assumptions Embedded in This Message" (the head
+ * maps the final hidden state, 7168 wide on Kimi K2.6, to the vocabulary).
+ *
+ * Definition: am[b][i] = the lowest v among those with the largest
+ *   z[v] = sum_c hidden[b][i][c] * w_vocab[v][c]; then the walk, outputs and
+ *   compaction of ddt_accept_compact. z is evaluated in float32: every
+ *   bf16 x bf16 product is exact, and a product passes through at most
+ *   15 + ceil(d_model / 16) float32 roundings (16-product tensor-core steps
+ *   added in sequence). Where several tokens lie within that rounding of
+ *   the maximum, any of them may be picked.
+ * Inputs (device): hidden [B][N][d_model] bf16 (rows i >= n_nodes[b] are
+ *   read but ignored), w_vocab [V][d_model] bf16 (one row per token); both
+ *   16-byte aligned, d_model a multiple of 8. The other arguments, the
+ *   outputs and the device statuses are ddt_accept_compact's, with one more
+ *   status: DDT_ERR_TIMEOUT in dev_status[b] (and in the workspace's first
+ *   word) when a bounded wait inside the head kernel gave up -- nothing is
+ *   accepted then; zero the workspace before reusing it.
+ * workspace: ddt_accept_compact_workspace_size(B, N, V) bytes, zeroed once
+ *   after allocation, left zeroed by every call that does not time out.
+ * Runs as two kernels: a persistent 2-CTA tcgen05 GEMM with the vocabulary
+ *   as M (256 head rows per CTA pair, streamed by TMA, read once per pass of
+ *   up to 512 verify rows) and the verify rows as N, whose epilogue reduces
+ *   every tensor-memory tile to per-row (max, lowest index) keys; then the
+ *   walk and compaction kernel of ddt_accept_compact.
+ * Errors: ddt_accept_compact's, and DDT_ERR_UNSUPPORTED for d_model not a
+ *   multiple of 8 or misaligned hidden / w_vocab.
+ */
+DDT_API int ddt_accept_compact_lmhead(const void* hidden, const void* w_vocab, int d_model, int V,
+                                      const int32_t* node_tok, const int32_t* parent, const int32_t* n_nodes,
+                                      int B, int N, void* kv, int64_t kv_rows, int kv_dtype, int row_elems,
+                                      int n_layers, int64_t layer_stride_rows, const int64_t* cache_off,
+                                      int32_t* cache_len, const int32_t* cache_cap, int32_t* am, int32_t* acc_len,
+                                      int32_t* acc_nodes, int32_t* out_tok, int32_t* bonus, int32_t* dev_status,
+                                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * ddt_accept_compact_noalloc -- ddt_accept_compact without a workspace.
@@ -278,7 +337,7 @@ DDT_API int ddt_accept_compact(const void* logits, int logits_dtype, int V, cons
  * the host application, or a latency-critical decode loop that must not call
  * cudaMalloc (which can synchronise the device). This entry point takes the
  * same arguments as ddt_accept_compact minus the workspace and allocates
- * nothing: its scratch (status word and per-row argmax keys) lives in one
+ * nothing: its scratch (reserved header and per-row argmax keys) lives in one
  * fixed 4 MiB array inside the library, which every GPU
  * that loads the library keeps until the process exits.
  *
@@ -288,7 +347,8 @@ DDT_API int ddt_accept_compact(const void* logits, int logits_dtype, int V, cons
  *   DDT_ERR_UNSUPPORTED without launching anything.
  * Set-up: the first call on each device looks up the array's device address
  *   (with that device current); make that first call before any stream
- *   capture.
+ *   capture. The address is kept for the life of the process, so do not use
+ *   the library across cudaDeviceReset.
  * Sharing: every call on every stream uses the same array, which keeps what
  *   the last call left in it. Each call first clears the counters it needs on
  *   its own stream; calls that overlap on the GPU race on the array and give
@@ -298,7 +358,7 @@ DDT_API int ddt_accept_compact(const void* logits, int logits_dtype, int V, cons
  */
 DDT_API int ddt_accept_compact_noalloc(const void* logits, int logits_dtype, int V, const int32_t* node_tok,
                                        const int32_t* parent, const int32_t* n_nodes, int B, int N, void* kv,
-                                       int kv_dtype, int row_elems, int n_layers, int64_t layer_stride_rows,
+                                       int64_t kv_rows, int kv_dtype, int row_elems, int n_layers, int64_t layer_stride_rows,
                                        const int64_t* cache_off, int32_t* cache_len, const int32_t* cache_cap,
                                        int32_t* am, int32_t* acc_len, int32_t* acc_nodes, int32_t* out_tok,
                                        int32_t* bonus, int32_t* dev_status, cudaStream_t stream);

@@ -353,10 +353,12 @@ def drafter_topk(logits, K):
 # ---------------------------------------------------------------------------
 
 
-def lmhead_logits(hidden, w_vocab):
+def lmhead_logits(hidden, w_vocab, v_chunk=None):
     """The target's logits from its final hidden states: z[r][v] = sum over c of
     hidden[r][c] * w_vocab[v][c], in float64 from the stored values (bf16
-    already widened exactly).
+    already widened exactly). ``v_chunk``: evaluate the product one slice of
+    the vocabulary at a time (each logit is still one float64 dot product;
+    only the memory of the widened head is bounded).
 
     Source: AR page, "What the Message Actually Says" (the greedy token of a
     verify row is the argmax of the target's logits, checked exactly);
@@ -364,8 +366,12 @@ def lmhead_logits(hidden, w_vocab):
     hidden size 7168; the tests' tiny model: hidden 64, vocabulary 400).
     hidden: [R, d]; w_vocab: [V, d] (one row per token). Returns [R, V]."""
     h = np.asarray(hidden, dtype=np.float64)
-    w = np.asarray(w_vocab, dtype=np.float64)
-    return h @ w.T
+    V = np.shape(w_vocab)[0]
+    step = V if v_chunk is None else int(v_chunk)
+    z = np.empty((h.shape[0], V), np.float64)
+    for v0 in range(0, V, step):
+        z[:, v0:v0 + step] = h @ np.asarray(w_vocab[v0:v0 + step], dtype=np.float64).T
+    return z
 
 
 def lmhead_argmax(hidden, w_vocab):
@@ -389,24 +395,28 @@ def lmhead_argmax(hidden, w_vocab):
 LMHEAD_U = 2.0 ** -22
 
 
-def lmhead_f32_error_bound(hidden, w_vocab, depth=None):
+def lmhead_f32_error_bound(hidden, w_vocab, depth=None, v_chunk=None):
     """Per row, the largest over v of the float32 evaluation bound above, for
     at most ``depth`` roundings per product (default d - 1: any order).
     Returns [R] float64."""
     h = np.abs(np.asarray(hidden, dtype=np.float64))
-    w = np.abs(np.asarray(w_vocab, dtype=np.float64))
     n = max(h.shape[1] - 1, 0) if depth is None else int(depth)
     gamma = n * LMHEAD_U / (1.0 - n * LMHEAD_U)
-    return gamma * (h @ w.T).max(axis=-1)
+    V = np.shape(w_vocab)[0]
+    step = V if v_chunk is None else int(v_chunk)
+    top = np.zeros(h.shape[0], np.float64)
+    for v0 in range(0, V, step):
+        top = np.maximum(top, (h @ np.abs(np.asarray(w_vocab[v0:v0 + step], dtype=np.float64)).T).max(axis=-1))
+    return gamma * top
 
 
-def lmhead_valid_argmax(hidden, w_vocab, depth=None):
+def lmhead_valid_argmax(hidden, w_vocab, depth=None, v_chunk=None):
     """The tokens a float32 evaluation within the bound may pick for each row:
     every v with z[v] >= max(z) - 2 * bound (a pick g has z[g] >= z32[g] - bound
     >= z32[am] - bound >= z[am] - 2 * bound). Returns (am [R] int32, valid: a
     list of R sorted int32 arrays, each holding am)."""
-    z = lmhead_logits(hidden, w_vocab)
-    bound = lmhead_f32_error_bound(hidden, w_vocab, depth)
+    z = lmhead_logits(hidden, w_vocab, v_chunk)
+    bound = lmhead_f32_error_bound(hidden, w_vocab, depth, v_chunk)
     am = np.argmax(z, axis=-1).astype(np.int32)
     top = z.max(axis=-1)
     valid = [np.flatnonzero(z[r] >= top[r] - 2.0 * bound[r]).astype(np.int32) for r in range(z.shape[0])]

@@ -7,6 +7,8 @@ import subprocess
 import sys
 import time
 
+import numpy as np
+
 import bench
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -42,16 +44,29 @@ def test_reference_line_on_the_tiny_workload():
 def test_cpu_baseline_reports_all_threads_and_one():
     import argparse
 
-    import oracle
     from ddtree_speculative_decode_b200 import synth
     shape = synth.tiny_f32()
-    x = synth.make_step(shape)
-    tree = oracle.build_tree(x.logp, x.tok, x.root_tok, x.cache_len, shape.N)
-    logits = synth.target_logits(shape, tree["parent"], tree["node_tok"], tree["n_nodes"])
-    cb = bench.cpu_baseline(argparse.Namespace(ref_nodes=8, cpu_seconds=1.0), shape, x, logits, None)
+    x, logits = bench.oracle_inputs(shape)
+    cb = bench.cpu_baseline(argparse.Namespace(cpu_seconds=1.0), shape, x, logits)
     assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
     assert cb["value_1thread"] is None or cb["value_1thread"] > 0
-    assert int(cb["sample"].split()[0]) > 1  # many step estimates within the second
+    assert "nothing scaled" in cb["sample"]
+
+
+def test_request_step_is_the_whole_step_of_one_request():
+    """The oracle timings' unit: one request of the workload, rebased to pool
+    row 0, whose whole step (every node attended) runs without scaling."""
+    from ddtree_speculative_decode_b200 import synth
+    shape = synth.custom(B=3, D=3, K=2, N=6, H=2, d_l=16, d_r=8, V=50, L=(4, 9, 2), seed=5)
+    x, logits = bench.oracle_inputs(shape)
+    r = bench.request_slice(x, logits, 1)
+    assert r["kv"].shape[0] == x.cache_cap[1] and int(r["off"][0]) == 0
+    assert np.array_equal(r["kv"], x.kv[x.cache_off[1]:x.cache_off[1] + x.cache_cap[1]])
+    t, ta, m, n = bench.oracle_request_step(shape, r)
+    assert m == n == 6 and 0 < ta <= t
+    t, ta, m, n = bench.oracle_request_step(shape, r, attn_nodes=2)
+    assert m == 2 and n == 6
+    assert bench.synth_nodes(shape) == 6
 
 
 def test_seed_flag_changes_the_draws():
@@ -84,31 +99,26 @@ def test_two_ranks_under_torchrun_print_one_line():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
 
 
-def test_profiled_traffic_follows_the_captured_sources(tmp_path, monkeypatch):
-    """roofline.traffic comes from the ncu summary only while the captured
-    kernel sources are unchanged (the summary records their sha256), and only
+def test_profiled_traffic_follows_the_captured_sources(tmp_path):
+    """roofline.traffic is the captured DRAM count only while the captured
+    kernel sources are unchanged (the table records their sha256), and only
     for the captured workload."""
     import hashlib
 
     from ddtree_speculative_decode_b200 import synth
     csrc = tmp_path / "ddtree_speculative_decode_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (tmp_path / "profiles").mkdir()
     (csrc / "verify_attn_tc.cu").write_text("kernel A\n")
     (csrc / "sm100_ptx.cuh").write_text("helpers B\n")
 
     def sha(name):
         return hashlib.sha256((csrc / name).read_bytes()).hexdigest()
 
-    (tmp_path / "profiles" / "attn_tc_kimi-1req.md").write_text(
-        "Source captured (sha256):\n\n"
-        f"    verify_attn_tc.cu {sha('verify_attn_tc.cu')}\n"
-        f"    sm100_ptx.cuh     {sha('sm100_ptx.cuh')}\n\n"
-        "| metric | value |\n|---|---|\n"
-        "| dram__bytes_read.sum | 9.5 MB |\n| dram__bytes_write.sum | 512 B |\n")
-    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    table = {"kimi-1req-L4096-N64": {"bytes": 9.5e6 + 512,
+                                     "sources": {"verify_attn_tc.cu": sha("verify_attn_tc.cu"),
+                                                 "sm100_ptx.cuh": sha("sm100_ptx.cuh")}}}
     shape = synth.kimi_1req()
-    assert bench.profiled_traffic(shape) == 9.5e6 + 512
-    assert bench.profiled_traffic(synth.NAMED["kimi-16req"]()) is None  # no capture of that workload
+    assert bench.profiled_traffic(shape, table, str(tmp_path)) == 9.5e6 + 512
+    assert bench.profiled_traffic(synth.NAMED["kimi-16req"](), table, str(tmp_path)) is None  # not captured
     (csrc / "sm100_ptx.cuh").write_text("helpers B, changed\n")
-    assert bench.profiled_traffic(shape) is None
+    assert bench.profiled_traffic(shape, table, str(tmp_path)) is None

@@ -150,11 +150,68 @@ def _run_accept_and_compare(s, x, tree, logits, n_layers=1, stride=0, kv_host=No
 
 @pytest.mark.parametrize("name", ["tiny-f32", "kimi-1req", "kimi-16req", "kimi-4req-32k"])
 def test_accept_named(name):
+    """The workloads' own seeded logits. Whatever they accept must match the
+    oracle; the single-request draw happens to reject at the root (its biased
+    child scores below the row's N(0, 1) maximum), so acceptance of long paths
+    is checked separately with planted logits below."""
     s = synth.NAMED[name]()
     x, tree, logits = _accept_case(s)
+    _run_accept_and_compare(s, x, tree, logits)
+
+
+def _set_logit(logits, dtype, b, i, v, value):
+    if dtype == "bf16":
+        logits[b, i, v] = synth.f32_to_bf16_bits(np.array([value], np.float32))[0]
+    else:
+        logits[b, i, v] = value
+
+
+def _deepest_path(tree, b):
+    n = int(tree["n_nodes"][b])
+    node = int(np.argmax(tree["depth"][b, :n]))  # deepest node, lowest index on ties
+    path = []
+    while node > 0:
+        path.append(node)
+        node = int(tree["parent"][b, node])
+    return path[::-1]
+
+
+@pytest.mark.parametrize("name", ["tiny-f32", "kimi-1req", "kimi-16req", "kimi-4req-32k"])
+def test_accept_planted_deepest_path(name):
+    """Along each tree's deepest path the next node's token is made the row's
+    argmax, so every request accepts that whole path (several tokens per step,
+    as the pages' runs do) and the compaction moves a long, non-contiguous set
+    of rows."""
+    s = synth.NAMED[name]()
+    x, tree, logits = _accept_case(s)
+    want = []
+    for b in range(s.B):
+        path = _deepest_path(tree, b)
+        prev = 0
+        for node in path:
+            _set_logit(logits, s.dtype, b, prev, int(tree["node_tok"][b, node]), 30.0)
+            prev = node
+        want.append(len(path))
     got, ref = _run_accept_and_compare(s, x, tree, logits)
-    if s.B > 1:
-        assert got["acc_len"].sum() > 0  # the bias makes some drafts acceptable
+    assert np.array_equal(got["acc_len"], np.array(want, np.int32))
+    assert min(want) >= min(s.D, s.N - 1) // 2  # deep paths, not a trivial case
+
+
+@pytest.mark.parametrize("name", ["tiny-f32", "kimi-1req", "kimi-16req"])
+def test_accept_reject_path(name):
+    """Every child's token is pushed far below its parent row's maximum: no
+    draft is accepted, the bonus is the root row's argmax and only the root's
+    row is committed."""
+    s = synth.NAMED[name]()
+    x, tree, logits = _accept_case(s)
+    for b in range(s.B):
+        n = int(tree["n_nodes"][b])
+        for c in range(1, n):
+            _set_logit(logits, s.dtype, b, int(tree["parent"][b, c]), int(tree["node_tok"][b, c]), -30.0)
+    got, ref = _run_accept_and_compare(s, x, tree, logits)
+    assert np.all(got["acc_len"] == 0)
+    assert np.array_equal(got["bonus"], got["am"][:, 0])
+    assert np.array_equal(got["acc_nodes"][:, 0], np.zeros(s.B, np.int32))
 
 
 @pytest.mark.parametrize("V", [1, 7, 8, 9, 16383, 16384, 16385, 40000])
@@ -207,3 +264,106 @@ def test_accept_capacity_and_empty_tree():
     got, ref = _run_accept_and_compare(s, x, tree, logits)
     assert got["status"][1] == lib.DDT_ERR_CAPACITY and got["acc_len"][1] == 0 and got["bonus"][1] == -1
     assert got["bonus"][2] == -1 and got["status"][2] == 0
+
+
+def test_accept_node_count_and_pool_bounds():
+    """Device-side guards: a request whose n_nodes exceeds N is bad input, and
+    one whose compaction rows would fall outside the pool is out of bounds;
+    both are skipped (nothing copied, cache_len kept) while the others match
+    the oracle."""
+    s = synth.custom(B=4, D=3, K=3, N=10, H=1, d_l=32, d_r=8, V=700, L=(5, 9, 2, 4), dtype="bf16", seed=3,
+                     accept_p=1.0)
+    x, tree, logits = _accept_case(s)
+    d = step_to_device(x, DEV)
+    kv = t_from(x.kv, DEV, True)
+    rows = x.kv.shape[0]
+    off = x.cache_off.copy()
+    off[1] = rows - 3               # rows [off + L, off + L + n) run past the pool
+    nn = tree["n_nodes"].copy()
+    nn[2] = s.N + 1                 # more nodes than rows per request
+    cl = d["cache_len"].clone()
+    out = lib.accept_compact(t_from(logits, DEV, True), t_from(tree["node_tok"], DEV), t_from(tree["parent"], DEV),
+                             t_from(nn, DEV), kv, t_from(off, DEV), cl, d["cache_cap"])
+    torch.cuda.synchronize()
+    got = {k: v.cpu().numpy() for k, v in out.items()}
+    assert got["status"][1] == lib.DDT_ERR_BOUNDS and got["status"][2] == lib.DDT_ERR_INPUT
+    for b in (1, 2):
+        assert got["acc_len"][b] == 0 and got["bonus"][b] == -1
+        assert np.all(got["acc_nodes"][b] == -1) and np.all(got["out_tok"][b] == -1)
+    assert np.array_equal(cl.cpu().numpy()[[1, 2]], x.cache_len[[1, 2]])
+    kv_ref = x.kv.copy()
+    keep = tree["n_nodes"].copy()
+    keep[[1, 2]] = 0
+    ref = oracle.accept_compact(logits, "bf16", tree["node_tok"], tree["parent"], keep, kv_ref, x.cache_off,
+                                x.cache_len, x.cache_cap)
+    for b in (0, 3):
+        for k in ("am", "acc_len", "acc_nodes", "out_tok", "bonus"):
+            assert np.array_equal(got[k][b], ref[k][b]), (k, b)
+        assert got["status"][b] == 0
+    assert np.array_equal(bf16_tensor_bits(kv), kv_ref)  # requests 1 and 2 copied nothing
+
+
+# ---------------------------------------------------------------------------
+# the sweep's largest batch x budget corner: B 64, N 256, K 16, V 163840
+# ---------------------------------------------------------------------------
+
+
+@pytest.fixture(scope="module")
+def corner():
+    s = synth.kimi_sweep(64, 256, 512)
+    x = synth.make_step(s)
+    return s, x, oracle.build_tree(x.logp, x.tok, x.root_tok, x.cache_len, s.N)
+
+
+def test_build_sweep_corner(corner):
+    s, x, ref = corner
+    assert s.K == 16 and int(ref["n_nodes"].min()) == 256
+    _compare_tree(_run_build(x, s.N), ref)
+
+
+def test_accept_sweep_corner(corner):
+    """64 requests x 256 rows x 163840 bf16 logits (5.4 GB), drawn on the GPU
+    with a seeded generator (the same bytes go to the oracle, one request at a
+    time). Each request gets a planted path to a random node, plus +5 on a
+    random child of 70 % of the nodes."""
+    s, x, tree = corner
+    B, N, V = s.B, s.N, s.V
+    g = torch.Generator(device=DEV)
+    g.manual_seed(4242)
+    logits = torch.randn(B, N, V, generator=g, device=DEV).to(torch.bfloat16)
+    rng = np.random.default_rng(99)
+    for b in range(B):
+        n = int(tree["n_nodes"][b])
+        for i in range(n):
+            kids = np.flatnonzero(tree["parent"][b, :n] == i)
+            if len(kids) and rng.random() < 0.7:
+                c = int(kids[rng.integers(len(kids))])
+                logits[b, i, int(tree["node_tok"][b, c])] += 5.0
+        node = int(rng.integers(1, n))
+        path = []
+        while node > 0:
+            path.append(node)
+            node = int(tree["parent"][b, node])
+        prev = 0
+        for node in path[::-1]:
+            logits[b, prev, int(tree["node_tok"][b, node])] = 30.0
+            prev = node
+    d = step_to_device(x, DEV)
+    kv = t_from(x.kv, DEV, True)
+    cl = d["cache_len"].clone()
+    out = lib.accept_compact(logits, t_from(tree["node_tok"], DEV), t_from(tree["parent"], DEV),
+                             t_from(tree["n_nodes"], DEV), kv, d["cache_off"], cl, d["cache_cap"])
+    torch.cuda.synchronize()
+    got = {k: v.cpu().numpy() for k, v in out.items()}
+    kv_got = bf16_tensor_bits(kv)
+    kv_ref = x.kv.copy()
+    for b in range(B):
+        lg = logits[b:b + 1].view(torch.int16).cpu().numpy().view(np.uint16)
+        sl = {k: tree[k][b:b + 1] for k in ("node_tok", "parent", "n_nodes")}
+        ref = oracle.accept_compact(lg, "bf16", sl["node_tok"], sl["parent"], sl["n_nodes"], kv_ref,
+                                    x.cache_off[b:b + 1], x.cache_len[b:b + 1], x.cache_cap[b:b + 1])
+        for k in ("am", "acc_len", "acc_nodes", "out_tok", "bonus", "status"):
+            assert np.array_equal(got[k][b:b + 1], ref[k]), (k, b)
+        assert cl[b].item() == ref["cache_len"][0]
+    assert got["acc_len"].min() >= 1
+    assert np.array_equal(kv_got, kv_ref)

@@ -73,10 +73,29 @@ def test_host_validation_without_gpu(so):
     args = [p] * 4 + [1, 40, 32, 1024] + [p] * 8 + [None]  # 5 bits x 40 levels > 64
     assert so.ddt_build_tree(*args) == lib.DDT_ERR_UNSUPPORTED
     st = so.ddt_verify_attn(p, p, 10, p, p, p, p, 1, 8, 4, 64, 16, ctypes.c_float(-1.0), 32, 0, 0, p, None, None,
-                            0, None)
+                            None, 0, None)
     assert st == lib.DDT_ERR_INVALID_ARG
-    st = so.ddt_accept_compact(p, 0, 10, p, p, p, 1, 4, p, 0, 8, 1, 0, p, p, p, p, p, p, p, p, p, p, 0, None)
+    st = so.ddt_accept_compact(p, 0, 10, p, p, p, 1, 4, p, 100, 0, 8, 1, 0, p, p, p, p, p, p, p, p, p, p, 0, None)
     assert st == lib.DDT_ERR_INVALID_ARG  # workspace too small
+    st = so.ddt_accept_compact(p, 0, 10, p, p, p, 1, 4, p, 0, 0, 8, 1, 0, p, p, p, p, p, p, p, p, p, p, 1 << 20,
+                               None)
+    assert st == lib.DDT_ERR_INVALID_ARG  # an empty pool
+
+
+def test_wait_limit_setting(so):
+    prev = lib.set_wait_limit_ns(10_000_000)
+    try:
+        assert prev == 2_000_000_000
+        assert lib.set_wait_limit_ns(5) == 10_000_000  # raised to the 1 ms floor
+        assert lib.set_wait_limit_ns(0) == 1_000_000   # 0 restores the default
+        assert lib.set_wait_limit_ns(0) == 2_000_000_000
+    finally:
+        lib.set_wait_limit_ns(0)
+
+
+def test_status_names(so):
+    assert lib.status_string(lib.DDT_ERR_TIMEOUT) == "DDT_ERR_TIMEOUT"
+    assert lib.status_string(lib.DDT_ERR_BOUNDS) == "DDT_ERR_BOUNDS"
 
 
 def test_noalloc_accept_rejects_sizes_beyond_its_array(so):
@@ -84,11 +103,11 @@ def test_noalloc_accept_rejects_sizes_beyond_its_array(so):
     # rejected on the host before anything touches the GPU
     p = ctypes.c_void_p(256)
     assert lib.accept_compact_workspace_size(512, 1024, 163840) > 4 << 20
-    st = so.ddt_accept_compact_noalloc(p, 1, 163840, p, p, p, 512, 1024, p, 1, 576, 1, 0, p, p, p, p, p, p, p, p, p,
-                                       None)
+    st = so.ddt_accept_compact_noalloc(p, 1, 163840, p, p, p, 512, 1024, p, 1 << 20, 1, 576, 1, 0, p, p, p, p, p, p,
+                                       p, p, p, None)
     assert st == lib.DDT_ERR_UNSUPPORTED
-    st = so.ddt_accept_compact_noalloc(None, 1, 163840, p, p, p, 1, 64, p, 1, 576, 1, 0, p, p, p, p, p, p, p, p, p,
-                                       None)
+    st = so.ddt_accept_compact_noalloc(None, 1, 163840, p, p, p, 1, 64, p, 1 << 20, 1, 576, 1, 0, p, p, p, p, p, p,
+                                       p, p, p, None)
     assert st == lib.DDT_ERR_INVALID_ARG
 
 

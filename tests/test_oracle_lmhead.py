@@ -157,3 +157,17 @@ def test_planted_rows_take_the_planted_token():
     paths = [oracle.accept_walk(am[b], tree["node_tok"][b], tree["parent"][b], int(tree["n_nodes"][b]))
              for b in range(2)]
     assert max(len(p) for p in paths) >= 2
+
+
+def test_vocab_slices_give_the_same_picks():
+    """Evaluating the head one slice of the vocabulary at a time (to bound the
+    widened head's memory) changes nothing: same logits, bound and valid sets."""
+    rng = np.random.default_rng(8)
+    h = _bf16(rng.standard_normal((7, 64)))
+    w = _bf16(rng.standard_normal((1000, 64)) / 8.0)
+    assert np.allclose(oracle.lmhead_logits(h, w, v_chunk=97), oracle.lmhead_logits(h, w), rtol=0, atol=1e-12)
+    assert np.allclose(oracle.lmhead_f32_error_bound(h, w, 19, v_chunk=97), oracle.lmhead_f32_error_bound(h, w, 19),
+                       rtol=1e-12, atol=0)
+    am1, v1 = oracle.lmhead_valid_argmax(h, w, 19, v_chunk=128)
+    am2, v2 = oracle.lmhead_valid_argmax(h, w, 19)
+    assert np.array_equal(am1, am2) and all(np.array_equal(a, b) for a, b in zip(v1, v2))
