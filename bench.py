@@ -43,11 +43,9 @@ L2_BYTES = 126 * 1024 * 1024
 # ---------------------------------------------------------------------------
 
 
-# (B, N, L) points of the Kimi-shaped sweep: step time against context length
-# at one and at 16 requests, and the tree budget at one request
-SWEEP_POINTS = [(1, 64, 512), (1, 64, 4096), (1, 64, 16384), (1, 64, 65536),
-                (16, 64, 512), (16, 64, 4096), (16, 64, 16384), (4, 64, 65536),
-                (1, 16, 4096), (1, 256, 4096), (64, 16, 4096)]
+# (B, N, L) points of the Kimi-shaped sweep: every batch x tree budget x
+# context length of the workload definition (36 points)
+SWEEP_POINTS = [(b, n, l) for b in (1, 4, 16, 64) for n in (16, 64, 256) for l in (512, 4096, 65536)]
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -293,20 +291,28 @@ def measure_step(args, shape: synth.Shape, dev, world: int, full: bool):
             return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
         return torch.from_numpy(a).to(dev)
 
-    # ---- inputs (host draw, then resident in HBM) ---------------------------
-    x = synth.make_step(shape)
+    # ---- inputs (host draw, then resident in HBM; sweep points: the latent
+    # rows, queries and logits drawn on the device, same distributions) ------
+    on_device = bool(args.sweep)
+    x = synth.make_step(shape, rows=not on_device)
     logp, tok = dev_t(x.logp), dev_t(x.tok)
     root, cl0 = dev_t(x.root_tok), dev_t(x.cache_len)
     off, cap = dev_t(x.cache_off), dev_t(x.cache_cap)
     tree = lib.build_tree(logp, tok, root, cl0, shape.N)
     torch.cuda.synchronize()
     t_host = {k: v.cpu().numpy() for k, v in tree.items()}
-    logits_h = synth.target_logits(shape, t_host["parent"], t_host["node_tok"], t_host["n_nodes"])
-    set_bytes = x.kv.nbytes + x.q.nbytes + logits_h.nbytes
-    n_sets = max(1, min(16, math.ceil(2 * L2_BYTES / set_bytes)))
-    sets = []
-    for _ in range(n_sets):
-        sets.append({"kv": dev_t(x.kv, bf), "q": dev_t(x.q, bf), "logits": dev_t(logits_h, bf)})
+    if on_device:
+        logits_h = None
+        set_bytes = device_set_bytes(shape, x)
+        n_sets = max(1, min(16, math.ceil(2 * L2_BYTES / set_bytes)))
+        sets = [device_set(shape, x, t_host, dev, k) for k in range(n_sets)]
+    else:
+        logits_h = synth.target_logits(shape, t_host["parent"], t_host["node_tok"], t_host["n_nodes"])
+        set_bytes = x.kv.nbytes + x.q.nbytes + logits_h.nbytes
+        n_sets = max(1, min(16, math.ceil(2 * L2_BYTES / set_bytes)))
+        sets = []
+        for _ in range(n_sets):
+            sets.append({"kv": dev_t(x.kv, bf), "q": dev_t(x.q, bf), "logits": dev_t(logits_h, bf)})
     maxL = int(max(shape.L))
     B, N, H = shape.B, shape.N, shape.H
     ws_attn = torch.zeros(max(256, lib.verify_attn_workspace_size(B, N, H, shape.d_l, shape.d_r, maxL, tdt)),
@@ -530,6 +536,44 @@ def measure_lmhead(args, shape, lib, dev, x, t_host, step_parts):
     return {"rows": B * N, "d_model": d, "V": V, "us": us, "flops": 2.0 * B * N * d * V,
             "head_bytes": float(V * d * 2), "tokens_per_call": int((acc_len + 1).sum()),
             "w": w, "hidden": hidden, "timing": f"graph of {reps} calls, each after a cache_len restore"}
+
+
+def device_set_bytes(shape: synth.Shape, x) -> int:
+    elt = 2 if shape.dtype == "bf16" else 4
+    rows = int(x.cache_cap.astype(np.int64).sum())
+    return elt * (rows * shape.d_qk + shape.B * shape.N * shape.H * shape.d_qk + shape.B * shape.N * shape.V)
+
+
+def device_set(shape: synth.Shape, x, t_host: dict, dev, k: int) -> dict:
+    """One input set drawn on the device with seeded generators, the host
+    recipe's distributions (latent rows N(0, 1) x kv_scale, queries N(0, 1),
+    logits N(0, 1) with +bias on a uniformly chosen child's token at the
+    workload's fraction of nodes), for points too large to draw on the host
+    in reasonable time."""
+    import torch
+    tdt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+    g = torch.Generator(device=dev)
+    g.manual_seed(shape.seed * 1000 + k)
+    rows = int(x.cache_cap.astype(np.int64).sum())
+    kv = (torch.randn(rows, shape.d_qk, generator=g, device=dev) * shape.kv_scale).to(tdt)
+    q = torch.randn(shape.B, shape.N, shape.H, shape.d_qk, generator=g, device=dev).to(tdt)
+    logits = torch.empty(shape.B, shape.N, shape.V, dtype=tdt, device=dev)
+    rng = np.random.default_rng([shape.seed, 11, k])
+    for b in range(shape.B):
+        z = torch.randn(shape.N, shape.V, generator=g, device=dev)
+        n = int(t_host["n_nodes"][b])
+        rows_i, toks = [], []
+        for i in range(n):
+            u, pick = rng.random(), rng.random()
+            kids = np.flatnonzero(t_host["parent"][b, :n] == i)
+            if len(kids) and u < shape.accept_p:
+                rows_i.append(i)
+                toks.append(int(t_host["node_tok"][b, int(kids[min(len(kids) - 1, int(pick * len(kids)))])]))
+        if rows_i:
+            z[torch.tensor(rows_i, device=dev), torch.tensor(toks, device=dev)] += shape.accept_bias
+        logits[b] = z.to(tdt)
+        del z
+    return {"kv": kv, "q": q, "logits": logits}
 
 
 def stage_rooflines(res: dict, pk: dict) -> dict:
@@ -959,7 +1003,12 @@ def main():
             pts = SWEEP_POINTS if args.sweep == "default" else [tuple(int(v) for v in p.split(":"))
                                                                  for p in args.sweep.split(",")]
             for (b, n, l) in pts:
-                run_ours(args, seeded(synth.kimi_sweep(b, n, l)), rank, world, local_rank)
+                sh = seeded(synth.kimi_sweep(b, n, l))
+                # about half a second of timed steps per point (at least 5, at most --steps)
+                est_s = 2.0 * b * n * sh.H * (l + 8) * (sh.d_qk + sh.d_l) / 1.0e15 + 60e-6
+                pa = dataclasses.replace(args) if dataclasses.is_dataclass(args) else argparse.Namespace(**vars(args))
+                pa.steps = int(max(5, min(args.steps, 0.5 / est_s)))
+                run_ours(pa, sh, rank, world, local_rank)
                 torch.cuda.empty_cache()
         else:
             run_ours(args, shape, rank, world, local_rank)

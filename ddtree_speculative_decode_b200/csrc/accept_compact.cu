@@ -31,6 +31,7 @@
 #include <mutex>
 
 #include "ddt_kernels.cuh"
+#include "sm100_ptx.cuh"
 
 namespace ddt {
 
@@ -162,6 +163,143 @@ __global__ void __launch_bounds__(kArgmaxThreads) accept_argmax_kernel(AcceptPar
   if (cur_row >= 0) flush();
 }
 
+// The same argmax for 16-byte aligned rows, fed by 1-D bulk copies: each
+// warp streams its contiguous range of slices through a ring of kBulkBufs
+// shared-memory buffers (one mbarrier each), so every SM keeps 192 KB of
+// logits in flight -- more than registers can hold -- and a launch of few
+// rows finishes in one round trip to HBM.
+constexpr int kBulkWarps = kArgmaxThreads / 32;
+constexpr int kBulkBufs = 3;
+constexpr int kSliceBytes = 32 * kSliceVec * 16;
+constexpr int kBulkSmem = kBulkWarps * kBulkBufs * (kSliceBytes + 8);
+
+template <bool kBF16>
+__global__ void __launch_bounds__(kArgmaxThreads, 1) accept_argmax_bulk_kernel(AcceptParams p) {
+  using C = SliceCfg<kBF16>;
+  extern __shared__ __align__(128) unsigned char smem[];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // a status word already holding an error (an earlier wait gave up): nothing to do
+  if (*reinterpret_cast<const volatile int*>(p.status_word) != 0) return;
+  const long long gw = (long long)blockIdx.x * kBulkWarps + warp;
+  const long long nw = (long long)gridDim.x * kBulkWarps;
+  const int spr = (p.V + C::kElems - 1) / C::kElems;  // slices per row
+  const long long slices = (long long)p.B * p.N * spr;
+  const long long s_begin = slices * gw / nw, s_end = slices * (gw + 1) / nw;
+  const size_t esz = kBF16 ? 2 : 4;
+  unsigned char* wbuf = smem + warp * kBulkBufs * kSliceBytes;
+  const uint32_t bar0 = sm100::smem_u32(smem + kBulkWarps * kBulkBufs * kSliceBytes + warp * kBulkBufs * 8);
+  if (lane == 0) {
+    for (int k = 0; k < kBulkBufs; ++k) sm100::mbar_init(bar0 + 8u * k, 1);
+    sm100::fence_mbar_init_cluster();
+  }
+  __syncwarp();
+  // the next slice at or after s that belongs to a real row (pad rows are skipped)
+  auto advance = [&](long long sl) -> long long {
+    while (sl < s_end) {
+      const int r = (int)(sl / spr);
+      const int b = r / p.N, i = r - b * p.N;
+      if (i < __ldg(p.n_nodes + b)) return sl;
+      sl = (long long)(r + 1) * spr;
+    }
+    return s_end;
+  };
+  auto issue = [&](long long sl, int k) {  // lane 0
+    const int r = (int)(sl / spr), c = (int)(sl - (long long)r * spr);
+    const int v0 = c * C::kElems;
+    const uint32_t bytes = (uint32_t)(min(C::kElems, p.V - v0) * esz);
+    const unsigned char* src = static_cast<const unsigned char*>(p.logits) + ((size_t)r * p.V + v0) * esz;
+    sm100::mbar_arrive_expect_tx(bar0 + 8u * k, bytes);
+    sm100::bulk_load_1d(sm100::smem_u32(wbuf + k * kSliceBytes), src, bytes, bar0 + 8u * k);
+  };
+  long long qs[kBulkBufs];
+  uint32_t phases = 0;
+  long long next = advance(s_begin);
+  int issued = 0;
+  for (int k = 0; k < kBulkBufs && next < s_end; ++k) {
+    if (lane == 0) issue(next, k);
+    qs[k] = next;
+    next = advance(next + 1);
+    ++issued;
+  }
+  int cur_row = -1;
+  float best_v = -INFINITY;
+  int best_i = -1;
+  auto flush = [&]() {
+    const unsigned long long k = warp_max64(best_i < 0 ? 0ull : pack_key(best_v, best_i));
+    if (lane == 0 && k != 0ull) atomicMax(p.rowkey + cur_row, k);
+  };
+  for (int done = 0; done < issued; ++done) {
+    const int k = done % kBulkBufs;
+    const long long sl = qs[k];
+    if (!sm100::mbar_wait(bar0 + 8u * k, (phases >> k) & 1u, p.abort, p.wait_ns)) return;
+    phases ^= 1u << k;
+    const int r = (int)(sl / spr), c = (int)(sl - (long long)r * spr);
+    if (r != cur_row) {
+      if (cur_row >= 0) flush();
+      cur_row = r;
+      best_v = -INFINITY;
+      best_i = -1;
+    }
+    const int v0 = c * C::kElems;
+    const int nvec = min(C::kElems, p.V - v0) / C::kPer;
+    const uint4* src = reinterpret_cast<const uint4*>(wbuf + k * kSliceBytes);
+    uint4 v[kSliceVec];
+#pragma unroll
+    for (int kk = 0; kk < kSliceVec; ++kk) {
+      const int e = lane + 32 * kk;
+      v[kk] = e < nvec ? src[e]
+                       : (kBF16 ? make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u)
+                                : make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u));
+    }
+    __syncwarp();  // every lane has read the buffer: it may be refilled
+    if (next < s_end) {
+      if (lane == 0) issue(next, k);
+      qs[k] = next;
+      next = advance(next + 1);
+      ++issued;
+    }
+    float m;
+    if (kBF16) {
+      auto h = [](uint32_t w) { return *reinterpret_cast<const __nv_bfloat162*>(&w); };
+      __nv_bfloat162 mk[kSliceVec];
+#pragma unroll
+      for (int kk = 0; kk < kSliceVec; ++kk)
+        mk[kk] = __hmax2(__hmax2(h(v[kk].x), h(v[kk].y)), __hmax2(h(v[kk].z), h(v[kk].w)));
+#pragma unroll
+      for (int w = kSliceVec / 2; w > 0; w >>= 1)
+#pragma unroll
+        for (int kk = 0; kk < w; ++kk) mk[kk] = __hmax2(mk[kk], mk[kk + w]);
+      m = fmaxf(__low2float(mk[0]), __high2float(mk[0]));
+    } else {
+      float mk[kSliceVec];
+#pragma unroll
+      for (int kk = 0; kk < kSliceVec; ++kk)
+        mk[kk] = fmaxf(fmaxf(__uint_as_float(v[kk].x), __uint_as_float(v[kk].y)),
+                       fmaxf(__uint_as_float(v[kk].z), __uint_as_float(v[kk].w)));
+#pragma unroll
+      for (int w = kSliceVec / 2; w > 0; w >>= 1)
+#pragma unroll
+        for (int kk = 0; kk < w; ++kk) mk[kk] = fmaxf(mk[kk], mk[kk + w]);
+      m = mk[0];
+    }
+    if (lane < nvec && (m > best_v || best_i < 0)) {
+      int first = -1;  // lowest real index holding m (values compare as floats: -0 == +0)
+#pragma unroll
+      for (int kk = kSliceVec - 1; kk >= 0; --kk) {
+        const int e = lane + 32 * kk;
+#pragma unroll
+        for (int t = C::kPer - 1; t >= 0; --t)
+          if (e < nvec && vec_val<kBF16>(v[kk], t) == m) first = v0 + e * C::kPer + t;
+      }
+      best_v = m;
+      best_i = first;
+    }
+  }
+  if (cur_row >= 0) flush();
+}
+
 // Request epilogue: one CTA per request.
 __global__ void __launch_bounds__(kWalkThreads) accept_walk_kernel(AcceptParams p) {
   __shared__ int32_t s_am[kMaxN];
@@ -254,9 +392,15 @@ __global__ void __launch_bounds__(kWalkThreads) accept_walk_kernel(AcceptParams 
     p.bonus[b] = bonus;
   }
   if (skip) return;
-  // compaction: rows path[0..a] -> L + 0..a on every layer
+  // compaction: rows path[0..a] -> L + 0..a on every layer (several layers:
+  // compact_layers_kernel does it, spread over CTAs, after this kernel)
   const int L = p.cache_len[b];
   const int rows = a + 1;
+  if (p.layers_apart) {
+    __syncthreads();
+    if (tid == 0) p.cache_len[b] = L + rows;
+    return;
+  }
   const int64_t base_row = p.cache_off[b] + L;
   const bool v16 = (p.row_bytes % 16 == 0) && ((reinterpret_cast<uintptr_t>(p.kv) & 15u) == 0) &&
                    (p.layer_stride_bytes % 16 == 0);
@@ -297,6 +441,78 @@ __global__ void __launch_bounds__(kWalkThreads) accept_walk_kernel(AcceptParams 
   if (tid == 0) p.cache_len[b] = L + rows;
 }
 
+// Multi-layer compaction after the walk: CTA (b, g) moves request b's
+// accepted rows on layers [g * per, (g + 1) * per). The walk has written the
+// path (acc_nodes, -1 in slot 0 for a skipped request), acc_len and the new
+// cache_len, so the committed rows start at cache_len - (acc_len + 1). Rows
+// move in rounds of increasing destination index, each round read completely
+// before it is written: a path is increasing with path[j] >= j, so no round
+// writes a row a later round still reads.
+constexpr int kCopyThreads = 256;
+
+__global__ void __launch_bounds__(kCopyThreads) compact_layers_kernel(AcceptParams p, int groups, int per) {
+  __shared__ int32_t s_path[kMaxN];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int b = blockIdx.x / groups, g = blockIdx.x - b * groups;
+  const int tid = threadIdx.x;
+  const int N = p.N;
+  if (p.acc_nodes[(size_t)b * N] != 0) return;  // skipped request: nothing moves
+  const int rows = p.acc_len[b] + 1;
+  for (int j = tid; j < rows; j += kCopyThreads) s_path[j] = p.acc_nodes[(size_t)b * N + j];
+  __syncthreads();
+  const int64_t base_row = p.cache_off[b] + (p.cache_len[b] - rows);
+  const int l0 = g * per, l1 = min(p.n_layers, l0 + per);
+  const bool v16 = (p.row_bytes % 16 == 0) && ((reinterpret_cast<uintptr_t>(p.kv) & 15u) == 0) &&
+                   (p.layer_stride_bytes % 16 == 0);
+  const int vb = v16 ? 16 : 4;
+  const int vpr = p.row_bytes / vb;
+  const long long per_layer = (long long)rows * vpr;
+  const long long total = per_layer * (l1 - l0);
+  for (long long t0 = 0; t0 < total; t0 += (long long)kCopyThreads * kStageVec) {
+    uint4 buf[kStageVec];
+#pragma unroll
+    for (int u = 0; u < kStageVec; ++u) {
+      const long long e = t0 + u * kCopyThreads + tid;
+      if (e < total) {
+        const int layer = l0 + (int)(e / per_layer);
+        const long long rem = e % per_layer;
+        const int rr = (int)(rem / vpr), cc = (int)(rem - (long long)rr * vpr);
+        const unsigned char* src =
+            p.kv + layer * p.layer_stride_bytes + (base_row + s_path[rr]) * p.row_bytes + (size_t)cc * vb;
+        if (v16) buf[u] = __ldcs(reinterpret_cast<const uint4*>(src));
+        else buf[u].x = *reinterpret_cast<const uint32_t*>(src);
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kStageVec; ++u) {
+      const long long e = t0 + u * kCopyThreads + tid;
+      if (e < total) {
+        const int layer = l0 + (int)(e / per_layer);
+        const long long rem = e % per_layer;
+        const int rr = (int)(rem / vpr), cc = (int)(rem - (long long)rr * vpr);
+        unsigned char* dst = p.kv + layer * p.layer_stride_bytes + (base_row + rr) * p.row_bytes + (size_t)cc * vb;
+        if (v16) *reinterpret_cast<uint4*>(dst) = buf[u];
+        else *reinterpret_cast<uint32_t*>(dst) = buf[u].x;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// Launch the walk, then (several layers) the spread-out compaction.
+static int launch_walk_and_copy(AcceptParams p, cudaStream_t stream) {
+  p.layers_apart = p.n_layers > 1 ? 1 : 0;
+  const int st = launch_pdl(accept_walk_kernel, (unsigned)p.B, kWalkThreads, 0, stream, p);
+  if (st != DDT_OK || !p.layers_apart) return st;
+  // about two CTAs per SM over all requests, whole layers per CTA
+  const int groups = std::max(1, std::min(p.n_layers, ceil_div(2 * sm_count(), p.B)));
+  const int per = ceil_div(p.n_layers, groups);
+  const int used = ceil_div(p.n_layers, per);
+  return launch_pdl(compact_layers_kernel, (unsigned)(p.B * used), kCopyThreads, 0, stream, p, used, per);
+}
+
 static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 static size_t header_bytes() { return 256; }
 static size_t zeroed_bytes(int B, int N) { return header_bytes() + round256((size_t)B * N * 8); }
@@ -307,22 +523,55 @@ size_t accept_workspace_bytes(int B, int N, int V) {
 }
 
 
+// The bulk-copy argmax's shared-memory opt-in, set once per device.
+static bool bulk_argmax_ready(bool bf16) {
+  static std::mutex mu;
+  static int done[kMaxDevices][2] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  int& d = done[dev][bf16 ? 1 : 0];
+  if (d == 0) {
+    const cudaError_t e =
+        bf16 ? cudaFuncSetAttribute(accept_argmax_bulk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kBulkSmem)
+             : cudaFuncSetAttribute(accept_argmax_bulk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kBulkSmem);
+    d = e == cudaSuccess ? 1 : -1;
+    if (e != cudaSuccess) (void)cudaGetLastError();
+  }
+  return d == 1;
+}
+
 int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream) {
   unsigned char* ws = static_cast<unsigned char*>(workspace);
-  // the first 256 bytes are reserved (no kernel here waits on anything)
+  // the first 256 bytes: status word (a bounded wait of the argmax gave up)
+  p.abort = reinterpret_cast<int*>(ws);
+  p.status_word = reinterpret_cast<const int*>(ws);
+  p.wait_ns = wait_limit_ns();
   p.rowkey = reinterpret_cast<unsigned long long*>(ws + header_bytes());
   const size_t esz = p.logits_dtype == DDT_BF16 ? 2 : 4;
   p.tma = (reinterpret_cast<uintptr_t>(p.logits) % 16 == 0) && (((size_t)p.V * esz) % 16 == 0);
   const int elems = p.logits_dtype == DDT_BF16 ? SliceCfg<true>::kElems : SliceCfg<false>::kElems;
   const long long slices = (long long)p.B * p.N * ceil_div(p.V, elems);
-  const long long warps = std::max(1LL, std::min<long long>(slices, (long long)sm_count() * kArgmaxCtasPerSm *
-                                                                        (kArgmaxThreads / 32)));
-  const unsigned grid = (unsigned)((warps + kArgmaxThreads / 32 - 1) / (kArgmaxThreads / 32));
-  const int st = p.logits_dtype == DDT_BF16
-                     ? launch_pdl(accept_argmax_kernel<true>, grid, kArgmaxThreads, 0, stream, p)
-                     : launch_pdl(accept_argmax_kernel<false>, grid, kArgmaxThreads, 0, stream, p);
+  const bool bf = p.logits_dtype == DDT_BF16;
+  int st;
+  if (p.tma && bulk_argmax_ready(bf)) {
+    // one CTA of 16 warps per SM, each warp a contiguous range of slices
+    const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(sm_count(), ceil_div((int)std::min<long long>(
+                                                                                               slices, 1LL << 30),
+                                                                                           kBulkWarps)));
+    st = bf ? launch_pdl(accept_argmax_bulk_kernel<true>, grid, kArgmaxThreads, (size_t)kBulkSmem, stream, p)
+            : launch_pdl(accept_argmax_bulk_kernel<false>, grid, kArgmaxThreads, (size_t)kBulkSmem, stream, p);
+  } else {
+    const long long warps = std::max(1LL, std::min<long long>(slices, (long long)sm_count() * kArgmaxCtasPerSm *
+                                                                          (kArgmaxThreads / 32)));
+    const unsigned grid = (unsigned)((warps + kArgmaxThreads / 32 - 1) / (kArgmaxThreads / 32));
+    st = bf ? launch_pdl(accept_argmax_kernel<true>, grid, kArgmaxThreads, 0, stream, p)
+            : launch_pdl(accept_argmax_kernel<false>, grid, kArgmaxThreads, 0, stream, p);
+  }
   if (st != DDT_OK) return st;
-  return launch_pdl(accept_walk_kernel, (unsigned)p.B, kWalkThreads, 0, stream, p);
+  return launch_walk_and_copy(p, stream);
 }
 
 // The walk and compaction alone, on row keys another kernel (the LM-head
@@ -332,7 +581,7 @@ int launch_accept_walk(AcceptParams p, void* workspace, cudaStream_t stream) {
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   p.rowkey = reinterpret_cast<unsigned long long*>(ws + header_bytes());
   p.status_word = reinterpret_cast<const int*>(ws);
-  return launch_pdl(accept_walk_kernel, (unsigned)p.B, kWalkThreads, 0, stream, p);
+  return launch_walk_and_copy(p, stream);
 }
 
 // ---------------------------------------------------------------------------

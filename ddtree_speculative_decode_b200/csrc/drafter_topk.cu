@@ -182,18 +182,24 @@ __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams 
   __shared__ unsigned long long s_thr;
   if (tid == 0) s_thr = 0ull;
   __syncthreads();
-  unsigned long long wl = 0ull, wthr = 0ull, thr = 0ull, pub = 0ull;
+  // lo: a key just below the K-th largest of the warp's lanes' maxima over
+  // the first loads (those K keys are distinct values of the row, so no key
+  // below lo can be among the row's K best); it keeps the first batches,
+  // where the lists are still empty, from taking every value as a hit
+  unsigned long long wl = 0ull, wthr = 0ull, thr = 0ull, pub = 0ull, lo = 0ull;
   float m = -INFINITY, s = 0.0f;
   bool bad = false;
   // before each batch: the CTA's threshold; after it: publish this warp's
   auto refresh = [&]() {
     const unsigned long long c = *reinterpret_cast<volatile unsigned long long*>(&s_thr);
     thr = c > wthr ? c : wthr;
+    thr = thr > lo ? thr : lo;
   };
   auto publish = [&]() {
-    if (wthr > pub) {  // warp-uniform
-      if (lane == 0) atomicMax(&s_thr, wthr);
-      pub = wthr;
+    const unsigned long long w = wthr > lo ? wthr : lo;
+    if (w > pub) {  // warp-uniform
+      if (lane == 0) atomicMax(&s_thr, w);
+      pub = w;
     }
   };
   // a batch of n of this lane's values (all lanes of the warp call it together)
@@ -237,12 +243,34 @@ __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams 
     // eight 16-byte loads in flight per thread (64 KB per CTA) before any is
     // used; whole warps step together (lanes past the end take no values)
     constexpr int kU = 8;
+    bool first = true;
     for (int e0 = v0 / kPer + warp * 32; e0 < nvec; e0 += kU * kDrThreads) {
       uint4 v[kU];
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
         const int e = e0 + lane + u * kDrThreads;
         v[u] = e < nvec ? __ldcs(src + e) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      if (first) {
+        // each lane's largest key over its first loads, then the K-th
+        // largest of the warp's 32 (0 while fewer than K lanes hold a value)
+        first = false;
+        unsigned long long lk = 0ull;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int e = e0 + lane + u * kDrThreads;
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int t = 0; t < kPer; ++t) {
+            const float xv = kBF16 ? __uint_as_float((t & 1) ? (w[t >> 1] & 0xffff0000u) : (w[t >> 1] << 16))
+                                   : __uint_as_float(w[t]);
+            const unsigned long long key =
+                (e < nvec && fabsf(xv) <= 3.402823466e38f) ? drafter_key(xv, e * kPer + t) : 0ull;
+            lk = key > lk ? key : lk;
+          }
+        }
+        const unsigned long long kth = __shfl_sync(DDT_FULL_MASK, warp_sort_desc(lk, lane), p.K - 1);
+        lo = kth > 0ull ? kth - 1ull : 0ull;
       }
 #pragma unroll
       for (int u = 0; u < kU; ++u) {

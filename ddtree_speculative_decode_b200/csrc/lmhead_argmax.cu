@@ -144,6 +144,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int slot = 0;
     uint32_t phase = 0;
     bool ok = true;
+    // the head streams from HBM once (evict first); the hidden rows are read
+    // by every CTA for every tile (evict last)
+    const uint64_t pol_w = l2_policy_evict_first(), pol_h = l2_policy_evict_last();
     for (int t = pair; t < total && ok; t += npairs) {
       const int pass = t / p.vtiles, vt = t - pass * p.vtiles;
       const int v0 = vt * 256 + 128 * (int)rank;
@@ -156,9 +159,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (leader) mbar_arrive_expect_tx(bar(kBarFull + slot), 2u * (uint32_t)p.stage_bytes);
         const uint32_t dst = sbase + (uint32_t)(slot * p.stage_bytes);
         const uint32_t fb = full0 + 8u * (uint32_t)slot;
-        tma_load_2d_pair(dst, &tm_w, 64 * kb, v0, fb);
+        tma_load_2d_pair_hint(dst, &tm_w, 64 * kb, v0, fb, pol_w);
         for (int j = 0; j < p.parts; ++j)
-          tma_load_2d_pair(dst + kABytes + (uint32_t)(j * p.nh * 128), &tm_h, 64 * kb, h0 + 256 * j, fb);
+          tma_load_2d_pair_hint(dst + kABytes + (uint32_t)(j * p.nh * 128), &tm_h, 64 * kb, h0 + 256 * j, fb,
+                                pol_h);
         if (++slot == p.stages) {
           slot = 0;
           phase ^= 1u;
@@ -199,26 +203,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 2) {
     // ============================================================ reduction
     // thread = TMEM lane 32 q + lane = vocabulary row 128 rank + 32 q + lane
-    // of the tile; for every column (verify row) the warp's best over its 32
-    // rows, kept by lane (column % 32) in best[column / 32]
+    // of the tile. Per 32-column chunk the warp finds, for every column
+    // (verify row), the best of its 32 rows; lane c of the warp ends up with
+    // column c's and merges it into the CTA's running key for that column in
+    // shared memory. The loop over chunks stays rolled: the code the MMA
+    // issuer runs must stay in the instruction cache next to it.
     const int q = warp & 3;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
     const uint32_t empty0 = map_to_rank(bar(kBarAccEmpty), 0);
     const int ncols = p.parts == 2 ? kPassRows : p.npart;
     const int nchunks = (ncols + 31) / 32;
-    unsigned long long best[kMaxChunks];
-#pragma unroll
-    for (int m = 0; m < kMaxChunks; ++m) best[m] = 0ull;
     int cur_pass = -1;
     bool ok = true;
-    // the CTA's best per column into shared memory, then one global atomic
-    // max per real verify row of the pass
+    // the CTA's key per column of the pass out to the rows' global keys
     auto flush = [&](int pass) {
-#pragma unroll
-      for (int m = 0; m < kMaxChunks; ++m) {
-        if (m < nchunks && best[m] != 0ull) atomicMax(s_red + 32 * m + lane, best[m]);
-        best[m] = 0ull;
-      }
       named_bar_sync(1, 128);
       for (int c = (int)threadIdx.x - 64; c < ncols; c += 128) {
         const unsigned long long k = s_red[c];
@@ -230,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       named_bar_sync(1, 128);
     };
-    named_bar_sync(1, 128);  // s_red zeroed by the whole CTA before the barrier above; keep the 4 warps in step
+    named_bar_sync(1, 128);  // the 4 warps start together (s_red was zeroed before the set-up barrier)
     int lt = 0;
     for (int t = pair; t < total; t += npairs, ++lt) {
       const int pass = t / p.vtiles, vt = t - pass * p.vtiles;
@@ -244,31 +242,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int vrow = vt * 256 + 128 * (int)rank + 32 * q;  // vocabulary row of lane 0
       const bool valid = ok && vrow + lane < p.V;
       const uint32_t col0 = (uint32_t)(buf * p.parts * 256);
-#pragma unroll
-      for (int m = 0; m < kMaxChunks; ++m) {
-        if (m < nchunks) {
-          uint32_t r[32];
-          tmem_ld32(lane_addr + col0 + 32u * (uint32_t)m, r);
-          tmem_wait_ld();
-          if (m == nchunks - 1) {
-            // the accumulator buffer is free for the next tile's MMAs
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-              if (leader) mbar_arrive_local(bar(kBarAccEmpty + buf));
-              else mbar_arrive_cluster(empty0 + 8u * (uint32_t)buf);
-            }
-          }
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const uint32_t key = valid ? float_order_key(__uint_as_float(r[i])) : 0u;
-            const uint32_t mx = __reduce_max_sync(DDT_FULL_MASK, key);
-            const uint32_t hit = __ballot_sync(DDT_FULL_MASK, key == mx);
-            const unsigned long long packed =
-                ((unsigned long long)mx << 32) | (unsigned long long)(~(uint32_t)(vrow + __ffs(hit) - 1));
-            if (lane == i && mx != 0u && packed > best[m]) best[m] = packed;
+#pragma unroll 1
+      for (int m = 0; m < nchunks; ++m) {
+        uint32_t r[32];
+        tmem_ld32(lane_addr + col0 + 32u * (uint32_t)m, r);
+        tmem_wait_ld();
+        if (m == nchunks - 1) {
+          // the accumulator buffer is free for the next tile's MMAs
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (leader) mbar_arrive_local(bar(kBarAccEmpty + buf));
+            else mbar_arrive_cluster(empty0 + 8u * (uint32_t)buf);
           }
         }
+        unsigned long long mine = 0ull;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const uint32_t key = valid ? float_order_key(__uint_as_float(r[i])) : 0u;
+          const uint32_t mx = __reduce_max_sync(DDT_FULL_MASK, key);
+          const uint32_t hit = __ballot_sync(DDT_FULL_MASK, key == mx);
+          if (lane == i && mx != 0u)
+            mine = ((unsigned long long)mx << 32) | (unsigned long long)(~(uint32_t)(vrow + __ffs(hit) - 1));
+        }
+        if (mine != 0ull) atomicMax(s_red + 32 * m + lane, mine);
       }
     }
     if (cur_pass >= 0) flush(cur_pass);

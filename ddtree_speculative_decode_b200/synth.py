@@ -209,12 +209,13 @@ def drafter_topk(rng: np.random.Generator, D: int, K: int, V: int, sigma: float)
     return logp, tok
 
 
-def make_step(shape: Shape, requests: Optional[list] = None) -> StepInputs:
+def make_step(shape: Shape, requests: Optional[list] = None, rows: bool = True) -> StepInputs:
     """Draw all pre-tree inputs of one step.
 
     ``requests`` (optional) restricts the draws to a subset of request ids; the
     per-request streams are independent, so a subset sees the same values as a
-    full draw.
+    full draw. ``rows=False`` skips the latent rows and queries (kv and q are
+    then empty arrays of the right shape's dtype): the other draws are the same.
     """
     s = shape
     reqs = list(range(s.B)) if requests is None else list(requests)
@@ -223,10 +224,10 @@ def make_step(shape: Shape, requests: Optional[list] = None) -> StepInputs:
     cap = L + s.N
     off = np.zeros(B, np.int64)
     off[1:] = np.cumsum(cap[:-1].astype(np.int64))
-    rows = int(cap.astype(np.int64).sum())
+    n_rows = int(cap.astype(np.int64).sum())
     d_qk = s.d_qk
-    kv = np.zeros((rows, d_qk), np.float32 if s.dtype == "f32" else np.uint16)
-    q = np.zeros((B, s.N, s.H, d_qk), kv.dtype)
+    kv = np.zeros((n_rows if rows else 0, d_qk), np.float32 if s.dtype == "f32" else np.uint16)
+    q = np.zeros((B if rows else 0, s.N, s.H, d_qk), kv.dtype)
     logp = np.zeros((B, s.D, s.K), np.float32)
     tok = np.zeros((B, s.D, s.K), np.int32)
     root = np.zeros(B, np.int32)
@@ -234,6 +235,8 @@ def make_step(shape: Shape, requests: Optional[list] = None) -> StepInputs:
         r = _rng(s.seed, 1, b)
         root[j] = int(r.integers(0, s.V))
         logp[j], tok[j] = drafter_topk(_rng(s.seed, 2, b), s.D, s.K, s.V, s.drafter_sigma)
+        if not rows:
+            continue
         rk = _rng(s.seed, 3, b)
         blk = rk.standard_normal((int(L[j]) + s.N, d_qk), dtype=np.float32) * np.float32(s.kv_scale)
         kv[off[j]:off[j] + L[j] + s.N] = _store(blk, s.dtype)

@@ -263,17 +263,24 @@ DDT_API int ddt_verify_attn(const void* q, const void* kv, int64_t kv_rows, cons
  *   unchanged. Requests with n_nodes[b] == 0 are skipped the same way with
  *   DDT_OK.
  * workspace: ddt_accept_compact_workspace_size(B, N, V) bytes, 256-byte
- *   aligned: 256 reserved bytes, then one 8-byte running argmax key per row
- *   (B * N, rounded up to 256 bytes). All of it must be zero before the
+ *   aligned: a 256-byte status word, then one 8-byte running argmax key per
+ *   row (B * N, rounded up to 256 bytes). All of it must be zero before the
  *   first call -- zero the buffer once after allocating it; every call
- *   leaves it at zero again. Nothing in these kernels waits on another CTA.
- *   Calls that share a workspace must not overlap on the GPU.
+ *   leaves it at zero again. The argmax kernel waits (bounded, see
+ *   ddt_set_wait_limit_ns) for its own bulk copies; if a wait gives up, the
+ *   status word holds DDT_ERR_TIMEOUT, every request reports
+ *   DDT_ERR_TIMEOUT and accepts nothing, and later calls with that
+ *   workspace do the same until the caller zeroes it. Calls that share a
+ *   workspace must not overlap on the GPU.
  * Precondition the library cannot check: the layers and requests own
  *   disjoint rows.
- * Runs as two kernels: the logits stream once with 16-byte loads, each warp
- *   owning contiguous 2048-entry slices of the rows (two 512-thread CTAs per
- *   SM; row maxima published by 64-bit atomic max), then one CTA per request
- *   finds each node's accepted child, walks the path and compacts the rows.
+ * Runs as two kernels (three with several layers): the logits stream once,
+ *   each warp owning contiguous 2048-entry slices of the rows, brought into
+ *   a 3-deep shared-memory ring by 1-D bulk copies (16-byte aligned rows;
+ *   plain loads otherwise), row maxima published by 64-bit atomic max; then
+ *   one CTA per request finds each node's accepted child, walks the path and
+ *   (one layer) compacts the rows; with several layers a third kernel moves
+ *   the rows, spread over (request, layer group) CTAs.
  */
 DDT_API size_t ddt_accept_compact_workspace_size(int B, int N, int V);
 
@@ -337,7 +344,7 @@ DDT_API int ddt_accept_compact_lmhead(const void* hidden, const void* w_vocab, i
  * the host application, or a latency-critical decode loop that must not call
  * cudaMalloc (which can synchronise the device). This entry point takes the
  * same arguments as ddt_accept_compact minus the workspace and allocates
- * nothing: its scratch (reserved header and per-row argmax keys) lives in one
+ * nothing: its scratch (status word and per-row argmax keys) lives in one
  * fixed 4 MiB array inside the library, which every GPU
  * that loads the library keeps until the process exits.
  *

@@ -194,7 +194,10 @@ def test_accept_planted_deepest_path(name):
         want.append(len(path))
     got, ref = _run_accept_and_compare(s, x, tree, logits)
     assert np.array_equal(got["acc_len"], np.array(want, np.int32))
-    assert min(want) >= min(s.D, s.N - 1) // 2  # deep paths, not a trivial case
+    # every request accepts several drafts (how many depends on the tree: the
+    # workloads' drafters spread their mass over many tokens, so the budget
+    # goes to siblings and the trees are 2 to 3 nodes deep)
+    assert min(want) >= 2
 
 
 @pytest.mark.parametrize("name", ["tiny-f32", "kimi-1req", "kimi-16req"])
@@ -367,3 +370,29 @@ def test_accept_sweep_corner(corner):
         assert cl[b].item() == ref["cache_len"][0]
     assert got["acc_len"].min() >= 1
     assert np.array_equal(kv_got, kv_ref)
+
+
+def test_accept_status_word_timeout_skips_everything():
+    """A workspace whose status word holds a timeout (as an argmax kernel that
+    gave up a wait on its copies leaves it) makes the call accept nothing:
+    every request reports DDT_ERR_TIMEOUT, keeps its cache and cache_len, and
+    the row keys are left at zero; after the caller zeroes the workspace the
+    same call matches the oracle."""
+    s = synth.custom(B=3, D=3, K=3, N=12, H=1, d_l=32, d_r=8, V=4096, L=(3, 7, 11), dtype="bf16", seed=12,
+                     accept_p=1.0)
+    x, tree, logits = _accept_case(s)
+    d = step_to_device(x, DEV)
+    kv = t_from(x.kv, DEV, True)
+    ws = torch.zeros(lib.accept_compact_workspace_size(s.B, s.N, s.V), dtype=torch.uint8, device=DEV)
+    ws[:4].view(torch.int32)[0] = lib.DDT_ERR_TIMEOUT
+    cl = d["cache_len"].clone()
+    args = (t_from(logits, DEV, True), t_from(tree["node_tok"], DEV), t_from(tree["parent"], DEV),
+            t_from(tree["n_nodes"], DEV), kv, d["cache_off"])
+    out = lib.accept_compact(*args, cl, d["cache_cap"], workspace=ws)
+    torch.cuda.synchronize()
+    assert np.all(out["status"].cpu().numpy() == lib.DDT_ERR_TIMEOUT)
+    assert np.all(out["acc_len"].cpu().numpy() == 0) and np.array_equal(cl.cpu().numpy(), x.cache_len)
+    assert np.array_equal(bf16_tensor_bits(kv), x.kv)
+    assert int(ws[256:].view(torch.int64).abs().sum().item()) == 0
+    ws.zero_()
+    _run_accept_and_compare(s, x, tree, logits)
