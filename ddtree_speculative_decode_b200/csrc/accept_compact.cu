@@ -336,7 +336,8 @@ __global__ void __launch_bounds__(kWalkThreads) accept_walk_kernel(AcceptParams 
     if (p.dev_status) p.dev_status[b] = st;
   }
   pdl_wait();
-  pdl_launch_dependents();
+  // no early trigger of the next kernel: this one writes the pool and
+  // cache_len, which a following verify attention reads before it waits
   // the kernel that produced the row keys gave up a wait: they are not
   // complete, so nothing is accepted (the keys are still cleared)
   if (p.status_word != nullptr && tid == 0 && *reinterpret_cast<const volatile int*>(p.status_word) != 0) {
@@ -452,8 +453,7 @@ constexpr int kCopyThreads = 256;
 
 __global__ void __launch_bounds__(kCopyThreads) compact_layers_kernel(AcceptParams p, int groups, int per) {
   __shared__ int32_t s_path[kMaxN];
-  pdl_wait();
-  pdl_launch_dependents();
+  pdl_wait();  // (no early trigger of the next kernel: this one writes the pool)
   const int b = blockIdx.x / groups, g = blockIdx.x - b * groups;
   const int tid = threadIdx.x;
   const int N = p.N;
@@ -555,8 +555,14 @@ int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream) 
   const int elems = p.logits_dtype == DDT_BF16 ? SliceCfg<true>::kElems : SliceCfg<false>::kElems;
   const long long slices = (long long)p.B * p.N * ceil_div(p.V, elems);
   const bool bf = p.logits_dtype == DDT_BF16;
+  // the register-fed kernel keeps 128 KB per SM in flight: enough when the
+  // logits take several rounds of it; a launch of few rows (fewer slices
+  // than two of its rounds) finishes sooner with the bulk-copy ring, which
+  // keeps 192 KB per SM in flight (measured: 64 rows x 163840, 14.6 against
+  // 15.4 us per accept; 512 rows, 48 against 43 us)
+  const long long reg_warps = (long long)sm_count() * kArgmaxCtasPerSm * (kArgmaxThreads / 32);
   int st;
-  if (p.tma && bulk_argmax_ready(bf)) {
+  if (p.tma && slices <= 2 * reg_warps && bulk_argmax_ready(bf)) {
     // one CTA of 16 warps per SM, each warp a contiguous range of slices
     const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(sm_count(), ceil_div((int)std::min<long long>(
                                                                                                slices, 1LL << 30),

@@ -398,8 +398,7 @@ static int launch_dr(const DrafterParams& p, cudaStream_t stream) {
 int launch_drafter_topk(DrafterParams p, cudaStream_t stream) {
   const size_t esz = p.logits_dtype == DDT_BF16 ? 2 : 4;
   p.vec = (reinterpret_cast<uintptr_t>(p.logits) % 16 == 0) && (((size_t)p.V * esz) % 16 == 0);
-  // slices of at least 16384 logits, at most 8 CTAs (one portable cluster) per
-  // row; slice starts stay on a 16-byte vector
+  // slice starts stay on a 16-byte vector
   auto launch = [&](int C) -> int {
     p.C = C;
     p.chunk = ((p.V + C - 1) / C + 7) / 8 * 8;
@@ -407,7 +406,10 @@ int launch_drafter_topk(DrafterParams p, cudaStream_t stream) {
     if (p.K <= 16) return launch_dr<16>(p, stream);
     return launch_dr<32>(p, stream);
   };
-  const int C = std::max(1, std::min(8, (p.V + 16383) / 16384));
+  // one wave: rows x CTAs per row at most one CTA per SM (each CTA holds an
+  // SM's registers), slices of at least 16384 logits, at most 8 CTAs per row
+  const int by_rows = std::max(1, sm_count() / std::max(1, p.R));
+  const int C = std::max(1, std::min({8, (p.V + 16383) / 16384, by_rows}));
   if (C > 1) {
     if (launch(C) == DDT_OK) return DDT_OK;
     (void)cudaGetLastError();  // clusters of C not schedulable here: one CTA per row

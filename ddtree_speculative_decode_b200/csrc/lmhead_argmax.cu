@@ -51,7 +51,6 @@ constexpr int kABytes = 128 * 128;      // 128 head rows x 64 dims bf16 per CTA 
 constexpr int kPassRows = 512;          // verify rows per pass over the head
 constexpr int kMaxStages = 12;
 constexpr int kStageBudget = 200 * 1024;
-constexpr int kMaxChunks = kPassRows / 32;
 
 // shared memory after the stages
 constexpr int kBarFull = 0;                      // [kMaxStages] leader: TMA bytes of a stage (both CTAs)

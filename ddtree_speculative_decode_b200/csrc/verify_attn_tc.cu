@@ -19,18 +19,10 @@
 //    576-d rows through TMA), K-steps of 16 over 576 dims. PV: two MMAs with
 //    N = 256 output dims each (each CTA supplies 128 dims of the latent rows,
 //    read MN-major from the same TMA tile layout), K = 256 keys.
-//  * Both rings hand the tensor pipe 8 MMAs per stage release: a
-//    tcgen05.commit or an mbarrier wait in an issuing thread costs the pipe
-//    up to ~90 ns unless enough MMAs are queued around it.
-//  * Warp roles per CTA: warps 0 / 2 = TMA producers of the QK ring (query
-//    and key chunks; the query is re-streamed with every key tile so shared
-//    memory holds deeper rings) and of the value ring (both CTAs load their
-//    halves into their own shared memory, completion counted on the leader
-//    CTA's barriers), warps 1 / 3 = the QK and PV MMA issuers (leader CTA
-//    only; warp 1 also allocates TMEM),
-//    warps 4..11 = softmax (TMEM lane quarter = warp % 4, two warps per
-//    quarter; thread = one query row x one 64-key group of the tile, and one
-//    of the row's two 128-dim output accumulator blocks).
+//  * Each ring stage feeds 4 MMAs and is released on its own (the QK ring:
+//    this CTA's Q chunk + its keys' chunk for 64 dims; the V ring: 64 keys x
+//    one 128-dim block of each output half), so most of each ring is in
+//    flight at any time.
 //  * Two issuing threads because every mbarrier wait in an issuing thread
 //    stalls the tensor pipe for about as long as two MMAs (its issue queue
 //    is shallow); with QK and PV on separate threads and separate rings, one
@@ -42,6 +34,10 @@
 //    node's ancestor bitmask; key groups that run past the request's last key
 //    are loaded from a window that ends at that key (never outside the
 //    request's finite rows) and the duplicated keys are masked.
+//  * The kernel may start while the tree build (the kernel before it) still
+//    runs: a unit's key range is planned over cache_len + N, its committed-
+//    cache tiles need nothing from the build, and each role waits for the
+//    build only when it first needs the tree (unit_tree).
 //  * A request's keys can be split into several units (flash-decoding); each
 //    split writes unnormalised fp32 partials (O, running max, sum) and counts
 //    its arrival per (row tile, CTA half); the split that arrives last merges
@@ -146,30 +142,38 @@ struct TcParams {
   uint64_t wait_ns;  // wall-clock limit of every wait
 };
 
+// A unit's work: its key range is planned over the budget's keys (cache_len
+// + N) from inputs the tree build does not write, so a unit can start on its
+// committed-cache tiles while the build still runs; the tree's size (and the
+// pool-bound check) comes in once a role needs it (unit_tree, after waiting
+// for the build).
 struct UnitInfo {
   int b, rt, split;
-  int off_row;       // first pool row of the request (fits int: checked on host)
-  int L, n, nkeys;
-  int kb, ke, T;     // key range [kb, ke) of this unit, T tiles
+  int off_row;       // first pool row of the request (as an int; a bad offset is caught by unit_tree)
+  int L;             // committed keys (cache_len, at least 0)
+  int kb, kend_plan; // key range [kb, kend_plan) of this unit over the budget's keys
+  int T;             // tiles of the unit
+  int tt;            // tiles [0, tt) hold committed keys only (need nothing from the build)
   int active;        // splits of this request that get keys (splits [0, active))
-  bool pad_tile;     // every row of the row tile is a pad row
+  // set by unit_tree:
+  int n, nkeys, ke;  // tree nodes, keys, end of this unit's range over the real keys
   bool oob;          // the request's rows do not lie in the pool: all its rows are pad rows
+  bool tree;         // unit_tree has run
 };
 
-__device__ __forceinline__ UnitInfo unit_info(const TcParams& p, int unit) {
+__device__ __forceinline__ UnitInfo unit_plan(const TcParams& p, int unit) {
   UnitInfo u;
   u.split = unit % p.splits;
   const int t = unit / p.splits;
   u.rt = t % p.rowtiles;
   u.b = t / p.rowtiles;
   const int64_t off = p.cache_off[u.b];
-  const int L = p.cache_len[u.b], n = p.n_nodes[u.b];
-  u.oob = n < 0 || n > p.N || off < 0 || L < 0 || off + L + n > p.kv_rows;
-  u.off_row = u.oob ? 0 : (int)off;  // fits int: kv_rows does (checked on the host)
-  u.L = u.oob ? 0 : L;
-  u.n = u.oob ? 0 : n;
-  u.nkeys = u.L + u.n;
-  const int tiles = (u.nkeys + kTileKeys - 1) / kTileKeys;
+  const int L = p.cache_len[u.b];
+  u.off_row = (int)off;
+  u.L = max(L, 0);
+  const long long nk_plan = (long long)u.L + p.N;
+  const long long tiles_ll = (nk_plan + kTileKeys - 1) / kTileKeys;
+  const int tiles = (int)(tiles_ll < (1LL << 24) ? tiles_ll : (1LL << 24));
   // splits get floor or ceil(tiles / splits) tiles, the larger shares last
   // (where the request's ragged last tile is); splits past `tiles` get none
   u.active = min(p.splits, tiles);
@@ -177,12 +181,31 @@ __device__ __forceinline__ UnitInfo unit_info(const TcParams& p, int unit) {
   const int t1 = u.split < u.active ? (int)((long long)(u.split + 1) * tiles / u.active) : tiles;
   u.T = t1 - t0;
   u.kb = t0 * kTileKeys;
-  u.ke = min(u.nkeys, t1 * kTileKeys);
-  // a row tile whose first node is already a pad node has nothing to compute
-  const int first_node = (u.rt * 128) / p.H;
-  u.pad_tile = u.n <= 0 || first_node >= u.n;
-  if (u.pad_tile) u.T = 0;
+  const long long kend = (long long)t1 * kTileKeys;
+  u.kend_plan = (int)(nk_plan < kend ? nk_plan : kend);
+  u.tt = u.L > u.kb ? min(u.T, (u.L - u.kb) / kTileKeys) : 0;
+  u.n = 0;
+  u.nkeys = u.L;
+  u.ke = min(u.L, u.kend_plan);
+  u.oob = false;
+  u.tree = false;
   return u;
+}
+
+// The tree's part: wait for the build (programmatic launch: its writes are
+// visible after the wait), then the node count and the pool-bound check. A
+// request whose rows do not lie in the pool keeps the plan's loads (TMA
+// returns zeros outside the pool) and is written as pad rows.
+__device__ __forceinline__ void unit_tree(const TcParams& p, UnitInfo& u) {
+  if (u.tree) return;
+  pdl_wait();
+  const int64_t off = p.cache_off[u.b];
+  const int L = p.cache_len[u.b], n = p.n_nodes[u.b];
+  u.oob = n < 0 || n > p.N || off < 0 || L < 0 || off + L + n > p.kv_rows;
+  u.n = u.oob ? 0 : n;
+  u.nkeys = u.L + u.n;
+  u.ke = min(u.nkeys, u.kend_plan);
+  u.tree = true;
 }
 
 // 2^x with the hardware approximation, subnormal results flushed to zero: the
@@ -249,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  pdl_wait();
+  // no wait for the preceding kernel (the tree build) here: see unit_tree
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // A CTA pair (ranks 2k, 2k + 1 of the cluster) runs one unit with the
@@ -261,19 +284,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool leader = rank == 0;
   const uint16_t pmask = (uint16_t)(0x3u << pbase);
   const int unit = p.csize == 4 ? (int)((blockIdx.x >> 2) * 2 + (crank >> 1)) : (int)(blockIdx.x >> 1);
-  const UnitInfo u = unit_info(p, unit);
+  UnitInfo u = unit_plan(p, unit);
   const int rows_total = p.B * p.N * p.H;
   const int req_rows = p.N * p.H;
   const int row0 = u.rt * 128 + 64 * (int)rank;  // first request-relative row of this CTA
-  if (p.dev_status && u.rt == 0 && u.split == 0 && rank == 0 && threadIdx.x == 0)
-    p.dev_status[u.b] = u.oob ? DDT_ERR_BOUNDS : DDT_OK;
 
   auto bar = [&](int i) -> uint32_t { return sbase + kOffMisc + 8u * (uint32_t)i; };
 
   // ---------------------------------------------------------------- empty unit
-  // a split past the last one that gets keys has nothing to do; a row tile of
-  // pad rows only is written (zeros, lse -inf) by split 0. In a 4-CTA cluster
-  // an idle pair still takes part in the cluster-wide barriers below.
+  // a split past the last one that gets keys has nothing to do (in a 4-CTA
+  // cluster an idle pair still takes part in the cluster-wide barriers
+  // below); pad rows of real units are written as zeros by their epilogue.
   // this CTA's 64 rows as pad rows (zeros, lse -inf), all threads
   auto write_pad_rows = [&]() {
     for (int r = threadIdx.x; r < 64; r += kThreads) {
@@ -295,10 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
   const bool idle = u.T == 0;
-  if (idle) {
-    if (u.pad_tile && u.split == 0) write_pad_rows();
-    if (p.csize == 2) return;
-  }
+  if (idle && p.csize == 2) return;
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
@@ -325,16 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_kv);
   }
-  // masks of this CTA's 64 rows (node = row / H)
+  // masks of this CTA's 64 rows (node = row / H): loaded by the softmax
+  // threads once the build is done (the first tile that reaches tree keys)
   uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem + kOffMask);
-  for (int e = threadIdx.x; e < 64 * kMaxW; e += kThreads) {
-    const int r = e / kMaxW, w = e % kMaxW;
-    const int rr = row0 + r;
-    const int node = rr / p.H;
-    uint32_t v = 0u;
-    if (rr < req_rows && node < p.N && w < p.W) v = p.mask[((size_t)u.b * p.N + node) * p.W + w];
-    s_mask[e] = v;
-  }
   if (warp == 1) {
     tmem_alloc_pair(sbase + kOffTmem, 512);
     tmem_relinquish_pair();
@@ -362,7 +373,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (idle || aborted) {
     // nothing to compute: straight to the cluster-wide teardown (after an
     // earlier timeout split 0 writes its rows as pad rows)
-    if (aborted && !idle && u.split == 0) write_pad_rows();
+    if (aborted && !idle && u.split == 0) {
+      write_pad_rows();
+      if (p.dev_status && u.rt == 0 && rank == 0 && threadIdx.x == 0) p.dev_status[u.b] = DDT_ERR_TIMEOUT;
+    }
   } else if (warp == 0 && lane == 0) {
     // ============================================================ QK producer
     // per tile and 64-dim chunk: this CTA's Q chunk and its 128 keys' chunk
@@ -370,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Ring rg;
     const int qrow = u.b * req_rows + row0;
     for (int t = 0; t < u.T; ++t) {
+      if (t >= u.tt) unit_tree(p, u);  // windows of a tile that reaches tree keys depend on the tree's size
       const int tile0 = u.kb + t * kTileKeys;
       const int y0 = u.off_row + group_window(tile0 + 128 * (int)rank, u.nkeys);
       const int y1 = u.off_row + group_window(tile0 + 128 * (int)rank + 64, u.nkeys);
@@ -413,6 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Ring rg;
     const int x = 128 * (int)rank;
     for (int t = 0; t < u.T; ++t) {
+      if (t >= u.tt) unit_tree(p, u);  // live groups and windows of a tile that reaches tree keys
       const int tile0 = u.kb + t * kTileKeys;
       bool ok = true;
       const int ng = live_groups(u, t);
@@ -470,6 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < u.T && ok; ++t) {
         if (!mbar_wait(bar(kBarPFull), (uint32_t)(t & 1), abort, wlim)) { ok = false; break; }
         tc_fence_after();
+        if (t >= u.tt) unit_tree(p, u);  // live key groups of a tile that reaches tree keys
         const int ng = live_groups(u, t);
         for (int g = 0; g < ng && ok; ++g) {
           const uint32_t a0 = sbase + kOffP + g * kBoxBytes;
@@ -511,9 +528,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     float m_used = -INFINITY, lsum = 0.0f;
     bool ok = true;
+    // the tree's part, once: the build's results (node count, pool check)
+    // and this CTA's 64 mask rows into shared memory
+    auto tree_part = [&]() {
+      unit_tree(p, u);
+      for (int e = (int)threadIdx.x - 128; e < 64 * kMaxW; e += 32 * kSoftmaxWarps) {
+        const int r = e / kMaxW, w = e % kMaxW;
+        const int rr = row0 + r;
+        const int node = rr / p.H;
+        uint32_t v = 0u;
+        if (rr < req_rows && node < p.N && w < p.W) v = p.mask[((size_t)u.b * p.N + node) * p.W + w];
+        s_mask[e] = v;
+      }
+      named_bar_sync(1, 32 * kSoftmaxWarps);
+    };
     // every thread runs all T iterations (and so every named barrier) even
     // after an aborted wait; later waits then return at once
     for (int t = 0; t < u.T; ++t) {
+      if (t == u.tt) tree_part();  // the first tile that reaches tree keys
       const int sb = t & 1;
       if (ok && !mbar_wait(bar(kBarSFull + sb), (uint32_t)((t >> 1) & 1), abort, wlim)) ok = false;
       tc_fence_after();
@@ -635,6 +667,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     //   O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
     if (ok) ok = mbar_wait(bar(kBarOFull), (uint32_t)((u.T - 1) & 1), abort, wlim);
     tc_fence_after();
+    unit_tree(p, u);  // a unit of committed keys only still needs the tree's size for its rows
+    if (p.dev_status && u.rt == 0 && u.split == 0 && rank == 0 && threadIdx.x == 128)
+      p.dev_status[u.b] = u.oob ? DDT_ERR_BOUNDS : DDT_OK;
     lred[grp * 64 + rho] = lsum;
     const int rr = row0 + rho;
     const bool in_range = rr < req_rows;

@@ -116,8 +116,9 @@ DDT_API uint64_t ddt_set_wait_limit_ns(uint64_t ns);
  *   logit (that row's tok = -1, logp = -inf).
  * Sizes: R >= 1, V >= 1, 1 <= K <= min(V, 32); R < 2^28 and V <= 2^30
  *   (DDT_ERR_UNSUPPORTED beyond).
- * A row is split over a cluster of min(8, ceil(V / 16384)) CTAs (one CTA
- *   per row where such a cluster cannot be scheduled); no workspace. Errors:
+ * A row is split over a cluster of min(8, ceil(V / 16384), SMs / R) CTAs
+ *   (at least one; one CTA per row where such a cluster cannot be
+ *   scheduled), so the launch is one wave; no workspace. Errors:
  *   DDT_ERR_INVALID_ARG (nulls, sizes, dtype), DDT_ERR_UNSUPPORTED (sizes
  *   above), DDT_ERR_CUDA (launch).
  */
@@ -193,8 +194,21 @@ DDT_API int ddt_build_tree(const float* logp, const int32_t* tok, const int32_t*
  * Outputs (device): out [B][N][H][d_l] out_dtype; lse [B][N][H] float32
  *   (nullable); dev_status [B] int32 (nullable): DDT_OK, or DDT_ERR_BOUNDS
  *   when cache_off[b] + cache_len[b] + n_nodes[b] > kv_rows, a value is
- *   negative, or n_nodes[b] > N -- that request then reads nothing and all
- *   its rows are written as pad rows.
+ *   negative, or n_nodes[b] > N -- all that request's rows are then written
+ *   as pad rows (the bf16 kernel may already have read committed rows
+ *   through TMA, which returns zeros outside the pool; the f32 kernel reads
+ *   nothing) -- or DDT_ERR_TIMEOUT when the workspace's status word already
+ *   held a timeout (bf16 kernel).
+ * Launch order: the bf16 kernel is launched as a programmatic dependent and
+ *   may start while the kernel before it on the stream still runs, if that
+ *   kernel allows it (of this library's kernels, the tree build does: the
+ *   verify attention then computes over the committed cache while the tree
+ *   is built). It reads q, kv, cache_off and cache_len at once, and waits
+ *   for the preceding kernel before it reads mask or n_nodes. So q, kv,
+ *   cache_off and cache_len must not be written by the kernel issued just
+ *   before this call; the library's kernels that write the pool or
+ *   cache_len (the accept's walk and compaction) never let a dependent start
+ *   early, and kernels that are not programmatic-launch aware never do.
  * Supported: in_dtype F32 (CUDA-core kernel, any d_l, d_r with d_qk <= 1024)
  *   and BF16 with (d_l, d_r) = (512, 64) (tensor-core kernel); out_dtype F32
  *   or BF16. Accumulation is float32 throughout. The bf16 kernel rounds the
