@@ -69,7 +69,16 @@ def replica_throughput(nodes_per_step: int, steps: int, world: int, elapsed_ms: 
 # capture per workload (the capture command and figures are summarised under
 # profiles/), valid only while the kernel sources still have the sha256 they
 # had when captured.
-PROFILED_ATTN_DRAM = {}
+PROFILED_ATTN_DRAM = {
+    # ncu --set full, one launch of the long-context workload's attention
+    # (bench.py --steps 3 --warmup 3 --no-cpu-baseline --e2e-steps 3 --layers 1
+    # --extra=, -k regex:attn_tc -s 2 -c 1): dram__bytes_read.sum 338.873344 MB
+    # + dram__bytes_write.sum 82.572032 MB
+    "kimi-4req-L32768-N128": {
+        "bytes": 421445376.0,
+        "sources": {"verify_attn_tc.cu": "6c4e301d687384245554f015c0b53d97b75bb4bfb18e1bf698b933b8e416d4e3",
+                    "sm100_ptx.cuh": "742a701fc79bc45f49ed1e6b9494f89da884dc911c9353fdb120e72dbac572a6"}},
+}
 
 
 def profiled_traffic(shape: synth.Shape, table=None, root=None):

@@ -18,7 +18,8 @@
 // of them), so one head row is read from HBM once per pass however few rows
 // are verified. The head and hidden tiles stream through a ring of stages by
 // TMA (64 dims per stage, 128-byte swizzle); warp 0 loads, warp 1 of the
-// leader CTA issues the MMAs, warps 2..5 reduce each finished accumulator:
+// leader CTA issues the MMAs (with two N parts, warp 6 issues the second
+// part's), warps 2..5 reduce each finished accumulator:
 // per verify row (column) a warp-wide maximum of order-preserving value keys
 // (redux.sync) and the lowest lane holding it (ballot), so every tile yields,
 // per row, (largest logit, lowest vocabulary index) packed in 64 bits. Rows
@@ -46,7 +47,7 @@ namespace lmh {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;           // warp 0 TMA, warp 1 MMA (+ TMEM), warps 2..5 reduction
+constexpr int kThreads = 224;           // warp 0 TMA, warps 1 and 6 MMA (warp 1: + TMEM), warps 2..5 reduction
 constexpr int kABytes = 128 * 128;      // 128 head rows x 64 dims bf16 per CTA and stage
 constexpr int kPassRows = 512;          // verify rows per pass over the head
 constexpr int kMaxStages = 12;
@@ -106,12 +107,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t wlim = p.wait_ns;
 
   if (threadIdx.x == 0) {
+    // with two N parts each has its own issuing thread: a stage is free, and
+    // an accumulator complete, when both have committed
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(bar(kBarFull + s), 1);
-      mbar_init(bar(kBarEmpty + s), 1);
+      mbar_init(bar(kBarEmpty + s), (uint32_t)p.parts);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(kBarAccFull + b), 1);
+      mbar_init(bar(kBarAccFull + b), (uint32_t)p.parts);
       mbar_init(bar(kBarAccEmpty + b), 8);
     }
     fence_mbar_init_cluster();
@@ -168,9 +171,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1 && lane == 0 && leader) {
-    // ============================================================ MMA issuer
+  } else if ((warp == 1 || (warp == 6 && p.parts == 2)) && lane == 0 && leader) {
+    // ============================================================ MMA issuers
+    // one thread per N part (warp 6 only with two): a barrier wait in an
+    // issuing thread costs the tensor pipe about two MMAs, and the other
+    // thread's queued MMAs cover it; the parts' accumulators are disjoint
     const uint32_t idesc = idesc_bf16_f32(256, p.npart, false, false);
+    const int j0 = p.parts == 2 ? (warp == 6 ? 1 : 0) : 0, j1 = p.parts == 2 ? j0 + 1 : p.parts;
     int slot = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -187,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a0 = sbase + (uint32_t)(slot * p.stage_bytes);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          for (int j = 0; j < p.parts; ++j)
+          for (int j = j0; j < j1; ++j)
             mma_pair_ss(tmem + (uint32_t)((buf * p.parts + j) * 256), smem_desc_sw128(a0 + 32 * k, 16, 1024),
                         smem_desc_sw128(a0 + kABytes + (uint32_t)(j * p.nh * 128) + 32 * k, 16, 1024), idesc,
                         (kb | k) != 0 ? 1u : 0u);
@@ -199,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok) mma_commit_pair_mc(bar(kBarAccFull + buf), (uint16_t)0x3u);
     }
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && warp <= 5) {
     // ============================================================ reduction
     // thread = TMEM lane 32 q + lane = vocabulary row 128 rank + 32 q + lane
     // of the tile. Per 32-column chunk the warp finds, for every column
