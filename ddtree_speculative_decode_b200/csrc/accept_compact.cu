@@ -11,13 +11,20 @@
 // Two launches:
 //  * accept_argmax_kernel streams the logits once with coalesced 16-byte
 //    loads, eight in flight per lane, 32 warps per SM. Work is cut into
-//    slices of 2048 entries of one row, and every warp owns a contiguous
-//    range of slices, so it folds a row's slices itself and publishes one
+//    slices of 2048 entries of one row, handed out to warps in chunks of
+//    consecutive slices by atomic counters in the workspace; a warp folds
+//    each row's slices of a chunk itself and publishes one
 //    packed 64-bit key per row segment with a fire-and-forget atomic max
 //    (key = order-preserving value bits << 32 | ~index: the max key is the
 //    largest logit at its lowest index). A lane only searches for an index
 //    when a batch beats its running maximum, so the common batch costs one
-//    packed max per two values.
+//    packed max per two values. The argmax reads nothing the tree build or
+//    the verify attention writes (every row of the logits is reduced, pad
+//    rows included), so it starts as soon as the kernel before it lets its
+//    dependents launch: its CTAs take SMs the attention leaves idle (its
+//    last, ragged wave) and, through the shared counter, most of the work.
+//    Each CTA waits for the kernel before it only at its end, so this grid
+//    still ends after that kernel.
 //  * accept_walk_kernel, one CTA per request (launched programmatically: it
 //    stages the tree while the argmax runs), turns the row keys into am[],
 //    finds every node's accepted child (the lowest-index child whose token is
@@ -41,6 +48,7 @@ constexpr int kArgmaxCtasPerSm = 2;
 constexpr int kWalkThreads = 512;
 constexpr int kMaxN = 1024;
 constexpr int kStageVec = 4;                      // 16-byte vectors per thread per copy round
+constexpr int kChunkSlices = 4;                   // slices per chunk of the register-fed argmax's work feed
 
 template <bool kBF16>
 struct SliceCfg {
@@ -71,17 +79,50 @@ __device__ __forceinline__ float vec_val(const uint4& r, int t) {
   return __uint_as_float((t & 1) ? (w & 0xffff0000u) : (w << 16));
 }
 
+// Work feed: chunks of `chunk` consecutive slices handed out by counters in
+// the workspace header (kCounters of them, 32 bytes apart; a warp draws from
+// counter gw % kCounters, which serves chunks ctr, ctr + kCounters, ...), so
+// warps that start early -- beside the kernel before this one -- take more of
+// the work. Lane 0 keeps the next draw in flight while the current chunk is
+// read. (A static first chunk per warp, or several draws in flight per warp,
+// measured slower steps.)
+constexpr int kCounters = 7;
+struct ChunkFeed {
+  unsigned* work;
+  long long slices, chunk, nchunks;
+  int ctr;             // this warp's counter
+  unsigned pre;        // lane 0: the next counter value (in flight)
+  long long cs, ce;    // warp-uniform: the current chunk's slices [cs, ce)
+  __device__ void start(long long gw, int lane) {
+    ctr = (int)(gw % kCounters);
+    cs = ce = 0;
+    pre = lane == 0 ? atomicAdd(work + 8 * ctr, 1u) : 0u;
+  }
+  // the warp's next slice, or -1 once its counter is past the last chunk
+  // (every later draw of that counter is larger)
+  __device__ long long next(int lane) {
+    if (cs >= ce) {
+      const long long c = (long long)__shfl_sync(DDT_FULL_MASK, pre, 0) * kCounters + ctr;
+      if (c >= nchunks) return -1;
+      if (lane == 0) pre = atomicAdd(work + 8 * ctr, 1u);
+      cs = c * chunk;
+      ce = cs + chunk < slices ? cs + chunk : slices;
+    }
+    return cs++;
+  }
+};
+
 template <bool kBF16>
 __global__ void __launch_bounds__(kArgmaxThreads) accept_argmax_kernel(AcceptParams p) {
   using C = SliceCfg<kBF16>;
-  pdl_wait();
+  // no wait for the kernel before: see the file comment (it comes at the end)
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
-  const long long gw = ((long long)blockIdx.x * kArgmaxThreads + threadIdx.x) >> 5;
-  const long long nw = ((long long)gridDim.x * kArgmaxThreads) >> 5;
   const int spr = (p.V + C::kElems - 1) / C::kElems;  // slices per row
   const long long slices = (long long)p.B * p.N * spr;
-  const long long s_begin = slices * gw / nw, s_end = slices * (gw + 1) / nw;
+  const long long gw = ((long long)blockIdx.x * kArgmaxThreads + threadIdx.x) >> 5;
+  ChunkFeed feed{p.work, slices, kChunkSlices, (slices + kChunkSlices - 1) / kChunkSlices};
+  feed.start(gw, lane);
   const size_t esz = kBF16 ? 2 : 4;
   int cur_row = -1;
   float best_v = -INFINITY;   // this lane's running max of cur_row and its lowest index
@@ -90,10 +131,8 @@ __global__ void __launch_bounds__(kArgmaxThreads) accept_argmax_kernel(AcceptPar
     const unsigned long long k = warp_max64(best_i < 0 ? 0ull : pack_key(best_v, best_i));
     if (lane == 0 && k != 0ull) atomicMax(p.rowkey + cur_row, k);  // result unused: no wait
   };
-  for (long long sl = s_begin; sl < s_end; ++sl) {
+  for (long long sl = feed.next(lane); sl >= 0; sl = feed.next(lane)) {
     const int r = (int)(sl / spr), c = (int)(sl - (long long)r * spr);
-    const int b = r / p.N, i = r - b * p.N;
-    if (i >= __ldg(p.n_nodes + b)) continue;
     if (r != cur_row) {
       if (cur_row >= 0) flush();
       cur_row = r;
@@ -161,10 +200,11 @@ __global__ void __launch_bounds__(kArgmaxThreads) accept_argmax_kernel(AcceptPar
     }
   }
   if (cur_row >= 0) flush();
+  pdl_wait();  // this grid ends after the kernel before it (the walk relies on that)
 }
 
 // The same argmax for 16-byte aligned rows, fed by 1-D bulk copies: each
-// warp streams its contiguous range of slices through a ring of kBulkBufs
+// warp streams the slices of its chunks through a ring of kBulkBufs
 // shared-memory buffers (one mbarrier each), so every SM keeps 192 KB of
 // logits in flight -- more than registers can hold -- and a launch of few
 // rows finishes in one round trip to HBM.
@@ -177,16 +217,19 @@ template <bool kBF16>
 __global__ void __launch_bounds__(kArgmaxThreads, 1) accept_argmax_bulk_kernel(AcceptParams p) {
   using C = SliceCfg<kBF16>;
   extern __shared__ __align__(128) unsigned char smem[];
-  pdl_wait();
+  // no wait for the kernel before: see the file comment (it comes at the end)
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // a status word already holding an error (an earlier wait gave up): nothing to do
-  if (*reinterpret_cast<const volatile int*>(p.status_word) != 0) return;
-  const long long gw = (long long)blockIdx.x * kBulkWarps + warp;
-  const long long nw = (long long)gridDim.x * kBulkWarps;
+  if (*reinterpret_cast<const volatile int*>(p.status_word) != 0) {
+    pdl_wait();
+    return;
+  }
   const int spr = (p.V + C::kElems - 1) / C::kElems;  // slices per row
   const long long slices = (long long)p.B * p.N * spr;
-  const long long s_begin = slices * gw / nw, s_end = slices * (gw + 1) / nw;
+  const long long gw = (long long)blockIdx.x * kBulkWarps + warp;
+  // single slices: few rows give each warp only a couple
+  ChunkFeed feed{p.work, slices, 1, slices};
   const size_t esz = kBF16 ? 2 : 4;
   unsigned char* wbuf = smem + warp * kBulkBufs * kSliceBytes;
   const uint32_t bar0 = sm100::smem_u32(smem + kBulkWarps * kBulkBufs * kSliceBytes + warp * kBulkBufs * 8);
@@ -195,16 +238,7 @@ __global__ void __launch_bounds__(kArgmaxThreads, 1) accept_argmax_bulk_kernel(A
     sm100::fence_mbar_init_cluster();
   }
   __syncwarp();
-  // the next slice at or after s that belongs to a real row (pad rows are skipped)
-  auto advance = [&](long long sl) -> long long {
-    while (sl < s_end) {
-      const int r = (int)(sl / spr);
-      const int b = r / p.N, i = r - b * p.N;
-      if (i < __ldg(p.n_nodes + b)) return sl;
-      sl = (long long)(r + 1) * spr;
-    }
-    return s_end;
-  };
+  feed.start(gw, lane);
   auto issue = [&](long long sl, int k) {  // lane 0
     const int r = (int)(sl / spr), c = (int)(sl - (long long)r * spr);
     const int v0 = c * C::kElems;
@@ -215,12 +249,12 @@ __global__ void __launch_bounds__(kArgmaxThreads, 1) accept_argmax_bulk_kernel(A
   };
   long long qs[kBulkBufs];
   uint32_t phases = 0;
-  long long next = advance(s_begin);
+  long long next = feed.next(lane);
   int issued = 0;
-  for (int k = 0; k < kBulkBufs && next < s_end; ++k) {
+  for (int k = 0; k < kBulkBufs && next >= 0; ++k) {
     if (lane == 0) issue(next, k);
     qs[k] = next;
-    next = advance(next + 1);
+    next = feed.next(lane);
     ++issued;
   }
   int cur_row = -1;
@@ -233,7 +267,17 @@ __global__ void __launch_bounds__(kArgmaxThreads, 1) accept_argmax_bulk_kernel(A
   for (int done = 0; done < issued; ++done) {
     const int k = done % kBulkBufs;
     const long long sl = qs[k];
-    if (!sm100::mbar_wait(bar0 + 8u * k, (phases >> k) & 1u, p.abort, p.wait_ns)) return;
+    if (!sm100::mbar_wait(bar0 + 8u * k, (phases >> k) & 1u, p.abort, p.wait_ns)) {
+      // gave up: the copies still in flight land in this CTA's shared memory,
+      // so wait (bounded) for them before leaving
+      for (int j = done; j < issued; ++j) {
+        const int kj = j % kBulkBufs;
+        (void)sm100::mbar_wait_own(bar0 + 8u * kj, (phases >> kj) & 1u, p.abort, p.wait_ns);
+        phases ^= 1u << kj;
+      }
+      pdl_wait();
+      return;
+    }
     phases ^= 1u << k;
     const int r = (int)(sl / spr), c = (int)(sl - (long long)r * spr);
     if (r != cur_row) {
@@ -254,10 +298,10 @@ __global__ void __launch_bounds__(kArgmaxThreads, 1) accept_argmax_bulk_kernel(A
                                 : make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u));
     }
     __syncwarp();  // every lane has read the buffer: it may be refilled
-    if (next < s_end) {
+    if (next >= 0) {
       if (lane == 0) issue(next, k);
       qs[k] = next;
-      next = advance(next + 1);
+      next = feed.next(lane);
       ++issued;
     }
     float m;
@@ -298,6 +342,7 @@ __global__ void __launch_bounds__(kArgmaxThreads, 1) accept_argmax_bulk_kernel(A
     }
   }
   if (cur_row >= 0) flush();
+  pdl_wait();  // this grid ends after the kernel before it (the walk relies on that)
 }
 
 // Request epilogue: one CTA per request.
@@ -310,49 +355,73 @@ __global__ void __launch_bounds__(kWalkThreads) accept_walk_kernel(AcceptParams 
   __shared__ int s_misc[3];
   const int b = blockIdx.x, tid = threadIdx.x;
   const int N = p.N;
-  // The tree and the cache bookkeeping are inputs the argmax kernel does not
-  // write, and this grid starts only after that kernel has waited for all
-  // earlier work: stage them before waiting for the argmax.
-  // a node count outside [0, N] is bad input: the request is skipped, and
-  // only [0, N) is ever indexed
-  const int n_raw = p.n_nodes[b];
-  const int n = min(max(n_raw, 0), N);
-  for (int i = tid; i < n; i += kWalkThreads) {
-    s_par[i] = p.parent[(size_t)b * N + i];
-    s_tok[i] = p.node_tok[(size_t)b * N + i];
-    s_child[i] = 0x7fffffff;
-  }
-  if (tid == 0) {
-    int st = DDT_OK;
-    const int L = p.cache_len[b];
-    const int64_t off = p.cache_off[b];
-    // the rows the compaction may touch on every layer, l * stride + off +
-    // [L, L + n), must lie in the pool
-    const int64_t last = (int64_t)(p.n_layers - 1) * (p.layer_stride_bytes / p.row_bytes) + off + L + n;
-    if (n_raw > N) st = DDT_ERR_INPUT;
-    else if (n > 0 && (off < 0 || L < 0 || last > p.kv_rows)) st = DDT_ERR_BOUNDS;
-    else if (n > 0 && (int64_t)L + n > (int64_t)p.cache_cap[b]) st = DDT_ERR_CAPACITY;
-    s_misc[0] = (n <= 0 || st != DDT_OK);
-    if (p.dev_status) p.dev_status[b] = st;
-  }
+  // the argmax before this kernel starts without waiting for the tree build
+  // and waits for the kernels before it only at its end, so the tree, the
+  // cache bookkeeping and the row keys are all read after this wait, in one
+  // round of independent loads
   pdl_wait();
   // no early trigger of the next kernel: this one writes the pool and
   // cache_len, which a following verify attention reads before it waits
-  // the kernel that produced the row keys gave up a wait: they are not
-  // complete, so nothing is accepted (the keys are still cleared)
-  if (p.status_word != nullptr && tid == 0 && *reinterpret_cast<const volatile int*>(p.status_word) != 0) {
-    s_misc[0] = 1;
-    if (p.dev_status) p.dev_status[b] = DDT_ERR_TIMEOUT;
+  constexpr int kPer = kMaxN / kWalkThreads;
+  const int n_raw = p.n_nodes[b];
+  int L0 = 0, cap0 = 0, sw = 0;  // thread 0's copies
+  int64_t off0 = 0;
+  if (tid == 0) {
+    L0 = p.cache_len[b];
+    off0 = p.cache_off[b];
+    cap0 = p.cache_cap[b];
+    if (p.status_word != nullptr) sw = *reinterpret_cast<const volatile int*>(p.status_word);
   }
-  for (int i = tid; i < N; i += kWalkThreads) {
-    int a = -1;
-    if (i < n) {
-      const unsigned long long k = p.rowkey[(size_t)b * N + i];
-      p.rowkey[(size_t)b * N + i] = 0ull;  // zero for the next call
-      a = static_cast<int>(~static_cast<uint32_t>(k & 0xffffffffull));
-      s_am[i] = a;
+  int32_t r_par[kPer], r_tok[kPer];
+  unsigned long long r_key[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = tid + u * kWalkThreads;
+    if (i < N) {
+      r_par[u] = p.parent[(size_t)b * N + i];
+      r_tok[u] = p.node_tok[(size_t)b * N + i];
+      r_key[u] = p.rowkey[(size_t)b * N + i];
     }
-    if (p.am) p.am[(size_t)b * N + i] = a;
+  }
+  // a node count outside [0, N] is bad input: the request is skipped, and
+  // only [0, N) is ever indexed
+  const int n = min(max(n_raw, 0), N);
+  if (tid == 0) {
+    int st = DDT_OK;
+    // the rows the compaction may touch on every layer, l * stride + off +
+    // [L, L + n), must lie in the pool
+    const int64_t last = (int64_t)(p.n_layers - 1) * (p.layer_stride_bytes / p.row_bytes) + off0 + L0 + n;
+    if (n_raw > N) st = DDT_ERR_INPUT;
+    else if (n > 0 && (off0 < 0 || L0 < 0 || last > p.kv_rows)) st = DDT_ERR_BOUNDS;
+    else if (n > 0 && (int64_t)L0 + n > (int64_t)cap0) st = DDT_ERR_CAPACITY;
+    bool skip = n <= 0 || st != DDT_OK;
+    // the kernel that produced the row keys gave up a wait: they are not
+    // complete, so nothing is accepted (the keys are still cleared)
+    if (sw != 0) {
+      skip = true;
+      st = DDT_ERR_TIMEOUT;
+    }
+    s_misc[0] = skip;
+    if (p.dev_status) p.dev_status[b] = st;
+    // the argmax's work counters back to zero for the next call (its grid has ended)
+    if (b == 0 && p.work != nullptr)
+      for (int k = 0; k < kCounters; ++k) p.work[8 * k] = 0u;
+  }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = tid + u * kWalkThreads;
+    if (i < N) {
+      int a = -1;
+      p.rowkey[(size_t)b * N + i] = 0ull;  // zero for the next call (pad rows have keys too)
+      if (i < n) {
+        a = static_cast<int>(~static_cast<uint32_t>(r_key[u] & 0xffffffffull));
+        s_am[i] = a;
+        s_par[i] = r_par[u];
+        s_tok[i] = r_tok[u];
+        s_child[i] = 0x7fffffff;
+      }
+      if (p.am) p.am[(size_t)b * N + i] = a;
+    }
   }
   __syncthreads();
   const bool skip = s_misc[0] != 0;
@@ -515,6 +584,7 @@ static int launch_walk_and_copy(AcceptParams p, cudaStream_t stream) {
 
 static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 static size_t header_bytes() { return 256; }
+constexpr size_t kWorkCounterOffset = 32;  // the argmax's work counters: header bytes 32, 64, ..., 224
 static size_t zeroed_bytes(int B, int N) { return header_bytes() + round256((size_t)B * N * 8); }
 
 size_t accept_workspace_bytes(int B, int N, int V) {
@@ -546,8 +616,10 @@ static bool bulk_argmax_ready(bool bf16) {
 int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream) {
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   // the first 256 bytes: status word (a bounded wait of the argmax gave up)
+  // at byte 0, the argmax's work counters at bytes 32, 64, ..., 224
   p.abort = reinterpret_cast<int*>(ws);
   p.status_word = reinterpret_cast<const int*>(ws);
+  p.work = reinterpret_cast<unsigned*>(ws + kWorkCounterOffset);
   p.wait_ns = wait_limit_ns();
   p.rowkey = reinterpret_cast<unsigned long long*>(ws + header_bytes());
   const size_t esz = p.logits_dtype == DDT_BF16 ? 2 : 4;
@@ -563,7 +635,7 @@ int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream) 
   const long long reg_warps = (long long)sm_count() * kArgmaxCtasPerSm * (kArgmaxThreads / 32);
   int st;
   if (p.tma && slices <= 2 * reg_warps && bulk_argmax_ready(bf)) {
-    // one CTA of 16 warps per SM, each warp a contiguous range of slices
+    // at most one CTA of 16 warps per SM; warps take chunks of slices
     const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(sm_count(), ceil_div((int)std::min<long long>(
                                                                                                slices, 1LL << 30),
                                                                                            kBulkWarps)));
@@ -587,6 +659,7 @@ int launch_accept_walk(AcceptParams p, void* workspace, cudaStream_t stream) {
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   p.rowkey = reinterpret_cast<unsigned long long*>(ws + header_bytes());
   p.status_word = reinterpret_cast<const int*>(ws);
+  p.work = reinterpret_cast<unsigned*>(ws + kWorkCounterOffset);
   return launch_walk_and_copy(p, stream);
 }
 

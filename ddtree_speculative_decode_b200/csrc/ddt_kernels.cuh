@@ -49,9 +49,10 @@ struct AcceptParams {
   unsigned long long* rowkey;   // [B*N] packed (value, ~index) row maxima (zero between calls)
   const int* status_word;       // nullable: non-zero when the argmax producer gave up a wait
   int* abort;                   // the same word, for the argmax kernel's bounded waits
+  unsigned* work;               // argmax work counter: chunks of slices handed out (zero between calls)
   uint64_t wait_ns;
-  int tma;
-  int layers_apart;             // several layers: a second kernel moves the rows                      // logits rows stream by bulk copies (16-byte aligned rows)
+  int tma;                      // logits rows stream by bulk copies (16-byte aligned rows)
+  int layers_apart;             // several layers: a second kernel moves the rows
 };
 size_t accept_workspace_bytes(int B, int N, int V);
 int launch_accept_compact(AcceptParams p, void* workspace, cudaStream_t stream);

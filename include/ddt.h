@@ -277,10 +277,12 @@ DDT_API int ddt_verify_attn(const void* q, const void* kv, int64_t kv_rows, cons
  *   unchanged. Requests with n_nodes[b] == 0 are skipped the same way with
  *   DDT_OK.
  * workspace: ddt_accept_compact_workspace_size(B, N, V) bytes, 256-byte
- *   aligned: a 256-byte status word, then one 8-byte running argmax key per
- *   row (B * N, rounded up to 256 bytes). All of it must be zero before the
- *   first call -- zero the buffer once after allocating it; every call
- *   leaves it at zero again. The argmax kernel waits (bounded, see
+ *   aligned: a 256-byte header (the status word at byte 0, the argmax's
+ *   seven work counters at bytes 32, 64, ..., 224), then one 8-byte running
+ *   argmax key per row (B * N,
+ *   rounded up to 256 bytes). All of it must be zero before the first call --
+ *   zero the buffer once after allocating it; every call leaves it at zero
+ *   again. The argmax kernel waits (bounded, see
  *   ddt_set_wait_limit_ns) for its own bulk copies; if a wait gives up, the
  *   status word holds DDT_ERR_TIMEOUT, every request reports
  *   DDT_ERR_TIMEOUT and accepts nothing, and later calls with that
@@ -289,12 +291,20 @@ DDT_API int ddt_verify_attn(const void* q, const void* kv, int64_t kv_rows, cons
  * Precondition the library cannot check: the layers and requests own
  *   disjoint rows.
  * Runs as two kernels (three with several layers): the logits stream once,
- *   each warp owning contiguous 2048-entry slices of the rows, brought into
- *   a 3-deep shared-memory ring by 1-D bulk copies (16-byte aligned rows;
- *   plain loads otherwise), row maxima published by 64-bit atomic max; then
+ *   warps taking chunks of 2048-entry row slices from the work counters
+ *   (few rows: brought into a 3-deep shared-memory ring by 1-D bulk copies;
+ *   otherwise 16-byte loads), row maxima published by 64-bit atomic max; then
  *   one CTA per request finds each node's accepted child, walks the path and
  *   (one layer) compacts the rows; with several layers a third kernel moves
  *   the rows, spread over (request, layer group) CTAs.
+ * Launch order: the argmax kernel is a programmatic dependent and reads only
+ *   logits and the workspace, every row of the logits (pad rows too), so it
+ *   may start while the kernel before it in the stream still runs (this
+ *   library's tree build and verify attention let dependents start early);
+ *   it waits for that kernel before it ends, and the walk and compaction run
+ *   after it. So the logits must not be written by a kernel just before the
+ *   call that lets its dependents start early; kernels that are not
+ *   programmatic-launch aware never do.
  */
 DDT_API size_t ddt_accept_compact_workspace_size(int B, int N, int V);
 
@@ -358,7 +368,7 @@ DDT_API int ddt_accept_compact_lmhead(const void* hidden, const void* w_vocab, i
  * the host application, or a latency-critical decode loop that must not call
  * cudaMalloc (which can synchronise the device). This entry point takes the
  * same arguments as ddt_accept_compact minus the workspace and allocates
- * nothing: its scratch (status word and per-row argmax keys) lives in one
+ * nothing: its scratch (status word, work counters and per-row argmax keys) lives in one
  * fixed 4 MiB array inside the library, which every GPU
  * that loads the library keeps until the process exits.
  *
