@@ -10,18 +10,24 @@
 // top-k).
 //
 // A row is split over the CTAs of one cluster (up to 8); each streams its
-// slice once with 16-byte loads, eight in flight per thread. Each thread keeps
-// a running (max, sum of exponentials) for the log-sum-exp; each warp keeps a
-// sorted list of its K best packed keys (order-preserving value bits << 32 |
-// ~index, so a larger key is a larger value or, on equal values, a lower
-// index). A new value costs one compare unless it beats the larger of the
-// warp's K-th best and the best K-th entry any warp of the CTA has published
-// (no value below either can be among the row's K best); the few that do are
-// taken by one out-of-line routine, inserted one by one or, when many lanes
-// hit at once, by a bitonic sort of the hits and a bitonic merge with the
-// list. One warp per CTA merges the warps' lists by K rounds of a warp-wide
-// maximum, and the cluster's first CTA merges the CTAs' lists, read through
-// distributed shared memory, the same way.
+// slice once with 16-byte loads, a round of eight per thread in flight while
+// the round before is processed. Each thread keeps a running (max, sum of
+// exponentials) for the log-sum-exp; each warp keeps a sorted list of its K
+// best packed keys (order-preserving value bits << 32 | ~index, so a larger
+// key is a larger value or, on equal values, a lower index). Aligned rows:
+// after the first round the CTA takes the K-th largest of its threads'
+// maxima (a bisection over order keys, one block-wide count per bit): at
+// least K of its values reach it, so no value below can be among the K
+// best, and from then on a vector costs its log-sum-exp terms, a packed
+// maximum and one warp vote unless its largest value reaches the threshold
+// (the larger of that bound, the warp's K-th best and the best K-th entry
+// any warp of the CTA has published). The few vectors that do are keyed one
+// value at a time; a warp's hits are taken by one out-of-line routine,
+// inserted one by one or, when many lanes hit at once, by a bitonic sort of
+// the hits and a bitonic merge with the list. Unaligned rows take every
+// value through that key path. One warp per CTA merges the warps' lists by
+// K rounds of a warp-wide maximum, and the cluster's first CTA merges the
+// CTAs' lists, read through distributed shared memory, the same way.
 #include <algorithm>
 
 #include "ddt_kernels.cuh"
@@ -243,48 +249,132 @@ __global__ void __launch_bounds__(kDrThreads) drafter_topk_kernel(DrafterParams 
     // eight 16-byte loads in flight per thread (64 KB per CTA) before any is
     // used; whole warps step together (lanes past the end take no values)
     constexpr int kU = 8;
-    bool first = true;
-    for (int e0 = v0 / kPer + warp * 32; e0 < nvec; e0 += kU * kDrThreads) {
-      uint4 v[kU];
+    auto value_of = [](const uint4& r, int t) -> float {
+      const uint32_t w = t < (kBF16 ? 2 : 1) ? r.x : t < (kBF16 ? 4 : 2) ? r.y : t < (kBF16 ? 6 : 3) ? r.z : r.w;
+      if (!kBF16) return __uint_as_float(w);
+      return __uint_as_float((t & 1) ? (w & 0xffff0000u) : (w << 16));
+    };
+    // largest and smallest value of a vector (pairs of bf16 folded first)
+    auto vec_max_min = [](const uint4& r, float& mx, float& mn) {
+      if (kBF16) {
+        auto h = [](uint32_t w) { return *reinterpret_cast<const __nv_bfloat162*>(&w); };
+        const __nv_bfloat162 a = __hmax2(__hmax2(h(r.x), h(r.y)), __hmax2(h(r.z), h(r.w)));
+        const __nv_bfloat162 c = __hmin2(__hmin2(h(r.x), h(r.y)), __hmin2(h(r.z), h(r.w)));
+        mx = fmaxf(__low2float(a), __high2float(a));
+        mn = fminf(__low2float(c), __high2float(c));
+      } else {
+        mx = fmaxf(fmaxf(__uint_as_float(r.x), __uint_as_float(r.y)), fmaxf(__uint_as_float(r.z), __uint_as_float(r.w)));
+        mn = fminf(fminf(__uint_as_float(r.x), __uint_as_float(r.y)), fminf(__uint_as_float(r.z), __uint_as_float(r.w)));
+      }
+    };
+    // One round of kU vectors per lane: the log-sum-exp over every value,
+    // then the keys of the vectors whose largest value reaches the threshold
+    // (thr's value); a vector no lane of the warp needs costs one vote.
+    auto round = [&](const uint4 (&v)[kU], int e0) {
+      float vmax[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int e = e0 + lane + u * kDrThreads;
+        float mx, mn;
+        vec_max_min(v[u], mx, mn);
+        if (e >= nvec) mx = -INFINITY;
+        // a non-finite value: +inf shows in the max, -inf in the min, NaN in
+        // the sum of exponentials below
+        if (e < nvec && !(fabsf(mx) <= 3.402823466e38f && fabsf(mn) <= 3.402823466e38f)) bad = true;
+        vmax[u] = mx;
+        if (e < nvec) {
+          const float ym = mx * kLog2e;
+          if (ym > m) {
+            s *= ex2_ftz(m - ym);
+            m = ym;
+          }
+          float bs = 0.0f;
+#pragma unroll
+          for (int t = 0; t < kPer; ++t) bs += ex2_ftz(fmaf(value_of(v[u], t), kLog2e, -m));
+          s += bs;
+        }
+      }
+      if (!(s == s)) bad = true;
+      refresh();
+      // vectors some lane of the warp may need: a vote each; then one copy of
+      // the key code walks them (kept out of the unrolled path: rare, and the
+      // instruction cache is what a second copy per vector would cost)
+      const float tv = key_value(thr);
+      unsigned need = 0u;
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int e = e0 + lane + u * kDrThreads;
+        if (__any_sync(DDT_FULL_MASK, e < nvec && (thr == 0ull || vmax[u] >= tv))) need |= 1u << u;
+      }
+      while (need) {  // warp-uniform
+        const int u = __ffs(need) - 1;
+        need &= need - 1u;
+        uint4 cur = v[0];
+        float cmax = vmax[0];
+#pragma unroll
+        for (int q = 1; q < kU; ++q)
+          if (q == u) {
+            cur = v[q];
+            cmax = vmax[q];
+          }
+        const int e = e0 + lane + u * kDrThreads;
+        const bool maybe = e < nvec && (thr == 0ull || cmax >= key_value(thr));
+#pragma unroll 1
+        for (int t = 0; t < kPer; ++t) {
+          const float xv = value_of(cur, t);
+          const unsigned long long key =
+              (maybe && fabsf(xv) <= 3.402823466e38f) ? drafter_key(xv, e * kPer + t) : 0ull;
+          const bool hit = key > thr;
+          const unsigned hits = __ballot_sync(DDT_FULL_MASK, hit);
+          if (hits) {  // warp-uniform
+            wl = take_hits(wl, hit ? key : 0ull, hits, p.K, lane);
+            wthr = __shfl_sync(DDT_FULL_MASK, wl, p.K - 1);
+            thr = wthr > thr ? wthr : thr;
+          }
+        }
+      }
+      publish();
+    };
+    // The first round of every warp (all warps take part, lanes past the end
+    // with no values), then the CTA's K-th largest of its threads' maxima by
+    // a bisection over order keys: at least K of the slice's values reach
+    // it, so every value below it is out, and lo starts at that bound. Each
+    // round's loads are issued before the round before it is processed.
+    auto load = [&](uint4 (&v)[kU], int e0) {
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
         const int e = e0 + lane + u * kDrThreads;
         v[u] = e < nvec ? __ldcs(src + e) : make_uint4(0u, 0u, 0u, 0u);
       }
-      if (first) {
-        // each lane's largest key over its first loads, then the K-th
-        // largest of the warp's 32 (0 while fewer than K lanes hold a value)
-        first = false;
-        unsigned long long lk = 0ull;
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int e = e0 + lane + u * kDrThreads;
-          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-          for (int t = 0; t < kPer; ++t) {
-            const float xv = kBF16 ? __uint_as_float((t & 1) ? (w[t >> 1] & 0xffff0000u) : (w[t >> 1] << 16))
-                                   : __uint_as_float(w[t]);
-            const unsigned long long key =
-                (e < nvec && fabsf(xv) <= 3.402823466e38f) ? drafter_key(xv, e * kPer + t) : 0ull;
-            lk = key > lk ? key : lk;
-          }
-        }
-        const unsigned long long kth = __shfl_sync(DDT_FULL_MASK, warp_sort_desc(lk, lane), p.K - 1);
-        lo = kth > 0ull ? kth - 1ull : 0ull;
-      }
+    };
+    int e0 = v0 / kPer + warp * 32;
+    uint4 v[kU], nv[kU];
+    load(v, e0);
+    load(nv, e0 + kU * kDrThreads);
+    {
+      float tm = -INFINITY;
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
         const int e = e0 + lane + u * kDrThreads;
-        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-        float x[8];
-#pragma unroll
-        for (int t = 0; t < kPer; ++t)
-          x[t] = kBF16 ? __uint_as_float((t & 1) ? (w[t >> 1] & 0xffff0000u) : (w[t >> 1] << 16))
-                       : __uint_as_float(w[t]);
-        refresh();
-        batch(x, e < nvec ? kPer : 0, e * kPer);
-        publish();
+        float mx, mn;
+        vec_max_min(v[u], mx, mn);
+        if (e < nvec && fabsf(mx) <= 3.402823466e38f) tm = fmaxf(tm, mx);
       }
+      const uint32_t tk = tm > -INFINITY ? float_order_key(tm) : 0u;
+      uint32_t t = 0u;
+      for (int bit = 31; bit >= 0; --bit) {  // every thread of the CTA, same trips
+        const uint32_t cand = t | (1u << bit);
+        if (__syncthreads_count(tk >= cand) >= p.K) t = cand;
+      }
+      lo = t > 0u ? (static_cast<unsigned long long>(t) << 32) - 1ull : 0ull;
+    }
+    while (e0 < nvec) {  // warp-uniform
+      const int en = e0 + kU * kDrThreads;
+      round(v, e0);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) v[u] = nv[u];
+      if (en + kU * kDrThreads < nvec) load(nv, en + kU * kDrThreads);
+      e0 = en;
     }
   } else {
     for (int i0 = v0 + warp * 32; i0 < v1; i0 += kDrThreads) {  // whole warps step together
