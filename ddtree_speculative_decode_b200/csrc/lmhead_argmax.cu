@@ -19,15 +19,20 @@
 // are verified. The head and hidden tiles stream through a ring of stages by
 // TMA (64 dims per stage, 128-byte swizzle); warp 0 loads, warp 1 of the
 // leader CTA issues the MMAs (with two N parts, warp 6 issues the second
-// part's), warps 2..5 reduce each finished accumulator:
-// per verify row (column) a warp-wide maximum of order-preserving value keys
-// (redux.sync) and the lowest lane holding it (ballot), so every tile yields,
-// per row, (largest logit, lowest vocabulary index) packed in 64 bits. Rows
-// keep their running best in registers across the pass's tiles and publish it
-// once per CTA with a 64-bit atomic max into the same per-row keys the
+// part's), warps 2..5 and 7..10 reduce each finished accumulator (two warps
+// per TMEM lane quarter, alternate 32-column chunks, the next chunk's TMEM
+// load in flight while one is reduced): per verify row (column) the best of
+// the warp's 32 vocabulary rows as a packed 64-bit key (order-preserving
+// value bits << 32 | ~row: the larger key is the larger logit at the lower
+// index), found by halving the columns over the lanes (5 shuffle steps per
+// 32 columns, lane c ending with column c) and merged into the CTA's running
+// key for that column in shared memory; the CTA's keys are published once
+// per pass with a 64-bit atomic max into the same per-row keys the
 // materialised-logits argmax writes, so the accept walk that follows is the
 // same kernel. The accumulator is double-buffered when a pass has at most
-// 256 rows, so the reduction of one tile overlaps the MMAs of the next.
+// 256 rows, so the reduction of one tile overlaps the MMAs of the next; with
+// 512 rows it fills the tensor memory and the reduction (about 15 % of a
+// tile) runs between tiles.
 //
 // Rounding: each MMA adds 16 exact bf16 x bf16 products to the float32
 // accumulator and the 64-dim stages follow one another, so a product passes
@@ -47,7 +52,7 @@ namespace lmh {
 
 using namespace sm100;
 
-constexpr int kThreads = 224;           // warp 0 TMA, warps 1 and 6 MMA (warp 1: + TMEM), warps 2..5 reduction
+constexpr int kThreads = 352;           // warp 0 TMA, warps 1 and 6 MMA (warp 1: + TMEM), warps 2..5 and 7..10 reduction
 constexpr int kABytes = 128 * 128;      // 128 head rows x 64 dims bf16 per CTA and stage
 constexpr int kPassRows = 512;          // verify rows per pass over the head
 constexpr int kMaxStages = 12;
@@ -57,7 +62,7 @@ constexpr int kStageBudget = 200 * 1024;
 constexpr int kBarFull = 0;                      // [kMaxStages] leader: TMA bytes of a stage (both CTAs)
 constexpr int kBarEmpty = kBarFull + kMaxStages;  // [kMaxStages] each CTA: MMAs done with a stage
 constexpr int kBarAccFull = kBarEmpty + kMaxStages;  // [2] each CTA: accumulator buffer complete
-constexpr int kBarAccEmpty = kBarAccFull + 2;        // [2] leader: accumulator read (4 warps x 2 CTAs)
+constexpr int kBarAccEmpty = kBarAccFull + 2;        // [2] leader: accumulator read (8 warps x 2 CTAs)
 constexpr int kNumBars = kBarAccEmpty + 2;
 constexpr int kMiscBytes = 256;                  // barriers
 constexpr int kSlotBytes = 16;                   // TMEM address + abort flag
@@ -78,6 +83,19 @@ struct Params {
   int* abort;
   uint64_t wait_ns;
 };
+
+// Wait for this thread's TMEM loads, with the loaded registers as operands of
+// the wait, so no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+        "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+        "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
 
 __device__ __forceinline__ int ld_volatile_i32(const int* p) {
   int v;
@@ -115,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(kBarAccFull + b), (uint32_t)p.parts);
-      mbar_init(bar(kBarAccEmpty + b), 8);
+      mbar_init(bar(kBarAccEmpty + b), 16);
     }
     fence_mbar_init_cluster();
   }
@@ -206,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok) mma_commit_pair_mc(bar(kBarAccFull + buf), (uint16_t)0x3u);
     }
-  } else if (warp >= 2 && warp <= 5) {
+  } else if ((warp >= 2 && warp <= 5) || (warp >= 7 && warp <= 10)) {
     // ============================================================ reduction
     // thread = TMEM lane 32 q + lane = vocabulary row 128 rank + 32 q + lane
     // of the tile. Per 32-column chunk the warp finds, for every column
@@ -214,7 +232,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // column c's and merges it into the CTA's running key for that column in
     // shared memory. The loop over chunks stays rolled: the code the MMA
     // issuer runs must stay in the instruction cache next to it.
-    const int q = warp & 3;
+    const int q = warp & 3;                 // TMEM lane quarter (two warps each)
+    const int h = warp >= 7 ? 1 : 0;        // which of the quarter's two warps: even or odd chunks
+    const int rt = warp >= 7 ? (int)threadIdx.x - 224 + 128 : (int)threadIdx.x - 64;  // 0 .. 255
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
     const uint32_t empty0 = map_to_rank(bar(kBarAccEmpty), 0);
     const int ncols = p.parts == 2 ? kPassRows : p.npart;
@@ -223,8 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     // the CTA's key per column of the pass out to the rows' global keys
     auto flush = [&](int pass) {
-      named_bar_sync(1, 128);
-      for (int c = (int)threadIdx.x - 64; c < ncols; c += 128) {
+      named_bar_sync(1, 256);
+      for (int c = rt; c < ncols; c += 256) {
         const unsigned long long k = s_red[c];
         s_red[c] = 0ull;
         const int r = pass * kPassRows + c;
@@ -232,9 +252,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = r / p.N, i = r - b * p.N;
         if (i < __ldg(p.n_nodes + b)) atomicMax(p.rowkey + r, k);
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(1, 256);
     };
-    named_bar_sync(1, 128);  // the 4 warps start together (s_red was zeroed before the set-up barrier)
+    named_bar_sync(1, 256);  // the 8 warps start together (s_red was zeroed before the set-up barrier)
     int lt = 0;
     for (int t = pair; t < total; t += npairs, ++lt) {
       const int pass = t / p.vtiles, vt = t - pass * p.vtiles;
@@ -245,33 +265,65 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int buf = lt % p.nbuf;
       if (ok && !mbar_wait(bar(kBarAccFull + buf), (uint32_t)((lt / p.nbuf) & 1), abort, wlim)) ok = false;
       tc_fence_after();
-      const int vrow = vt * 256 + 128 * (int)rank + 32 * q;  // vocabulary row of lane 0
-      const bool valid = ok && vrow + lane < p.V;
+      const int vrow = vt * 256 + 128 * (int)rank + 32 * q + lane;  // this thread's vocabulary row
+      const bool valid = ok && vrow < p.V;
       const uint32_t col0 = (uint32_t)(buf * p.parts * 256);
-#pragma unroll 1
-      for (int m = 0; m < nchunks; ++m) {
-        uint32_t r[32];
-        tmem_ld32(lane_addr + col0 + 32u * (uint32_t)m, r);
-        tmem_wait_ld();
-        if (m == nchunks - 1) {
-          // the accumulator buffer is free for the next tile's MMAs
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            if (leader) mbar_arrive_local(bar(kBarAccEmpty + buf));
-            else mbar_arrive_cluster(empty0 + 8u * (uint32_t)buf);
+      // per column, the best (value, lowest row) over the warp's 32 rows as
+      // packed keys (order-preserving value << 32 | ~row), by halving: at
+      // width h a lane keeps the upper h columns of its 2h if its h bit is
+      // set, the lower ones otherwise, and takes the larger of its key and
+      // its partner's (lane ^ h) for each; after h = 16 .. 1 lane l holds
+      // column l of the chunk
+      auto reduce = [&](const uint32_t (&r)[32], int m) {
+        unsigned long long k[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          k[i] = valid ? ((unsigned long long)float_order_key(__uint_as_float(r[i])) << 32) |
+                             (unsigned long long)(~(uint32_t)vrow)
+                       : 0ull;
+#pragma unroll
+        for (int h = 16; h >= 1; h >>= 1) {
+          const bool up = (lane & h) != 0;
+#pragma unroll
+          for (int i = 0; i < h; ++i) {
+            const unsigned long long keep = up ? k[i + h] : k[i];
+            const unsigned long long send = up ? k[i] : k[i + h];
+            const unsigned long long got = __shfl_xor_sync(DDT_FULL_MASK, send, h);
+            k[i] = got > keep ? got : keep;
           }
         }
-        unsigned long long mine = 0ull;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const uint32_t key = valid ? float_order_key(__uint_as_float(r[i])) : 0u;
-          const uint32_t mx = __reduce_max_sync(DDT_FULL_MASK, key);
-          const uint32_t hit = __ballot_sync(DDT_FULL_MASK, key == mx);
-          if (lane == i && mx != 0u)
-            mine = ((unsigned long long)mx << 32) | (unsigned long long)(~(uint32_t)(vrow + __ffs(hit) - 1));
+        if (k[0] != 0ull) atomicMax(s_red + 32 * m + lane, k[0]);
+      };
+      // after this warp's last chunk's load its columns of the accumulator
+      // are in registers: once all eight warps of both CTAs have arrived the
+      // buffer is free for the next tile's MMAs
+      auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader) mbar_arrive_local(bar(kBarAccEmpty + buf));
+          else mbar_arrive_cluster(empty0 + 8u * (uint32_t)buf);
         }
-        if (mine != 0ull) atomicMax(s_red + 32 * m + lane, mine);
+      };
+      // this warp's chunks h, h + 2, ...; two register buffers: the next
+      // one loads while this one is reduced
+      const int cnt = nchunks > h ? (nchunks - h + 1) / 2 : 0;
+      auto col = [&](int j) { return lane_addr + col0 + 32u * (uint32_t)(h + 2 * j); };
+      uint32_t ra[32], rb[32];
+      if (cnt == 0) release();  // nothing to read in this buffer
+      else tmem_ld32(col(0), ra);
+#pragma unroll 1
+      for (int j = 0; j < cnt; j += 2) {
+        tmem_wait_ld_regs(ra);
+        if (j + 1 < cnt) tmem_ld32(col(j + 1), rb);
+        if (j + 1 == cnt) release();
+        reduce(ra, h + 2 * j);
+        if (j + 1 < cnt) {
+          tmem_wait_ld_regs(rb);
+          if (j + 2 < cnt) tmem_ld32(col(j + 2), ra);
+          if (j + 2 == cnt) release();
+          reduce(rb, h + 2 * (j + 1));
+        }
       }
     }
     if (cur_pass >= 0) flush(cur_pass);
