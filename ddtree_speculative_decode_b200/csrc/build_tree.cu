@@ -1,4 +1,5 @@
-// Best-first draft-tree build: one warp per request.
+// Best-first draft-tree build: one warp per request, or one CTA per request
+// for wide, shallow trees (the level-synchronous build further down).
 //
 // What it computes is fixed in ddt.h (ddt_build_tree): the first N - 1 rank
 // paths in (score desc, depth asc, ranks lexicographic asc) order, scores as
@@ -18,6 +19,8 @@
 // packed integer: ceil(log2 K) bits per level, first level most significant,
 // so equal-depth paths compare as integers. Ancestor masks are filled after
 // selection, one lane per node, by walking parent pointers (parent < child).
+#include <mutex>
+
 #include "ddt_kernels.cuh"
 
 namespace ddt {
@@ -576,6 +579,410 @@ __global__ void __launch_bounds__(32) build_tree_packed_kernel(BuildParams p) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Level-synchronous build for shallow, wide trees (one CTA of 512 threads per
+// request). With M = N - 1 paths wanted, let list_d be the best M paths of
+// depth d in (score desc, rank tuple asc) order among the children of
+// list_{d-1} (list_0 = the root). The first M paths of the whole order are
+// the best M of the union of the lists: a depth-d path left out of list_d
+// has M better paths of its own depth, and a path whose prefix was left out
+// ranks after that prefix, which already has M better paths. Each level's
+// best M (and finally the union's) are found by a radix select over the
+// packed order key (inverted score key, depth, rank tuple), one byte per
+// pass, most significant first, with shared-memory histograms; the final M
+// are then placed by their ranks among one another, so node i is the i-th
+// path of the best-first search's pops.
+// ---------------------------------------------------------------------------
+constexpr int kLvThreads = 512;
+constexpr int kLvMaxN = 256;     // M <= 255 entries per level
+constexpr int kLvMaxD = 16;
+constexpr int kLvMaxP = 4096;    // candidates of a level (at most 255 x 16) or the union (16 x 255)
+
+struct LvCand {
+  uint32_t hi;   // ~order key of the score: smaller is better
+  uint32_t tag;  // depth << 16 | index (index = parent entry * K + rank, or entry of its level)
+  uint64_t k;    // packed rank tuple: smaller is lexicographically first
+};
+
+__device__ __forceinline__ bool lv_less(const LvCand& a, const LvCand& b) {
+  if (a.hi != b.hi) return a.hi < b.hi;
+  if ((a.tag >> 16) != (b.tag >> 16)) return (a.tag >> 16) < (b.tag >> 16);
+  return a.k < b.k;
+}
+
+struct LvSmem {
+  LvCand cand[kLvMaxP];
+  LvCand order[kLvMaxN];             // the union's first M, then in order
+  float sc[kLvMaxD][kLvMaxN];
+  uint64_t key[kLvMaxD][kLvMaxN];
+  int16_t par[kLvMaxD][kLvMaxN];     // entry of the level above (-1: the root)
+  uint8_t rk[kLvMaxD][kLvMaxN];      // last rank
+  int16_t node[kLvMaxD][kLvMaxN];    // node index, or 0 when not among the first M
+  int32_t n_parent[kLvMaxN];
+  float lp[kLvMaxD * 32];
+  int32_t tk[kLvMaxD * 32];
+  int cnt[kLvMaxD + 1];
+  int hist[kLvThreads / 32][256];   // one histogram per warp (no contention between warps)
+  uint32_t lo_hi, hi_hi;             // smallest and largest hi of the candidates
+  uint32_t t_hi, t_dep;              // radix select: threshold's decided bits
+  uint64_t t_k;
+  int sel_digit, sel_rank, sel_full;
+  int fill;
+  int wsum[kLvThreads / 32];
+  int bad;
+};
+
+__device__ __forceinline__ uint32_t lv_hi(float sc) { return ~float_order_key(sc); }
+__device__ __forceinline__ float lv_score(uint32_t hi) {
+  const uint32_t u = ~hi;
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+// Radix select over S.cand[0, P): after it, a candidate is among the `want`
+// smallest keys iff lv_in(...) holds. Key bits, most significant first: hi
+// (32), depth (8, only when `depth`), k (64); one byte per pass. Passes stop
+// once every candidate sharing the decided prefix is taken.
+struct LvSel {
+  uint32_t m_hi, m_dep;  // decided bits
+  uint64_t m_k;
+};
+
+__device__ __forceinline__ bool lv_match(const LvSmem& S, const LvSel& m, const LvCand& c) {
+  return ((c.hi ^ S.t_hi) & m.m_hi) == 0u && (((c.tag >> 16) ^ S.t_dep) & m.m_dep) == 0u &&
+         ((c.k ^ S.t_k) & m.m_k) == 0ull;
+}
+
+// taken: the decided bits of the key are at most the threshold's
+__device__ __forceinline__ bool lv_in(const LvSmem& S, const LvSel& m, const LvCand& c) {
+  const uint32_t a = c.hi & m.m_hi, ta = S.t_hi & m.m_hi;
+  if (a != ta) return a < ta;
+  const uint32_t d = (c.tag >> 16) & m.m_dep, td = S.t_dep & m.m_dep;
+  if (d != td) return d < td;
+  return (c.k & m.m_k) <= (S.t_k & m.m_k);
+}
+
+// Exclusive offset of this thread's count among the CTA's threads (thread
+// order), and the total; the whole CTA calls it.
+__device__ __forceinline__ int lv_offset(LvSmem& S, int count, int& total) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int incl = count;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(DDT_FULL_MASK, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) S.wsum[warp] = incl;
+  __syncthreads();
+  int base = 0;
+  total = 0;
+  for (int w = 0; w < kLvThreads / 32; ++w) {
+    const int v = S.wsum[w];
+    if (w < warp) base += v;
+    total += v;
+  }
+  __syncthreads();
+  return base + incl - count;
+}
+
+// Radix select over S.cand[0, P): afterwards a candidate is among the `want`
+// smallest keys iff lv_in holds. The key, most significant first: hi (32
+// bits), depth (8, only when `depth`), k (kbits: the rank tuples' width).
+// Each pass histograms the next window of up to 8 undecided bits of the
+// candidates that match the decided prefix; hi's windows start at the first
+// bit where the candidates' scores differ. Passes stop once every candidate
+// sharing the decided prefix is taken (keys are distinct).
+__device__ LvSel lv_select(LvSmem& S, int P, int want, bool depth, int kbits) {
+  LvSel m{0u, 0u, 0ull};
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    S.t_hi = 0u;
+    S.t_dep = 0u;
+    S.t_k = 0ull;
+    S.lo_hi = 0xffffffffu;
+    S.hi_hi = 0u;
+  }
+  __syncthreads();
+  if (want >= P) return m;  // every candidate is taken
+  {
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int i = tid; i < P; i += kLvThreads) {
+      const uint32_t v = S.cand[i].hi;
+      lo = min(lo, v);
+      hi = max(hi, v);
+    }
+    lo = __reduce_min_sync(DDT_FULL_MASK, lo);
+    hi = __reduce_max_sync(DDT_FULL_MASK, hi);
+    if ((tid & 31) == 0) {
+      atomicMin(&S.lo_hi, lo);
+      atomicMax(&S.hi_hi, hi);
+    }
+  }
+  __syncthreads();
+  const uint32_t diff = S.lo_hi ^ S.hi_hi;
+  int hi_top = diff ? 31 - __clz(diff) : -1;  // highest undecided bit of hi (the bits above agree)
+  m.m_hi = hi_top < 0 ? 0xffffffffu : (hi_top >= 31 ? 0u : ~((2u << hi_top) - 1u));
+  const uint32_t t_hi0 = S.lo_hi & m.m_hi;
+  __syncthreads();
+  if (tid == 0) S.t_hi = t_hi0;
+  bool dep_left = depth;
+  int k_top = kbits - 1;
+  __syncthreads();
+  int rank = want;  // how many of the candidates matching the prefix are still to take
+  for (;;) {
+    int field, lo, width;
+    if (hi_top >= 0) {
+      field = 0;
+      lo = hi_top >= 7 ? hi_top - 7 : 0;
+      width = hi_top - lo + 1;
+    } else if (dep_left) {
+      field = 1;
+      lo = 0;
+      width = 8;
+    } else if (k_top >= 0) {
+      field = 2;
+      lo = k_top >= 7 ? k_top - 7 : 0;
+      width = k_top - lo + 1;
+    } else {
+      break;  // every bit decided
+    }
+    const uint32_t wmask = (1u << width) - 1u;
+    const int warp = tid >> 5;
+    for (int i = tid; i < (kLvThreads / 32) * 256; i += kLvThreads) (&S.hist[0][0])[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < P; i += kLvThreads) {
+      const LvCand c = S.cand[i];
+      if (!lv_match(S, m, c)) continue;
+      const uint32_t v = field == 0 ? c.hi >> lo : field == 1 ? (c.tag >> 16) : (uint32_t)(c.k >> lo);
+      atomicAdd(&S.hist[warp][v & wmask], 1);  // this warp's own histogram
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // bins 8 lane .. 8 lane + 7 summed over the warps: the bin where the
+      // running count reaches rank
+      const int lane = tid;
+      int h[8], sum = 0;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        int v = 0;
+#pragma unroll
+        for (int w = 0; w < kLvThreads / 32; ++w) v += S.hist[w][8 * lane + t];
+        h[t] = v;
+        sum += v;
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(DDT_FULL_MASK, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int before = incl - sum;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (before < rank && rank <= before + h[t]) {
+          S.sel_digit = 8 * lane + t;
+          S.sel_rank = rank - before;
+          S.sel_full = (h[t] == rank - before) ? 1 : 0;
+        }
+        before += h[t];
+      }
+    }
+    __syncthreads();
+    const uint32_t dg = (uint32_t)S.sel_digit;
+    rank = S.sel_rank;
+    const bool full = S.sel_full != 0;
+    if (field == 0) {
+      m.m_hi |= wmask << lo;
+      if (tid == 0) S.t_hi |= dg << lo;
+      hi_top = lo - 1;
+    } else if (field == 1) {
+      m.m_dep |= 0xffu;
+      if (tid == 0) S.t_dep |= dg;
+      dep_left = false;
+    } else {
+      m.m_k |= (uint64_t)wmask << lo;
+      if (tid == 0) S.t_k |= (uint64_t)dg << lo;
+      k_top = lo - 1;
+    }
+    __syncthreads();
+    if (full) break;
+  }
+  return m;
+}
+
+__global__ void __launch_bounds__(kLvThreads) build_tree_level_kernel(BuildParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  LvSmem& S = *reinterpret_cast<LvSmem*>(smem_raw);
+  pdl_wait();
+  pdl_launch_dependents();
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int N = p.N, D = p.D, K = p.K, W = p.W, bpl = p.bpl;
+  const int M = N - 1;
+  const int L = p.cache_len[b];
+  const int root = p.root_tok[b];
+  if (tid < 32) {
+    const bool bad = load_drafter(p, b, S.lp, S.tk, tid);
+    if (tid == 0) S.bad = bad ? 1 : 0;
+  }
+  __syncthreads();
+  const bool bad = S.bad != 0;
+  int32_t* o_tok = p.node_tok + (size_t)b * N;
+  int32_t* o_par = p.parent + (size_t)b * N;
+  int32_t* o_dep = p.depth + (size_t)b * N;
+  int32_t* o_pos = p.pos + (size_t)b * N;
+  float* o_sc = p.score + (size_t)b * N;
+  uint32_t* o_mask = p.mask + (size_t)b * N * W;
+  int n = 0;
+  if (!bad) {
+    // levels: list_d = the best M children of list_{d-1}
+    int prev = 1;  // list_0: the root
+    int total = 0;
+    for (int d = 1; d <= D && M > 0; ++d) {
+      const int P = prev * K;
+      for (int i = tid; i < P; i += kLvThreads) {
+        const int j = i / K, r = i - j * K;
+        const float ps = d == 1 ? 0.0f : S.sc[d - 2][j];
+        const uint64_t pk = d == 1 ? 0ull : S.key[d - 2][j];
+        LvCand c;
+        c.hi = lv_hi(__fadd_rn(ps, S.lp[(d - 1) * K + r]));
+        c.tag = (uint32_t)i;  // depth 0 here: every candidate of the level has the same one
+        c.k = (pk << bpl) | (uint64_t)r;
+        S.cand[i] = c;
+      }
+      if (tid == 0) S.fill = 0;
+      __syncthreads();
+      const int cnt = P < M ? P : M;
+      const LvSel m = lv_select(S, P, cnt, false, bpl * d);
+      {
+        // the taken candidates, in thread order, at offsets from a block scan
+        int mine = 0;
+        for (int i = tid; i < P; i += kLvThreads) mine += lv_in(S, m, S.cand[i]) ? 1 : 0;
+        int tot = 0;
+        int e = lv_offset(S, mine, tot);
+        for (int i = tid; i < P; i += kLvThreads) {
+          const LvCand c = S.cand[i];
+          if (!lv_in(S, m, c)) continue;
+          if (e < kLvMaxN) {  // exactly cnt are taken (keys are distinct)
+            const int ci = (int)(c.tag & 0xffffu);
+            const int j = ci / K, r = ci - j * K;
+            S.sc[d - 1][e] = lv_score(c.hi);
+            S.key[d - 1][e] = c.k;
+            S.par[d - 1][e] = (int16_t)(d == 1 ? -1 : j);
+            S.rk[d - 1][e] = (uint8_t)r;
+          }
+          ++e;
+        }
+      }
+      if (tid == 0) S.cnt[d] = cnt;
+      __syncthreads();
+      prev = cnt;
+      total += cnt;
+    }
+    // the union's best M, then their order by ranks among one another
+    const int levels = total > 0 ? D : 0;
+    for (int i = tid; i < total; i += kLvThreads) {
+      int d = 1, e = i;
+      while (d <= levels && e >= S.cnt[d]) {
+        e -= S.cnt[d];
+        ++d;
+      }
+      LvCand c;
+      c.hi = lv_hi(S.sc[d - 1][e]);
+      c.tag = ((uint32_t)d << 16) | (uint32_t)e;
+      c.k = S.key[d - 1][e];
+      S.cand[i] = c;
+    }
+    for (int i = tid; i < kLvMaxD * kLvMaxN; i += kLvThreads) (&S.node[0][0])[i] = 0;
+    if (tid == 0) S.fill = 0;
+    __syncthreads();
+    const int sel = total < M ? total : M;
+    if (sel > 0) {
+      const LvSel m = lv_select(S, total, sel, true, bpl * D);
+      {
+        int mine = 0;
+        for (int i = tid; i < total; i += kLvThreads) mine += lv_in(S, m, S.cand[i]) ? 1 : 0;
+        int tot = 0;
+        int q = lv_offset(S, mine, tot);
+        for (int i = tid; i < total; i += kLvThreads) {
+          const LvCand c = S.cand[i];
+          if (!lv_in(S, m, c)) continue;
+          if (q < kLvMaxN) S.order[q] = c;  // exactly sel are taken
+          ++q;
+        }
+      }
+      __syncthreads();
+      // rank of each taken path among the others: two threads per path, each
+      // counting over half of them
+      LvCand mine;
+      int rank = 0;
+      const int me = tid >> 1, half = tid & 1;
+      if (me < sel) {
+        mine = S.order[me];
+        const int u0 = half ? sel / 2 : 0, u1 = half ? sel : sel / 2;
+#pragma unroll 4
+        for (int u = u0; u < u1; ++u) rank += lv_less(S.order[u], mine) ? 1 : 0;
+      }
+      rank += __shfl_xor_sync(DDT_FULL_MASK, rank, 1);
+      __syncthreads();
+      if (me < sel && half == 0) {
+        S.cand[rank] = mine;
+        S.node[(mine.tag >> 16) - 1][mine.tag & 0xffffu] = (int16_t)(rank + 1);
+      }
+      __syncthreads();
+    }
+    n = 1 + sel;
+    // outputs: node 0 the root, node q + 1 the q-th path
+    for (int i = tid; i < n; i += kLvThreads) {
+      if (i == 0) {
+        o_tok[0] = root;
+        o_par[0] = -1;
+        o_dep[0] = 0;
+        o_pos[0] = L;
+        o_sc[0] = 0.0f;
+        S.n_parent[0] = -1;
+      } else {
+        const uint32_t tag = S.cand[i - 1].tag;
+        const int d = (int)(tag >> 16), e = (int)(tag & 0xffffu);
+        const int pe = S.par[d - 1][e];
+        const int pn = d == 1 ? 0 : (int)S.node[d - 2][pe];
+        o_tok[i] = S.tk[(d - 1) * K + S.rk[d - 1][e]];
+        o_par[i] = pn;
+        o_dep[i] = d;
+        o_pos[i] = L + d;
+        o_sc[i] = S.sc[d - 1][e];
+        S.n_parent[i] = pn;
+      }
+    }
+    __syncthreads();
+    // ancestor masks: one thread per node walks its parent chain (parent < child)
+    for (int i = tid; i < n; i += kLvThreads) {
+      uint32_t mk[kLvMaxN / 32];
+#pragma unroll
+      for (int w = 0; w < kLvMaxN / 32; ++w) mk[w] = 0u;
+      for (int j = i; j >= 0; j = S.n_parent[j]) {
+#pragma unroll
+        for (int w = 0; w < kLvMaxN / 32; ++w)
+          if ((j >> 5) == w) mk[w] |= 1u << (j & 31);
+      }
+      uint32_t* row = o_mask + (size_t)i * W;
+      for (int w = 0; w < W; ++w) row[w] = w < kLvMaxN / 32 ? mk[w] : 0u;
+    }
+  }
+  // pad rows [n, N)
+  for (int i = n + tid; i < N; i += kLvThreads) {
+    o_tok[i] = -1;
+    o_par[i] = -1;
+    o_dep[i] = -1;
+    o_pos[i] = -1;
+    o_sc[i] = -INFINITY;
+    uint32_t* row = o_mask + (size_t)i * W;
+    for (int w = 0; w < W; ++w) row[w] = 0u;
+  }
+  if (tid == 0) {
+    p.n_nodes[b] = n;
+    if (p.dev_status) p.dev_status[b] = bad ? DDT_ERR_INPUT : DDT_OK;
+  }
+}
+
 template <int SPL>
 static int launch_packed(const BuildParams& p, cudaStream_t stream) {
   const size_t smem = (size_t)p.N * 12 + (size_t)p.D * p.K * 8;
@@ -598,6 +1005,29 @@ static int launch_sorted(const BuildParams& p, cudaStream_t stream) {
   return launch_pdl(build_tree_sorted_kernel<SPL>, (unsigned)p.B, 32, smem, stream, p);
 }
 
+// The level build's shared-memory opt-in, set once per device (the attribute
+// applies to the device current when it is set).
+static bool level_build_ready() {
+  static std::mutex mu;
+  static int done[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev] == 0) {
+    const cudaError_t e = cudaFuncSetAttribute(build_tree_level_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)sizeof(LvSmem));
+    done[dev] = e == cudaSuccess ? 1 : -1;
+    if (e != cudaSuccess) (void)cudaGetLastError();
+  }
+  return done[dev] == 1;
+}
+
+// The level build pays D sorts of up to (N - 1) x K candidates; the warp
+// build pays N - 1 pops whose cost grows with the frontier it keeps sorted.
+static bool use_level_build(const BuildParams& p) {
+  return p.N > 128 && p.N <= kLvMaxN && p.D <= kLvMaxD && p.K <= 16;
+}
+
 int launch_build_tree(const BuildParams& p, cudaStream_t stream) {
   // every entry that can exist has depth <= min(D, N): its rank tuple needs
   // bpl bits per level
@@ -607,6 +1037,10 @@ int launch_build_tree(const BuildParams& p, cudaStream_t stream) {
   if (packed && p.N <= 256) return launch_packed<4>(p, stream);
   if (p.N <= 64) return launch_sorted<1>(p, stream);
   if (p.N <= 128) return launch_sorted<2>(p, stream);
+  if (use_level_build(p)) {
+    if (!level_build_ready()) return DDT_ERR_CUDA;
+    return launch_pdl(build_tree_level_kernel, (unsigned)p.B, kLvThreads, sizeof(LvSmem), stream, p);
+  }
   if (p.N <= 256) return launch_sorted<4>(p, stream);
   const size_t smem = build_smem_bytes(p.N, p.D, p.K);
   if (smem > 48 * 1024) {

@@ -156,7 +156,10 @@ DDT_API int ddt_drafter_topk(const void* logits, int logits_dtype, int V, int R,
  *   dev_status [B] int32 (nullable): DDT_OK, or DDT_ERR_INPUT when logp[b]
  *   breaks its precondition -- that request then gets n_nodes = 0 and every
  *   row padded.
- * One warp per request; no workspace.
+ * One warp per request (a best-first search; for 128 < N <= 256 with D <= 16
+ * and K <= 16 and rank tuples wider than 25 bits, one CTA of 512 threads per
+ * request that selects the best N - 1 paths depth by depth with radix
+ * selects, the same nodes in the same order); no workspace.
  */
 DDT_API int ddt_build_tree(const float* logp, const int32_t* tok, const int32_t* root_tok,
                    const int32_t* cache_len, int B, int D, int K, int N,

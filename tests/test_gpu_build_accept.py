@@ -56,11 +56,13 @@ def test_build_named(name):
 
 # Covers every kernel variant: rank tuples that fit a 25-bit field (bits per
 # level x min(D, N) <= 25) with N <= 64 / 128 / 256, wider tuples with the same
-# three budgets, and N > 256 (shared-memory frontier); 25 and 28 bits sit on
-# either side of the packed-key limit.
+# three budgets (N 129..256 with D <= 16 and K <= 16: the level-synchronous
+# build), and N > 256 (shared-memory frontier); 25 and 28 bits sit on either
+# side of the packed-key limit.
 EDGE = [(1, 1, 1), (3, 2, 2), (4, 3, 31), (4, 3, 32), (4, 3, 33), (8, 8, 255), (8, 8, 256), (8, 16, 1024),
         (16, 8, 128), (5, 1, 40), (2, 32, 700), (64, 2, 64), (12, 31, 300), (8, 8, 100), (16, 8, 200),
-        (5, 32, 64), (7, 16, 64), (25, 2, 26), (26, 2, 27)]
+        (5, 32, 64), (7, 16, 64), (25, 2, 26), (26, 2, 27), (8, 16, 256), (7, 16, 129), (16, 16, 256),
+        (7, 13, 250), (20, 8, 256)]
 
 
 @pytest.mark.parametrize("D,K,N", EDGE)
