@@ -627,7 +627,6 @@ struct LvSmem {
   uint32_t t_hi, t_dep;              // radix select: threshold's decided bits
   uint64_t t_k;
   int sel_digit, sel_rank, sel_full;
-  int fill;
   int wsum[kLvThreads / 32];
   int bad;
 };
@@ -848,7 +847,6 @@ __global__ void __launch_bounds__(kLvThreads) build_tree_level_kernel(BuildParam
         c.k = (pk << bpl) | (uint64_t)r;
         S.cand[i] = c;
       }
-      if (tid == 0) S.fill = 0;
       __syncthreads();
       const int cnt = P < M ? P : M;
       const LvSel m = lv_select(S, P, cnt, false, bpl * d);
@@ -892,7 +890,6 @@ __global__ void __launch_bounds__(kLvThreads) build_tree_level_kernel(BuildParam
       S.cand[i] = c;
     }
     for (int i = tid; i < kLvMaxD * kLvMaxN; i += kLvThreads) (&S.node[0][0])[i] = 0;
-    if (tid == 0) S.fill = 0;
     __syncthreads();
     const int sel = total < M ? total : M;
     if (sel > 0) {

@@ -398,3 +398,39 @@ def test_accept_status_word_timeout_skips_everything():
     assert int(ws[256:].view(torch.int64).abs().sum().item()) == 0
     ws.zero_()
     _run_accept_and_compare(s, x, tree, logits)
+
+
+@pytest.mark.parametrize("B,N,V,pad", [(1, 64, 163840, 0), (4, 128, 163840, 0), (3, 40, 20000, 9)])
+def test_accept_leaves_workspace_zero(B, N, V, pad):
+    """The argmax hands out its slices through counters in the workspace
+    header and reduces every row, pad rows included; after the call the whole
+    workspace (status word, counters, every row's key) is zero again, so the
+    next call on it starts clean. Two calls in a row give the same outputs.
+    (64 and 512 rows take the bulk-copy and the register-fed argmax.)"""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(B * 1000 + N)
+    lg = torch.randn(B, N, V, generator=g, device=DEV).to(torch.bfloat16)
+    nt = torch.zeros(B, N, dtype=torch.int32, device=DEV)
+    par = torch.full((B, N), -1, dtype=torch.int32, device=DEV)
+    par[:, 1:] = 0
+    nn = torch.full((B,), N - pad, dtype=torch.int32, device=DEV)
+    kv = torch.zeros(B * (N + 8), 64, dtype=torch.bfloat16, device=DEV)
+    off = (torch.arange(B, device=DEV) * (N + 8)).to(torch.int64)
+    cap = torch.full((B,), N + 8, dtype=torch.int32, device=DEV)
+    ws = torch.zeros(lib.accept_compact_workspace_size(B, N, V), dtype=torch.uint8, device=DEV)
+    outs = []
+    for _ in range(2):
+        cl = torch.zeros(B, dtype=torch.int32, device=DEV)
+        out = lib.accept_compact(lg, nt, par, nn, kv, off, cl, cap, workspace=ws)
+        torch.cuda.synchronize()
+        assert int(ws.to(torch.int64).abs().sum().item()) == 0
+        outs.append({k: v.cpu().numpy() for k, v in out.items()})
+    for k in ("am", "acc_len", "acc_nodes", "out_tok", "bonus", "status"):
+        assert np.array_equal(outs[0][k], outs[1][k]), k
+    # the argmax itself: every real row against the oracle's (lowest index on ties)
+    ref = oracle.row_argmax(lg.float().cpu().numpy())
+    am = outs[0]["am"]
+    for b in range(B):
+        n = N - pad
+        assert np.array_equal(am[b, :n], ref[b, :n])
+        assert np.all(am[b, n:] == -1)
