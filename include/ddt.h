@@ -284,8 +284,9 @@ DDT_API int ddt_verify_attn(const void* q, const void* kv, int64_t kv_rows, cons
  *   seven work counters at bytes 32, 64, ..., 224), then one 8-byte running
  *   argmax key per row (B * N,
  *   rounded up to 256 bytes). All of it must be zero before the first call --
- *   zero the buffer once after allocating it; every call leaves it at zero
- *   again. The argmax kernel waits (bounded, see
+ *   zero the buffer once after allocating it; every call that returns DDT_OK
+ *   leaves it at zero again (after a call that returned an error, zero it
+ *   again before the next). The argmax kernel waits (bounded, see
  *   ddt_set_wait_limit_ns) for its own bulk copies; if a wait gives up, the
  *   status word holds DDT_ERR_TIMEOUT, every request reports
  *   DDT_ERR_TIMEOUT and accepts nothing, and later calls with that
