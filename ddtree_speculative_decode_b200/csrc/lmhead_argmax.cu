@@ -210,12 +210,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const uint32_t a0 = sbase + (uint32_t)(slot * p.stage_bytes);
+        // descriptors once per stage: +32 bytes per K step is +2 in the address field
+        const uint64_t da = smem_desc_sw128(a0, 16, 1024);
+        for (int j = j0; j < j1; ++j) {
+          const uint64_t db = smem_desc_sw128(a0 + kABytes + (uint32_t)(j * p.nh * 128), 16, 1024);
+          const uint32_t d = tmem + (uint32_t)((buf * p.parts + j) * 256);
+          mma_pair_ss(d, da, db, idesc, kb != 0 ? 1u : 0u);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          for (int j = j0; j < j1; ++j)
-            mma_pair_ss(tmem + (uint32_t)((buf * p.parts + j) * 256), smem_desc_sw128(a0 + 32 * k, 16, 1024),
-                        smem_desc_sw128(a0 + kABytes + (uint32_t)(j * p.nh * 128) + 32 * k, 16, 1024), idesc,
-                        (kb | k) != 0 ? 1u : 0u);
+          for (int k = 1; k < 4; ++k) mma_pair_ss(d, da + 2 * k, db + 2 * k, idesc, 1u);
+        }
         mma_commit_pair_mc(bar(kBarEmpty + slot), (uint16_t)0x3u);
         if (++slot == p.stages) {
           slot = 0;

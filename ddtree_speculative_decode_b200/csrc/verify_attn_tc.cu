@@ -471,11 +471,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t a0 = sbase + kOffKRing + rg.slot * kKStageBytes;
-          const uint32_t b0 = a0 + kBoxBytes;
+          // descriptors once per stage: +32 bytes per K step is +2 in the address field
+          const uint64_t da = smem_desc_sw128(a0, 16, 1024), db = smem_desc_sw128(a0 + kBoxBytes, 16, 1024);
+          mma_pair_ss(d, da, db, kIdescQK, ch != 0);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_pair_ss(d, smem_desc_sw128(a0 + 32 * k, 16, 1024), smem_desc_sw128(b0 + 32 * k, 16, 1024), kIdescQK,
-                        (ch | k) != 0);
+          for (int k = 1; k < 4; ++k) mma_pair_ss(d, da + 2 * k, db + 2 * k, kIdescQK, 1u);
           if (rg.slot % kKGroup == kKGroup - 1) mma_commit_pair_mc(bar(kBarKEmpty + rg.slot / kKGroup), pmask);
           if (++rg.slot == kKStages) { rg.slot = 0; rg.phase ^= 1u; }
         }
@@ -489,16 +489,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t >= u.tt) unit_tree(p, u);  // live key groups of a tile that reaches tree keys
         const int ng = live_groups(u, t);
         for (int g = 0; g < ng && ok; ++g) {
-          const uint32_t a0 = sbase + kOffP + g * kBoxBytes;
+          const uint64_t da = smem_desc_sw128(sbase + kOffP + g * kBoxBytes, 16, 1024);
           for (int j = 0; j < 2; ++j) {
             if (!mbar_wait(bar(kBarVFull + rg.slot), rg.phase, abort, wlim)) { ok = false; break; }
-            const uint32_t b0 = sbase + kOffVRing + rg.slot * kVStageBytes;
+            // +2048 bytes per K step (16 keys) is +128 in the address field
+            const uint64_t db = smem_desc_sw128(sbase + kOffVRing + rg.slot * kVStageBytes, kBoxBytes, 1024);
             const uint32_t d = tmem + (j ? kColO1 : kColO0);
+            mma_pair_ss(d, da, db, kIdescPV, (t > 0 || g > 0) ? 1u : 0u);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_pair_ss(d, smem_desc_sw128(a0 + 32 * k, 16, 1024),
-                          smem_desc_sw128(b0 + 2048 * k, kBoxBytes, 1024), kIdescPV,
-                          (t > 0 || g > 0 || k > 0) ? 1u : 0u);
+            for (int k = 1; k < 4; ++k) mma_pair_ss(d, da + 2 * k, db + 128 * k, kIdescPV, 1u);
             mma_commit_pair_mc(bar(kBarVEmpty + rg.slot), pmask);
             if (++rg.slot == kVStages) { rg.slot = 0; rg.phase ^= 1u; }
           }
@@ -609,19 +608,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         rescale = true;
       }
       const float mref = (m_used == -INFINITY) ? 0.0f : m_used;
-      // probabilities (p = 2^(s * scale * log2e - m)), row sum, bf16 pack
+      // probabilities (p = 2^(s * scale * log2e - m)), row sum, bf16 pack; the
+      // scaling and the sums run on pairs (packed f32x2 FMA and add: the same
+      // correctly rounded operations, half the instructions, which matters
+      // here because these warps share issue slots with the MMA issuers)
       uint32_t pk[32];
-      float ps0 = 0.0f, ps1 = 0.0f;
+      const float2 sl2v = make_float2(sl2, sl2), nmv = make_float2(-mref, -mref);
+      float2 ps = make_float2(0.0f, 0.0f);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float p0 = ex2_ftz(fmaf(s[2 * i], sl2, -mref));
-        const float p1 = ex2_ftz(fmaf(s[2 * i + 1], sl2, -mref));
-        ps0 += p0;
-        ps1 += p1;
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+        const float2 y = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), sl2v, nmv);
+        const float2 pp = make_float2(ex2_ftz(y.x), ex2_ftz(y.y));
+        ps = __fadd2_rn(ps, pp);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(pp.x, pp.y);
         pk[i] = *reinterpret_cast<uint32_t*>(&h2);
       }
-      lsum = lsum * alpha + (ps0 + ps1);
+      lsum = lsum * alpha + (ps.x + ps.y);
       // the P buffer and the output accumulator are free once PV(t-1) is done
       if (t > 0) {
         if (ok && !mbar_wait(bar(kBarOFull), (uint32_t)((t - 1) & 1), abort, wlim)) ok = false;
