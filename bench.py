@@ -24,6 +24,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 import numpy as np
@@ -167,6 +168,74 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+class RegionClocks:
+    """SM clock and clock-event reasons polled through NVML (about once a
+    millisecond) while the timed region runs. nvidia-smi's 200 ms period is
+    longer than a short timed region, so its samples over the whole run are
+    mostly taken outside it, with the GPU idle or lightly loaded."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, uuid: str | None):
+        self.nv = None
+        self.h = None
+        self.th = None
+        self.rows = []
+        self.done = threading.Event()
+        if uuid is None:
+            return
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.h = None
+
+    def start(self):
+        if self.h is None:
+            return
+        nv, h = self.nv, self.h
+
+        def poll():
+            while not self.done.is_set():
+                try:
+                    self.rows.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                      int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                except Exception:
+                    return
+                time.sleep(0.001)
+
+        self.th = threading.Thread(target=poll, daemon=True)
+        self.th.start()
+
+    def stop(self):
+        if self.th is None:
+            return None
+        self.done.set()
+        self.th.join(timeout=5)
+        if not self.rows:
+            return None
+        reasons = sorted({k for _, bits in self.rows for k, name in self.REASONS
+                          if bits & int(getattr(self.nv, name, 0))})
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.max_mhz,
+                "sm_min_mhz": min(r[0] for r in self.rows), "reasons": reasons, "samples": len(self.rows),
+                "source": "NVML, polled about every millisecond during the timed region"}
+
+
+def clock_record(region: dict | None, whole: dict | None) -> dict | None:
+    """The clocks key: the timed region's NVML samples when there are any,
+    else nvidia-smi's samples over the whole run; the nvidia-smi summary is
+    kept beside the first."""
+    if region is None:
+        return None if whole is None else dict(whole, source="nvidia-smi every 200 ms over the whole run")
+    return dict(region, nvidia_smi_whole_run=whole)
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -281,7 +350,7 @@ def config_dict(shape: synth.Shape, extra=None):
 # ---------------------------------------------------------------------------
 
 
-def measure_step(args, shape: synth.Shape, dev, world: int, full: bool):
+def measure_step(args, shape: synth.Shape, dev, world: int, full: bool, clock_uuid: str | None = None):
     """One workload on this GPU: the timed loop of K whole steps, the per-stage
     kernel times and (when `full`) the drafter, compaction and end-to-end
     legs. Returns a dict of results (and the host-side step for the CPU
@@ -384,6 +453,8 @@ def measure_step(args, shape: synth.Shape, dev, world: int, full: bool):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    region = RegionClocks(clock_uuid)
+    region.start()
     t_start.record(stream)
     for k in range(args.steps):
         if graphs is not None:
@@ -392,6 +463,7 @@ def measure_step(args, shape: synth.Shape, dev, world: int, full: bool):
             step(sets[k % n_sets])
     t_end.record(stream)
     torch.cuda.synchronize()
+    region_clocks = region.stop()
     if world > 1:
         dist.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
@@ -422,6 +494,7 @@ def measure_step(args, shape: synth.Shape, dev, world: int, full: bool):
     accept_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     acc_len = acc["acc_len"].cpu().numpy().astype(np.int64)
     res = {"shape": shape, "x": x, "logits_h": logits_h, "t_host": t_host, "n_sets": n_sets, "set_bytes": set_bytes,
+           "region_clocks": region_clocks,
            "elapsed_ms": max_over_ranks(elapsed_ms, dev), "nodes": n_nodes_total,
            "flops": attn_flops(shape, x.cache_len, t_host["depth"], t_host["n_nodes"]),
            "acc_bytes": float(n_nodes_total) * shape.V * (2 if bf else 4),
@@ -612,7 +685,7 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
     except Exception:
         uuid = None
     sampler = ClockSampler(uuid) if rank == 0 else ClockSampler(None)
-    res = measure_step(args, shape, dev, world, full=not args.sweep)
+    res = measure_step(args, shape, dev, world, full=not args.sweep, clock_uuid=uuid if rank == 0 else None)
     clocks = sampler.stop()
     extra = {}
     if not args.sweep:
@@ -651,7 +724,7 @@ def run_ours(args, shape: synth.Shape, rank: int, world: int, local_rank: int):
         "tokens_per_step": int((acc_len + 1).sum()),
         "attn_gflop_per_step": res["flops"] / 1e9,
         "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks,
+        "clocks": clock_record(res["region_clocks"], clocks),
         "timed_loop": "cuda-graph replays of the step" if res["graphs"] else "plain library calls",
     }
     if args.sweep:
