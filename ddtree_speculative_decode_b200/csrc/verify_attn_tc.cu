@@ -26,10 +26,11 @@
 //    in flight at any time. Re-streaming the Q chunk with every key chunk
 //    instead (a fourth of the bytes every tile moves from L2) measured 3 %
 //    slower on the long-context workload.
-//  * Two issuing threads because every mbarrier wait in an issuing thread
+//  * Three issuing threads because every mbarrier wait in an issuing thread
 //    stalls the tensor pipe for about as long as two MMAs (its issue queue
-//    is shallow); with QK and PV on separate threads and separate rings, one
-//    thread's waits hide behind the other's MMAs.
+//    is shallow): QK on one, and PV on one per 256-column output block (the
+//    two blocks are separate accumulators, each fed by the V ring's slots of
+//    one parity), so one thread's waits hide behind the others' MMAs.
 //  * Online softmax in the base-2 domain; the running max is only moved (and
 //    the TMEM output rescaled) when it grows by more than 8, so P <= 256.
 //    P is rounded to bf16 into shared memory (K-major, 128-byte swizzle) and
@@ -69,7 +70,8 @@ constexpr int kBoxBytes = 8192;
 constexpr int kPBytes = 4 * kBoxBytes;        // 64 rows x 256 keys bf16
 constexpr int kMaxW = 8;                      // mask words per row (N <= 256)
 constexpr int kSoftmaxWarps = 8;               // warps 4..11, two per SM sub-partition
-constexpr int kThreads = 32 * (4 + kSoftmaxWarps);
+constexpr int kPV1Warp = 4 + kSoftmaxWarps;           // warp 12: the second P.V issuer
+constexpr int kThreads = 32 * (5 + kSoftmaxWarps);
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 // shared memory map (bytes from the 1024-aligned base)
@@ -112,6 +114,7 @@ constexpr int kSmemAlloc = kSmemBytes + 1024;           // slack for 1024 alignm
 static_assert(kNumBars * 8 <= 256, "barrier area");
 static_assert(kKStages % kKGroup == 0, "QK stages are released in whole groups");
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
+static_assert(kVStages % 2 == 0, "each P.V issuer owns the ring slots of one parity");
 
 // epilogue staging (reuses the rings once the last MMA has completed): the
 // CTA's 64 rows x 512 dims as 128-byte-wide boxes of 64 rows, 128B-swizzled,
@@ -340,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(kBarSEmpty + 0), 2 * kSoftmaxWarps);
     mbar_init(bar(kBarSEmpty + 1), 2 * kSoftmaxWarps);
     mbar_init(bar(kBarPFull), 2 * kSoftmaxWarps);
-    mbar_init(bar(kBarOFull), 1);
+    mbar_init(bar(kBarOFull), 2);
     for (int c = 0; c < 4; ++c) mbar_init(bar(kBarEpi + c), 1);
     mbar_init(bar(kBarXReady), kSoftmaxWarps);
     mbar_init(bar(kBarQFull), 1);
@@ -372,8 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t wlim = p.wait_ns;
 
   // one ring of 16 KB stages per operand stream, each with its own producer
-  // thread and its own MMA-issuing thread: while one issuer waits on a
-  // barrier, the other keeps the tensor pipe fed
+  // thread and its own MMA-issuing threads: while one issuer waits on a
+  // barrier, the others keep the tensor pipe fed
   struct Ring {
     int slot = 0;
     uint32_t phase = 0;
@@ -461,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
     }
-  } else if ((warp == 1 || warp == 3) && lane == 0 && leader) {
+  } else if ((warp == 1 || warp == 3 || warp == kPV1Warp) && lane == 0 && leader) {
     // ============================================================ MMA issuers
     bool ok = true;
     Ring rg;
@@ -494,30 +497,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) mma_commit_pair_mc(bar(kBarSFull + sb), pmask);
       }
     } else {
-      // P.V into the two 128-column output blocks
+      // P.V into one of the two 128-column output blocks (warp 3: block 0,
+      // the second P.V issuer: block 1). The V producer alternates the
+      // blocks, so block j's stages are the ring slots of parity j.
+      const int j = warp == 3 ? 0 : 1;
+      const uint32_t d = tmem + (j ? kColO1 : kColO0);
+      rg.slot = j;
       for (int t = 0; t < u.T && ok; ++t) {
         if (!mbar_wait(bar(kBarPFull), (uint32_t)(t & 1), abort, wlim)) { ok = false; break; }
         tc_fence_after();
         if (t >= u.tt) unit_tree(p, u);  // live key groups of a tile that reaches tree keys
         const int ng = live_groups(u, t);
-        for (int g = 0; g < ng && ok; ++g) {
+        for (int g = 0; g < ng; ++g) {
           const uint64_t da = smem_desc_sw128(sbase + kOffP + g * kBoxBytes, 16, 1024);
-          for (int j = 0; j < 2; ++j) {
-            if (!mbar_wait(bar(kBarVFull + rg.slot), rg.phase, abort, wlim)) { ok = false; break; }
-            // +2048 bytes per K step (16 keys) is +128 in the address field
-            const uint64_t db = smem_desc_sw128(sbase + kOffVRing + rg.slot * kVStageBytes, kBoxBytes, 1024);
-            const uint32_t d = tmem + (j ? kColO1 : kColO0);
-            mma_pair_ss(d, da, db, kIdescPV, (t > 0 || g > 0) ? 1u : 0u);
+          if (!mbar_wait(bar(kBarVFull + rg.slot), rg.phase, abort, wlim)) { ok = false; break; }
+          // +2048 bytes per K step (16 keys) is +128 in the address field
+          const uint64_t db = smem_desc_sw128(sbase + kOffVRing + rg.slot * kVStageBytes, kBoxBytes, 1024);
+          mma_pair_ss(d, da, db, kIdescPV, (t > 0 || g > 0) ? 1u : 0u);
 #pragma unroll
-            for (int k = 1; k < 4; ++k) mma_pair_ss(d, da + 2 * k, db + 128 * k, kIdescPV, 1u);
-            mma_commit_pair_mc(bar(kBarVEmpty + rg.slot), pmask);
-            if (++rg.slot == kVStages) { rg.slot = 0; rg.phase ^= 1u; }
-          }
+          for (int k = 1; k < 4; ++k) mma_pair_ss(d, da + 2 * k, db + 128 * k, kIdescPV, 1u);
+          mma_commit_pair_mc(bar(kBarVEmpty + rg.slot), pmask);
+          rg.slot += 2;
+          if (rg.slot >= kVStages) { rg.slot -= kVStages; rg.phase ^= 1u; }
         }
         if (ok) mma_commit_pair_mc(bar(kBarOFull), pmask);
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 4 + kSoftmaxWarps) {
     // ============================================================ softmax
     // warp w reads TMEM lane quarter w % 4; lane l holds one row (l % 64) and
     // one half of the tile's keys / output dims (l / 64); the two warps of a
