@@ -73,11 +73,11 @@ def replica_throughput(nodes_per_step: int, steps: int, world: int, elapsed_ms: 
 PROFILED_ATTN_DRAM = {
     # ncu --set full, one launch of the long-context workload's attention
     # (bench.py --steps 3 --warmup 3 --no-cpu-baseline --e2e-steps 3 --layers 1
-    # --extra=, -k regex:attn_tc -s 2 -c 1): dram__bytes_read.sum 297.342720 MB
-    # + dram__bytes_write.sum 80.217344 MB
+    # --extra=, -k regex:attn_tc -s 2 -c 1): dram__bytes_read.sum 317.055488 MB
+    # + dram__bytes_write.sum 81.800960 MB
     "kimi-4req-L32768-N128": {
-        "bytes": 377560064.0,
-        "sources": {"verify_attn_tc.cu": "c381e4e3da932c4f7d14928f9983dade1c276d53584a2b518d06d2b4f3fdcda1",
+        "bytes": 398856448.0,
+        "sources": {"verify_attn_tc.cu": "d7cd1b6e74e4b64c5a98ba4b00855840b7f11254464a9dc0bb6f3fbd65277c7a",
                     "sm100_ptx.cuh": "742a701fc79bc45f49ed1e6b9494f89da884dc911c9353fdb120e72dbac572a6"}},
 }
 
