@@ -190,11 +190,18 @@ class RegionClocks:
         try:
             import pynvml
             pynvml.nvmlInit()
-            self.nv = pynvml
+        except Exception:
+            return
+        self.nv = pynvml
+        try:
             self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
             self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
         except Exception:
             self.h = None
+            try:
+                pynvml.nvmlShutdown()
+            except Exception:
+                pass
 
     def start(self):
         if self.h is None:
@@ -218,6 +225,10 @@ class RegionClocks:
             return None
         self.done.set()
         self.th.join(timeout=5)
+        try:
+            self.nv.nvmlShutdown()  # balances the nvmlInit of this sampler
+        except Exception:
+            pass
         if not self.rows:
             return None
         reasons = sorted({k for _, bits in self.rows for k, name in self.REASONS

@@ -28,8 +28,17 @@ def _fake_nvml(clocks, reasons):
     m.nvmlClocksEventReasonHwSlowdown = 0x8
     m.nvmlClocksEventReasonSwThermalSlowdown = 0x20
     m.nvmlClocksEventReasonHwThermalSlowdown = 0x40
-    state = {"i": 0}
-    m.nvmlInit = lambda: None
+    state = {"i": 0, "open": 0}
+
+    def init():
+        state["open"] += 1
+
+    def shutdown():
+        state["open"] -= 1
+
+    m.nvmlInit = init
+    m.nvmlShutdown = shutdown
+    m.state = state
     m.nvmlDeviceGetHandleByUUID = lambda uuid: ("h", uuid)
     m.nvmlDeviceGetMaxClockInfo = lambda h, kind: 1965
 
@@ -64,6 +73,7 @@ def test_region_clocks_fake_nvml(monkeypatch, reasons, expect):
     assert 1500 <= r["sm_min_mhz"] <= r["sm_mhz"] <= 1540
     assert r["reasons"] == expect
     assert "timed region" in r["source"]
+    assert sys.modules["pynvml"].state["open"] == 0  # every nvmlInit is balanced
 
 
 def test_region_clocks_without_nvml(monkeypatch):
