@@ -195,7 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // issuing thread costs the tensor pipe about two MMAs, and the other
     // thread's queued MMAs cover it; the parts' accumulators are disjoint
     const uint32_t idesc = idesc_bf16_f32(256, p.npart, false, false);
-    const int j0 = p.parts == 2 ? (warp == 6 ? 1 : 0) : 0, j1 = p.parts == 2 ? j0 + 1 : p.parts;
+    const int j = warp == 6 ? 1 : 0;  // the N part this thread issues
+    const uint32_t boff = (uint32_t)(kABytes + j * p.nh * 128);  // its hidden box in a stage
     int slot = 0;
     uint32_t phase = 0;
     bool ok = true;
@@ -204,6 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int buf = lt % p.nbuf;
       if (!mbar_wait(bar(kBarAccEmpty + buf), (uint32_t)((lt / p.nbuf) & 1) ^ 1u, abort, wlim)) break;
       tc_fence_after();
+      const uint32_t d = tmem + (uint32_t)((buf * p.parts + j) * 256);
       for (int kb = 0; kb < p.nkb; ++kb) {
         if (!mbar_wait(bar(kBarFull + slot), phase, abort, wlim)) {
           ok = false;
@@ -211,14 +213,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const uint32_t a0 = sbase + (uint32_t)(slot * p.stage_bytes);
         // descriptors once per stage: +32 bytes per K step is +2 in the address field
-        const uint64_t da = smem_desc_sw128(a0, 16, 1024);
-        for (int j = j0; j < j1; ++j) {
-          const uint64_t db = smem_desc_sw128(a0 + kABytes + (uint32_t)(j * p.nh * 128), 16, 1024);
-          const uint32_t d = tmem + (uint32_t)((buf * p.parts + j) * 256);
-          mma_pair_ss(d, da, db, idesc, kb != 0 ? 1u : 0u);
+        const uint64_t da = smem_desc_sw128(a0, 16, 1024), db = smem_desc_sw128(a0 + boff, 16, 1024);
+        mma_pair_ss(d, da, db, idesc, kb != 0 ? 1u : 0u);
 #pragma unroll
-          for (int k = 1; k < 4; ++k) mma_pair_ss(d, da + 2 * k, db + 2 * k, idesc, 1u);
-        }
+        for (int k = 1; k < 4; ++k) mma_pair_ss(d, da + 2 * k, db + 2 * k, idesc, 1u);
         mma_commit_pair_mc(bar(kBarEmpty + slot), (uint16_t)0x3u);
         if (++slot == p.stages) {
           slot = 0;
